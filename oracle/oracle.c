@@ -1,0 +1,383 @@
+/*
+ * oracle.c -- plain, slow, CPU oracle for entropy-coded bf16 weights.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * CPU-baseline leg of the benchmark may load this file's library.  The
+ * product (libdfw and its Python binding) never links, imports or calls it,
+ * and it shares no code, header, table or constant with the product.
+ *
+ * What the method computes (sources):
+ *   - "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
+ *     Inference via Dynamic-Length Float" (DFloat11), abstract: bf16 weights
+ *     have low-entropy exponents; entropy coding gives each value a
+ *     frequency-based variable-length code; decoding is bit-for-bit exact;
+ *     the GPU decoder coordinates thread read/write positions with small
+ *     auxiliary arrays.
+ *   - "From a Lossless (~1.5:1) Compression Algorithm for Llama2 7B Weights
+ *     ...", abstract: lossless ~1.5:1 on Llama2-7B bf16 weights.
+ *   - The LazyWeights write-up (bedrocknews.com, arXiv 2611.17108v1) and the
+ *     Huff-LLM abstract: the entropy code is Huffman.
+ * The pages leave the exact format open; the readings taken here are:
+ *   R1 exponent = bits 14..7 of the bf16 pattern, raw byte = sign<<7 | mant7;
+ *   R2 code lengths = optimal length-limited prefix code (package-merge,
+ *      Larmore & Hirschberg 1990) with cap `cap` (<= 32), leaves ordered by
+ *      (count, symbol), and on equal weight a leaf is merged before a package;
+ *   R3 one distinct exponent -> length 0, empty bitstream;
+ *   R4 canonical codewords in (length, symbol) order (RFC 1951 sec. 3.2.2);
+ *   R5 codewords written MSB-first, first bit into bit 7 of byte 0; the byte
+ *      stream is zero-padded to a multiple of 64 bytes plus 16 guard bytes;
+ *   R6 aux: for a window of W bytes starting at bit 8*W*t, gap[t] is the
+ *      distance from the window start to the first code start at or after
+ *      it (or to total_bits when no code starts there); for a tile of T
+ *      windows, out_start[b] counts the code starts before bit 8*W*T*b, and
+ *      out_start[n_tiles] = n.
+ * Parity: every function here is pinned by tests in tests/test_oracle_*.py
+ * (round trip, Kraft equality, entropy bounds, brute-force optimality,
+ * closed forms, independent recounts).  The tie rule of R2 is this
+ * library's reading, pinned only by a hand-worked tie case.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_EINVAL 1
+#define OR_ECAP 2
+#define OR_ENOMEM 3
+#define OR_ECORRUPT 4
+
+/* ---- R1: split each bf16 pattern into exponent and sign+mantissa bytes. */
+void oracle_split(const uint16_t *u, uint64_t n, uint8_t *e, uint8_t *m)
+{
+    for (uint64_t i = 0; i < n; i++) {
+        uint16_t x = u[i];
+        e[i] = (uint8_t)((x >> 7) & 0xFFu);
+        m[i] = (uint8_t)(((x >> 8) & 0x80u) | (x & 0x7Fu));
+    }
+}
+
+/* Inverse of the split: sign from bit 7 of m, exponent e, mantissa m&0x7F. */
+uint16_t oracle_join(uint8_t e, uint8_t m)
+{
+    return (uint16_t)(((uint32_t)(m & 0x80u) << 8) | ((uint32_t)e << 7) | (m & 0x7Fu));
+}
+
+/* ---- frequency count that drives the code ("based on frequency"). */
+void oracle_histogram(const uint8_t *e, uint64_t n, uint64_t hist[256])
+{
+    for (int s = 0; s < 256; s++)
+        hist[s] = 0;
+    for (uint64_t i = 0; i < n; i++)
+        hist[e[i]]++;
+}
+
+/* ---- R2: package-merge.  Each list item carries how often every symbol
+ * occurs inside it, so a symbol's code length is read off directly as the
+ * number of times it occurs among the selected items. */
+typedef struct {
+    uint64_t weight;
+    int leaf;
+    uint16_t mult[256];
+} pm_item;
+
+int oracle_code_lengths(const uint64_t hist[256], int cap, uint8_t len[256])
+{
+    memset(len, 0, 256);
+    if (cap < 1 || cap > 32)
+        return OR_EINVAL;
+    int k = 0;
+    for (int s = 0; s < 256; s++)
+        if (hist[s] > 0)
+            k++;
+    if (k <= 1)
+        return OR_OK; /* R3: zero or one symbol needs no bits */
+    if (cap < 9 && (1 << cap) < k)
+        return OR_ECAP; /* no prefix code of k words fits in cap bits */
+
+    pm_item *leaves = (pm_item *)calloc((size_t)k, sizeof(pm_item));
+    pm_item *cur = (pm_item *)calloc((size_t)(2 * k), sizeof(pm_item));
+    pm_item *nxt = (pm_item *)calloc((size_t)(2 * k), sizeof(pm_item));
+    pm_item *pkg = (pm_item *)calloc((size_t)k, sizeof(pm_item));
+    if (!leaves || !cur || !nxt || !pkg) {
+        free(leaves); free(cur); free(nxt); free(pkg);
+        return OR_ENOMEM;
+    }
+    /* leaves in symbol order, then a stable insertion sort by count, which
+     * gives (count, symbol) order */
+    int nl = 0;
+    for (int s = 0; s < 256; s++) {
+        if (hist[s] == 0)
+            continue;
+        leaves[nl].weight = hist[s];
+        leaves[nl].leaf = 1;
+        leaves[nl].mult[s] = 1;
+        nl++;
+    }
+    for (int i = 1; i < k; i++) {
+        pm_item tmp = leaves[i];
+        int j = i - 1;
+        while (j >= 0 && leaves[j].weight > tmp.weight) {
+            leaves[j + 1] = leaves[j];
+            j--;
+        }
+        leaves[j + 1] = tmp;
+    }
+
+    int ncur = k;
+    memcpy(cur, leaves, (size_t)k * sizeof(pm_item));
+    for (int iter = 1; iter <= cap - 1; iter++) {
+        /* package adjacent pairs; an unpaired last item is dropped */
+        int np = ncur / 2;
+        for (int i = 0; i < np; i++) {
+            pkg[i].weight = cur[2 * i].weight + cur[2 * i + 1].weight;
+            pkg[i].leaf = 0;
+            for (int s = 0; s < 256; s++)
+                pkg[i].mult[s] = (uint16_t)(cur[2 * i].mult[s] + cur[2 * i + 1].mult[s]);
+        }
+        /* merge packages with the leaves; a leaf goes first on equal weight */
+        int i = 0, j = 0, o = 0;
+        while (i < k || j < np) {
+            if (j >= np || (i < k && leaves[i].weight <= pkg[j].weight))
+                nxt[o++] = leaves[i++];
+            else
+                nxt[o++] = pkg[j++];
+        }
+        pm_item *t = cur;
+        cur = nxt;
+        nxt = t;
+        ncur = o;
+    }
+    /* the 2k-2 cheapest items of the final list */
+    for (int i = 0; i < 2 * k - 2; i++)
+        for (int s = 0; s < 256; s++)
+            len[s] = (uint8_t)(len[s] + cur[i].mult[s]);
+
+    free(leaves); free(cur); free(nxt); free(pkg);
+    return OR_OK;
+}
+
+/* ---- R4: canonical codewords, RFC 1951 sec. 3.2.2. */
+void oracle_canonical_codes(const uint8_t len[256], uint32_t code[256])
+{
+    uint64_t bl_count[34];
+    uint64_t next_code[34];
+    for (int b = 0; b < 34; b++)
+        bl_count[b] = next_code[b] = 0;
+    for (int s = 0; s < 256; s++)
+        if (len[s] > 0)
+            bl_count[len[s]]++;
+    uint64_t c = 0;
+    for (int bits = 1; bits <= 32; bits++) {
+        c = (c + bl_count[bits - 1]) << 1;
+        next_code[bits] = c;
+    }
+    for (int s = 0; s < 256; s++) {
+        code[s] = 0;
+        if (len[s] > 0)
+            code[s] = (uint32_t)next_code[len[s]]++;
+    }
+}
+
+/* ---- R5: padded stream length for a given number of coded bits. */
+uint64_t oracle_stream_bytes(uint64_t total_bits)
+{
+    uint64_t raw = (total_bits + 7) / 8;
+    return (raw + 63) / 64 * 64 + 16;
+}
+
+/* ---- R5: MSB-first packing, one bit at a time. */
+int oracle_pack(const uint8_t *e, uint64_t n, const uint8_t len[256], const uint32_t code[256],
+                uint8_t *stream, uint64_t stream_cap, uint64_t *total_bits_out)
+{
+    uint64_t tb = 0;
+    for (uint64_t i = 0; i < n; i++)
+        tb += len[e[i]];
+    uint64_t need = oracle_stream_bytes(tb);
+    if (stream_cap < need)
+        return OR_ENOMEM;
+    memset(stream, 0, (size_t)need);
+    uint64_t pos = 0;
+    for (uint64_t i = 0; i < n; i++) {
+        int l = len[e[i]];
+        uint32_t c = code[e[i]];
+        for (int b = l - 1; b >= 0; b--) {
+            if ((c >> b) & 1u)
+                stream[pos >> 3] |= (uint8_t)(0x80u >> (pos & 7));
+            pos++;
+        }
+    }
+    *total_bits_out = tb;
+    return OR_OK;
+}
+
+/* Whole encoder: split, histogram, lengths, codes, pack. */
+int oracle_encode(const uint16_t *u, uint64_t n, int cap, uint8_t *stream, uint64_t stream_cap,
+                  uint8_t *mant, uint8_t len_out[256], uint64_t *total_bits_out)
+{
+    uint8_t *e = (uint8_t *)malloc(n ? (size_t)n : 1);
+    if (!e)
+        return OR_ENOMEM;
+    oracle_split(u, n, e, mant);
+    uint64_t hist[256];
+    oracle_histogram(e, n, hist);
+    int rc = oracle_code_lengths(hist, cap, len_out);
+    if (rc != OR_OK) {
+        free(e);
+        return rc;
+    }
+    uint32_t code[256];
+    oracle_canonical_codes(len_out, code);
+    rc = oracle_pack(e, n, len_out, code, stream, stream_cap, total_bits_out);
+    free(e);
+    return rc;
+}
+
+/* ---- textbook canonical decoder state: per length, the first codeword,
+ * the number of codewords, and where its symbols start in the list of
+ * symbols sorted by (length, symbol). */
+typedef struct {
+    uint64_t first[33];
+    uint64_t count[33];
+    uint64_t base[33];
+    uint8_t sorted[256];
+    int k;
+    int single;
+} canon_dec;
+
+static void canon_init(const uint8_t len[256], canon_dec *d)
+{
+    memset(d, 0, sizeof(*d));
+    d->single = -1;
+    for (int s = 0; s < 256; s++)
+        if (len[s] > 0)
+            d->count[len[s]]++;
+    uint64_t c = 0, idx = 0;
+    for (int l = 1; l <= 32; l++) {
+        c = (c + d->count[l - 1]) << 1;
+        d->first[l] = c;
+        d->base[l] = idx;
+        for (int s = 0; s < 256; s++)
+            if (len[s] == l)
+                d->sorted[idx++] = (uint8_t)s;
+    }
+    d->k = (int)idx;
+}
+
+/* Reads one codeword bit by bit starting at *pos; returns the symbol or -1. */
+static int canon_read(const canon_dec *d, const uint8_t *stream, uint64_t total_bits, uint64_t *pos)
+{
+    uint64_t code = 0;
+    for (int l = 1; l <= 32; l++) {
+        if (*pos >= total_bits)
+            return -1;
+        uint64_t bit = (stream[*pos >> 3] >> (7 - (*pos & 7))) & 1u;
+        code = (code << 1) | bit;
+        (*pos)++;
+        if (d->count[l] > 0 && code >= d->first[l] && code - d->first[l] < d->count[l])
+            return d->sorted[d->base[l] + (code - d->first[l])];
+    }
+    return -1;
+}
+
+/* ---- bit-serial decoder: emits exactly n weights; the coded bits must be
+ * used up exactly.  single_symbol is the exponent when the table has one
+ * symbol (R3) and is ignored otherwise. */
+int oracle_decode(const uint8_t *stream, uint64_t total_bits, const uint8_t len[256],
+                  int single_symbol, const uint8_t *mant, uint64_t n, uint16_t *out)
+{
+    canon_dec d;
+    canon_init(len, &d);
+    if (d.k == 0) {
+        if (total_bits != 0)
+            return OR_ECORRUPT;
+        if (n > 0 && (single_symbol < 0 || single_symbol > 255))
+            return OR_EINVAL;
+        for (uint64_t i = 0; i < n; i++)
+            out[i] = oracle_join((uint8_t)single_symbol, mant[i]);
+        return OR_OK;
+    }
+    uint64_t pos = 0;
+    for (uint64_t i = 0; i < n; i++) {
+        int s = canon_read(&d, stream, total_bits, &pos);
+        if (s < 0)
+            return OR_ECORRUPT;
+        out[i] = oracle_join((uint8_t)s, mant[i]);
+    }
+    return pos == total_bits ? OR_OK : OR_ECORRUPT;
+}
+
+/* Decodes the exponent symbols only, from bit `start_bit`, for `count`
+ * symbols (used to check a sampled tile of a large stream). */
+int oracle_decode_symbols(const uint8_t *stream, uint64_t total_bits, const uint8_t len[256],
+                          uint64_t start_bit, uint64_t count, uint8_t *sym_out)
+{
+    canon_dec d;
+    canon_init(len, &d);
+    if (d.k == 0)
+        return count == 0 ? OR_OK : OR_EINVAL;
+    uint64_t pos = start_bit;
+    for (uint64_t i = 0; i < count; i++) {
+        int s = canon_read(&d, stream, total_bits, &pos);
+        if (s < 0)
+            return OR_ECORRUPT;
+        sym_out[i] = (uint8_t)s;
+    }
+    return OR_OK;
+}
+
+/* ---- R6: auxiliary arrays, from the list of code start positions. */
+uint64_t oracle_n_windows(uint64_t total_bits, uint64_t W)
+{
+    return (total_bits + 8 * W - 1) / (8 * W);
+}
+
+int oracle_aux(const uint8_t *stream, uint64_t total_bits, const uint8_t len[256], uint64_t n,
+               uint64_t W, uint64_t T, uint8_t *gap, uint64_t *out_start)
+{
+    if (W == 0 || T == 0)
+        return OR_EINVAL;
+    uint64_t nwin = oracle_n_windows(total_bits, W);
+    uint64_t ntiles = (nwin + T - 1) / T;
+    uint64_t *starts = (uint64_t *)malloc((size_t)(n + 1) * sizeof(uint64_t));
+    if (!starts)
+        return OR_ENOMEM;
+    uint64_t nstarts = 0;
+    if (total_bits > 0) {
+        canon_dec d;
+        canon_init(len, &d);
+        uint64_t pos = 0;
+        while (pos < total_bits) {
+            if (nstarts >= n) {
+                free(starts);
+                return OR_ECORRUPT;
+            }
+            starts[nstarts++] = pos;
+            if (canon_read(&d, stream, total_bits, &pos) < 0) {
+                free(starts);
+                return OR_ECORRUPT;
+            }
+        }
+        if (nstarts != n) {
+            free(starts);
+            return OR_ECORRUPT;
+        }
+    }
+    uint64_t j = 0;
+    for (uint64_t t = 0; t < nwin; t++) {
+        uint64_t wstart = 8 * W * t;
+        while (j < nstarts && starts[j] < wstart)
+            j++;
+        uint64_t s = j < nstarts ? starts[j] : total_bits;
+        gap[t] = (uint8_t)(s - wstart);
+    }
+    j = 0;
+    for (uint64_t b = 0; b < ntiles; b++) {
+        uint64_t tstart = 8 * W * T * b;
+        while (j < nstarts && starts[j] < tstart)
+            j++;
+        out_start[b] = j;
+    }
+    out_start[ntiles] = n;
+    free(starts);
+    return OR_OK;
+}
