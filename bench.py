@@ -1,0 +1,453 @@
+#!/usr/bin/env python
+"""Benchmark: bit-exact GPU decode of entropy-coded bf16 weights.
+
+One step = decoding every code-table scope of the workload (for the default
+Llama-3-8B-shaped model: embedding, 32 transformer blocks, lm_head; 34
+launches of the decode kernel, one per block, into one reused scratch
+buffer).  Inputs are resident in HBM when the timed region starts.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload c5]
+  torchrun --nproc-per-node N bench.py --gpus N ...   (one replica per rank)
+  python bench.py --impl reference ...                (the CPU oracle, timed)
+
+Prints one JSON line on rank 0.  Multi-GPU runs are weak scaling: every rank
+decodes its own resident copy of the model; there is no data-path
+collective; time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import ctypes
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "decoded bf16 weights/sec & effective GB/s as % of HBM roofline; compression ratio"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["lossless_entropy_coded_canonical_b200/csrc/dfw_decode.cu",
+                  "lossless_entropy_coded_canonical_b200/csrc/dfw_internal.h"]
+
+
+# ------------------------------------------------------------------ helpers
+
+def workload_blocks(name: str):
+    if name == "c5":
+        return workloads.c5(), "llama3-8b-shaped model: embed + 32 blocks + lm_head, 34 code tables, N(0,0.02)"
+    table = {"c1": workloads.c1(), "c2": workloads.c2(), "c3": workloads.c3(), "c4a": workloads.c4("a"),
+             "c4b": workloads.c4("b"), "c4bp": workloads.c4("bp"), "c4c": workloads.c4("c")}
+    return [table[name]], f"{name} ({table[name].numel} weights)"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def committed_traffic(workload: str):
+    """Per-weight DRAM traffic of the decode kernel from a committed ncu
+    summary, used only if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", f"decode_tiles_{workload}_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    kv = {}
+    for line in open(p):
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+        return None
+    try:
+        return float(kv["dram_bytes_per_weight"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        try:
+            p = torch.cuda.get_device_properties(device)
+            self.gpu_id = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            self.gpu_id = str(device)
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def max_over_ranks(value: float, group=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    dev = "cuda" if dist.get_backend(group) == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ setup
+
+def prepare(blocks, device, window, tile, threads):
+    """Generates each block on the GPU, encodes and plans it on the host,
+    uploads it; returns the device-resident blocks and host copies (pinned)."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    host_threads = max(1, (os.cpu_count() or 8))
+    enc_threads = threads or max(1, host_threads // 2)
+    pool = cf.ThreadPoolExecutor(max_workers=min(8, host_threads))
+
+    def host_side(i, tensors):
+        enc = dfw.encode_multi(tensors, 32, n_threads=enc_threads, pin=True)
+        pl = dfw.plan(enc, window, tile, pin=True)
+        return i, enc, pl
+
+    futs = []
+    for i, b in enumerate(blocks):
+        ts = [t.cpu() for t in workloads.generate_block(b, device)]
+        futs.append(pool.submit(host_side, i, ts))
+        while sum(not f.done() for f in futs) >= 8:
+            time.sleep(0.01)
+    res = [None] * len(blocks)
+    for f in futs:
+        i, enc, pl = f.result()
+        res[i] = (enc, pl)
+    pool.shutdown()
+    devs = [dfw.DeviceCompressed.upload(enc, pl, device) for enc, pl in res]
+    torch.cuda.synchronize(device)
+    return devs, res
+
+
+def verify(blocks, devs, scratch, device):
+    """Decodes each block once more and compares with the regenerated input."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    for b, d in zip(blocks, devs):
+        _, views = dfw.decode_block(d, scratch)
+        dfw.check()
+        for v, t in zip(views, workloads.generate_block(b, device)):
+            if not torch.equal(v.view(torch.int16), t.view(torch.int16)):
+                return False
+    return True
+
+
+# ------------------------------------------------------------------ timed arms
+
+def run_device(devs, scratch, steps, warmup, stream):
+    import lossless_entropy_coded_canonical_b200 as dfw
+    for _ in range(warmup):
+        for d in devs:
+            dfw.decode_block(d, scratch, stream=stream)
+    dfw.check(stream)
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in devs]
+          for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for s in range(steps):
+        for j, d in enumerate(devs):
+            ev[s][j][0].record(stream)
+            dfw.decode_block(d, scratch, stream=stream)
+            ev[s][j][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = t0.elapsed_time(t1)
+    per_launch = [[a.elapsed_time(b) for a, b in row] for row in ev]
+    status = dfw.check_status(stream)
+    return total_ms, per_launch, status
+
+
+def run_e2e(results, devs, device, steps, stream):
+    """Same metric through the public API from pinned host buffers: per block
+    H2D of its compressed form, decode, D2H of the decoded weights; copies run
+    on their own streams, double-buffered so they overlap the decode."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    nmax = max(d.n for d in devs)
+    h2d_s, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    slots = []
+    for _ in range(2):
+        slots.append({
+            "stream": torch.empty(max(int(e.table.stream_bytes) for e, _ in results), dtype=torch.uint8, device=device),
+            "mant": torch.empty(max(e.mant.numel() for e, _ in results), dtype=torch.uint8, device=device),
+            "gap": torch.empty(max(p.gap.numel() for _, p in results) + 1, dtype=torch.uint8, device=device),
+            "out_start": torch.empty(max(p.out_start.numel() for _, p in results), dtype=torch.int64, device=device),
+            "lut": torch.empty(max(p.lut.numel() for _, p in results), dtype=torch.int32, device=device),
+            "scratch": torch.empty(nmax, dtype=torch.bfloat16, device=device),
+            "host_out": torch.empty(nmax, dtype=torch.bfloat16, pin_memory=True),
+            "loaded": torch.cuda.Event(), "decoded": torch.cuda.Event(), "drained": torch.cuda.Event(),
+        })
+    h2d = sum(int(e.table.stream_bytes) + e.mant.numel() + p.gap.numel() + 8 * p.out_start.numel()
+              + 4 * p.lut.numel() for e, p in results)
+    d2h = sum(2 * e.n for e, _ in results)
+
+    def one_step():
+        # slot i % 2 is reused by block i + 2: its H2D waits until block i's
+        # decode has read the inputs, and its decode waits until block i's
+        # D2H has read the scratch buffer
+        for i, (enc, pl) in enumerate(results):
+            sl = slots[i % 2]
+            h2d_s.wait_event(sl["decoded"])
+            with torch.cuda.stream(h2d_s):
+                sl["stream"][: enc.stream.numel()].copy_(enc.stream, non_blocking=True)
+                sl["mant"][: enc.mant.numel()].copy_(enc.mant, non_blocking=True)
+                sl["gap"][: pl.gap.numel()].copy_(pl.gap, non_blocking=True)
+                sl["out_start"][: pl.out_start.numel()].copy_(pl.out_start, non_blocking=True)
+                sl["lut"][: pl.lut.numel()].copy_(pl.lut, non_blocking=True)
+                sl["loaded"].record(h2d_s)
+            stream.wait_event(sl["loaded"])
+            stream.wait_event(sl["drained"])
+            dc = dfw.DeviceCompressed(sl["stream"], sl["mant"], sl["lut"], sl["gap"], sl["out_start"], enc.table,
+                                      pl.info, enc.tensor_offsets)
+            dfw.decode_block(dc, sl["scratch"], stream=stream)
+            sl["decoded"].record(stream)
+            d2h_s.wait_event(sl["decoded"])
+            with torch.cuda.stream(d2h_s):
+                sl["host_out"][: enc.n].copy_(sl["scratch"][: enc.n], non_blocking=True)
+                sl["drained"].record(d2h_s)
+
+    one_step()  # warm-up (allocator, first copies)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0.record(stream)
+    for _ in range(steps):
+        one_step()
+    stream.wait_stream(d2h_s)
+    stream.wait_stream(h2d_s)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    st = dfw.check_status(stream)
+    return t0.elapsed_time(t1) / steps, h2d, d2h, st
+
+
+def cpu_baseline_sample(sample_weights: int, reps: int):
+    """The oracle's bit-serial decoder, as it stands, on a prefix of the
+    workload's first transformer block (the oracle encodes it, untimed)."""
+    import oracle
+    oracle.build()
+    blk = workloads.c5()[1]
+    parts, got = [], 0
+    for t in blk.tensors:
+        take = min(t.numel, sample_weights - got)
+        if take <= 0:
+            break
+        spec = workloads.TensorSpec(t.name, t.numel, t.kind, t.seed, t.std)
+        parts.append(workloads.as_u16_numpy(workloads.generate(spec, "cpu"))[:take])
+        got += take
+    u = np.concatenate(parts)
+    enc = oracle.encode(u)
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        out = oracle.decode(enc)
+        times.append(time.perf_counter() - t0)
+    assert np.array_equal(out, u)
+    return u.size, statistics.median(times), enc
+
+
+# ------------------------------------------------------------------ main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dfw", choices=["dfw", "reference"])
+    ap.add_argument("--workload", default="c5")
+    ap.add_argument("--window", type=int, default=8)
+    ap.add_argument("--tile", type=int, default=256)
+    ap.add_argument("--threads", type=int, default=0)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    blocks, wdesc = workload_blocks(args.workload)
+    n_total = sum(b.numel for b in blocks)
+
+    if args.impl == "reference":
+        return reference_arm(args, rank, world, n_total, wdesc)
+
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", device_id=torch.device("cuda", local),
+                                timeout=__import__("datetime").timedelta(seconds=600))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import lossless_entropy_coded_canonical_b200 as dfw
+    dfw.lib()
+    dfw.check()
+
+    devs, results = prepare(blocks, device, args.window, args.tile, args.threads)
+    nmax = max(d.n for d in devs)
+    scratch = torch.empty(nmax, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+    comp = sum(d.compressed_bytes(with_aux=True) for d in devs)
+    comp_noaux = sum(d.compressed_bytes(with_aux=False) for d in devs)
+    alg_bytes = sum(d.algorithmic_bytes() for d in devs)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    total_ms, per_launch, status = run_device(devs, scratch, args.steps, args.warmup, stream)
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(total_ms / args.steps)
+    ok = status == dfw.OK and verify(blocks, devs, scratch, device)
+
+    # roofline of the decode kernel: algorithmic bytes / mean launch duration
+    launch_ms = np.array(per_launch)  # [steps, blocks]
+    mean_launch_ms = launch_ms.mean(axis=0)
+    achieved = alg_bytes / (mean_launch_ms.sum() * 1e-3) / 1e9
+    peak, peak_kind = measured_peak_hbm()
+    tpw = committed_traffic(args.workload)
+    traffic = None if tpw is None else tpw * n_total / len(devs)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h, st2 = run_e2e(results, devs, device, args.e2e_steps, stream)
+        e2e_ms = max_over_ranks(e2e_ms)
+        ok = ok and st2 == dfw.OK
+        e2e = {"value": world * n_total / (e2e_ms * 1e-3), "unit": "weights/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_s, sec, _ = cpu_baseline_sample(args.cpu_sample, 3)
+        cpu = {"value": n_s / sec, "unit": "weights/s", "cores": 1, "kind": "oracle",
+               "sample": f"bit-serial decode of the first {n_s} weights of transformer block 0 "
+                         f"(q, k, v, o, ...), median of 3, one host thread"}
+
+    value = world * n_total / (ms_step * 1e-3)
+    eff_gbs = alg_bytes / (ms_step * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": wdesc, "weights": n_total, "code_tables": len(devs),
+                   "window_bytes": args.window, "tile_windows": args.tile,
+                   "l2": "inputs larger than L2 (each step reads every block's compressed form and writes "
+                         "every block's bf16; no reuse between steps)",
+                   "parallelism": f"replica{world}" if world > 1 else "single GPU"},
+        "effective_gbs": eff_gbs, "hbm_frac": eff_gbs / peak,
+        "compression_ratio": 2 * n_total / comp, "compression_ratio_no_aux": 2 * n_total / comp_noaux,
+        "bits_per_weight": 8 * comp / n_total,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "peak_source": peak_kind,
+                     "kernel": "decode_tiles", "algorithmic_bytes_per_step": alg_bytes,
+                     "mean_launch_ms": float(mean_launch_ms.mean())},
+        "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": args.steps * len(devs),
+        "verified_bit_exact": bool(ok),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0 if ok else 1
+
+
+def reference_arm(args, rank, world, n_total, wdesc):
+    """The oracle as the reference arm: each step decodes a bounded sample of
+    the workload on one host core.  Rank 0 alone runs it."""
+    if rank != 0:
+        return 0
+    sample = min(args.cpu_sample // 4, 8 * 1024 * 1024)
+    n_s, _, enc = cpu_baseline_sample(sample, 1)
+    import oracle
+    for _ in range(args.warmup):
+        oracle.decode(enc)
+    steps = min(args.steps, 10)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.decode(enc)
+    sec = (time.perf_counter() - t0) / steps
+    v = n_s / sec
+    desc = f"bit-serial oracle decode of the first {n_s} weights of transformer block 0 per step, one host thread"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "weights/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": wdesc, "weights": n_total, "sample_weights": n_s},
+        "cpu_baseline": {"value": v, "unit": "weights/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,215 @@
+/*
+ * dfw.h -- C ABI of libdfw: lossless entropy-coded bf16 weights, decoded on
+ * an NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are the pages this library restates; see each call):
+ *   "70% Size, 100% Accuracy: Lossless LLM Compression for Efficient GPU
+ *   Inference via Dynamic-Length Float" (DFloat11), abstract -- bf16 weights
+ *   carry low-entropy exponents; entropy coding assigns frequency-based
+ *   variable-length codes; the GPU decoder (i) keeps compact lookup tables
+ *   in on-chip SRAM, (ii) coordinates thread read/write positions in two
+ *   phases with small auxiliary arrays, (iii) decompresses a whole
+ *   transformer block at a time; the output is bit-for-bit identical.
+ *   "From a Lossless (~1.5:1) Compression Algorithm for Llama2 7B Weights
+ *   ...", abstract -- ~1.5:1 on Llama2-7B bf16 weights.
+ *   The LazyWeights write-up (bedrocknews.com, arXiv 2611.17108v1) and the
+ *   Huff-LLM abstract -- the entropy code is Huffman.
+ *
+ * FORMAT (the pages leave it open; this library fixes it):
+ *   - Each bf16 bit pattern u splits into an exponent symbol
+ *     e = (u >> 7) & 0xFF and a raw byte m = ((u >> 8) & 0x80) | (u & 0x7F);
+ *     u = ((m & 0x80) << 8) | (e << 7) | (m & 0x7F).
+ *   - The exponents get an optimal prefix code whose lengths are capped at
+ *     `cap` bits (1..32), computed by package-merge with leaves ordered by
+ *     (count, symbol) and leaves merged before packages on equal weight.
+ *     One distinct exponent gets length 0 and an empty stream.
+ *   - Codewords are canonical: assigned in (length, symbol) order as in
+ *     RFC 1951 section 3.2.2.
+ *   - The stream is the codewords of e[0], e[1], ... written MSB-first (the
+ *     first bit is bit 7 of byte 0), zero-padded to a multiple of 64 bytes,
+ *     followed by 16 zero guard bytes (DFW_STREAM_PAD).
+ *   - The raw bytes m[0..n) are stored as they are, zero-padded to a
+ *     multiple of 16 bytes (dfw_mant_bytes).
+ *
+ * DECODE PLAN (auxiliary arrays, DFloat11 abstract point (ii)):
+ *   - The stream is cut into windows of W bytes; window t covers bits
+ *     [8Wt, 8W(t+1)).  gap[t] (one byte) = distance from the window start to
+ *     the first codeword that starts at or after it, or to total_bits if
+ *     none does.  Since no codeword exceeds 32 bits, gap[t] < 32.
+ *   - T consecutive windows form a tile, decoded by one CTA.
+ *     out_start[b] (u64) = number of codewords that start before bit 8WTb,
+ *     i.e. the output index of the tile's first weight; out_start[n_tiles]
+ *     = n.
+ *   - lut is a hierarchy of 256-entry tables keyed by the next 8 code bits
+ *     (DFloat11 abstract point (i)); table 0 resolves every codeword of at
+ *     most 8 bits and points to a subtable for longer ones (at most four
+ *     levels for 32-bit codes).
+ *
+ * MEMORY AND OWNERSHIP: the caller allocates every buffer (host or device).
+ * libdfw keeps no pointer after a call returns.  Device pointers must be
+ * 16-byte aligned (DFW_EALIGN otherwise).  Decode calls are asynchronous on
+ * the given CUDA stream; the caller keeps the buffers alive until the
+ * stream's work completes.
+ *
+ * ERRORS: every call returns a dfw_status.  Host-side validation happens
+ * before any launch.  Corruption that only the device can see (a tile whose
+ * decoded symbol count disagrees with out_start, a table entry that points
+ * outside the table, out_start out of order) is recorded in a per-device
+ * status word, the damaged tile writes nothing, and dfw_check reports it.
+ * Kernels never wait without bound and never trap.
+ */
+#ifndef DFW_H
+#define DFW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dfw_status {
+    DFW_OK = 0,
+    DFW_EINVAL = 1,   /* an argument is out of range or inconsistent */
+    DFW_ECAP = 2,     /* 2^cap is smaller than the number of distinct exponents */
+    DFW_ENOMEM = 3,   /* a caller buffer is too small, or a host allocation failed */
+    DFW_ECORRUPT = 4, /* stream, aux or table are inconsistent with each other */
+    DFW_EALIGN = 5,   /* a device pointer is not 16-byte aligned */
+    DFW_ECUDA = 6     /* a CUDA runtime call failed (launch or copy) */
+} dfw_status;
+
+#define DFW_FORMAT_VERSION 1u
+#define DFW_MAX_CAP 32
+#define DFW_STREAM_PAD 16 /* guard bytes after the 64-byte-rounded stream */
+
+/* Code table and stream metadata written by dfw_encode / dfw_encode_multi. */
+typedef struct dfw_table {
+    uint32_t version;       /* DFW_FORMAT_VERSION */
+    uint32_t cap;           /* length cap the lengths were built with */
+    uint64_t n;             /* number of weights */
+    uint64_t total_bits;    /* coded exponent bits (without padding) */
+    uint64_t stream_bytes;  /* padded stream length in bytes */
+    uint32_t n_symbols;     /* distinct exponents (0 only when n == 0) */
+    uint32_t single_symbol; /* the exponent when n_symbols == 1, else 0 */
+    uint8_t len[256];       /* code length per exponent, 0 = absent */
+} dfw_table;
+
+/* Shape of a decode plan, written by dfw_plan_query and completed by dfw_plan. */
+typedef struct dfw_plan_info {
+    uint32_t window_bytes;     /* W: bytes of stream per window */
+    uint32_t tile_windows;     /* T: windows per tile (one tile per CTA) */
+    uint64_t n_windows;        /* ceil(total_bits / 8W): length of gap[] */
+    uint64_t n_tiles;          /* ceil(n_windows / T): out_start[] has n_tiles + 1 */
+    uint64_t max_tile_symbols; /* largest out_start[b+1] - out_start[b] (dfw_plan) */
+    uint32_t lut_words;        /* u32 words of the LUT image: 256 * lut_tables */
+    uint32_t lut_tables;       /* 256-entry tables in the LUT image */
+} dfw_plan_info;
+
+/* Worst-case padded stream bytes for n weights (every code 32 bits long). */
+uint64_t dfw_stream_bound(uint64_t n);
+
+/* Padded raw-byte (sign+mantissa) array length for n weights. */
+uint64_t dfw_mant_bytes(uint64_t n);
+
+/*
+ * dfw_encode -- split, histogram, capped canonical code, MSB-first packing.
+ * Source: DFloat11 abstract (frequency-based dynamic-length encodings of
+ * bf16 exponents); Huffman per the LazyWeights write-up.  Host only.
+ *   bf16        host, n bf16 bit patterns (read only)
+ *   cap         length cap, 1..32
+ *   stream      host, stream_capacity bytes; receives table->stream_bytes
+ *   mant        host, mant_capacity bytes; receives dfw_mant_bytes(n) bytes
+ *   table       receives the code table and stream metadata
+ *   n_threads   worker threads (0 = all hardware threads); the output is
+ *               byte-identical for every thread count
+ * Errors: DFW_EINVAL (null pointer, cap out of range), DFW_ECAP, DFW_ENOMEM
+ * (table->stream_bytes then holds the size needed).
+ */
+dfw_status dfw_encode(const uint16_t *bf16, uint64_t n, int cap, uint8_t *stream,
+                      uint64_t stream_capacity, uint8_t *mant, uint64_t mant_capacity,
+                      dfw_table *table, int n_threads);
+
+/*
+ * dfw_encode_multi -- one code table over the concatenation of k tensors
+ * (a transformer block; DFloat11 abstract point (iii)).  The stream and the
+ * raw bytes are those of the concatenation in the given order.
+ *   tensors[i]       host pointer to sizes[i] bf16 patterns
+ *   tensor_offsets   host, k + 1 entries: prefix sums of sizes (output)
+ * Other arguments and errors as dfw_encode.
+ */
+dfw_status dfw_encode_multi(const uint16_t *const *tensors, const uint64_t *sizes, int k, int cap,
+                            uint8_t *stream, uint64_t stream_capacity, uint8_t *mant,
+                            uint64_t mant_capacity, dfw_table *table, uint64_t *tensor_offsets,
+                            int n_threads);
+
+/*
+ * dfw_plan_query -- sizes of the plan arrays for a table and (W, T), before
+ * allocation.  Supported: W in {8, 16}, T in {128, 256, 512}.  Fills every
+ * field of info except max_tile_symbols.  Errors: DFW_EINVAL.
+ */
+dfw_status dfw_plan_query(const dfw_table *table, uint32_t window_bytes, uint32_t tile_windows,
+                          dfw_plan_info *info);
+
+/*
+ * dfw_plan -- auxiliary arrays and LUT image for one stream (DFloat11
+ * abstract points (i) and (ii)).  Host only; walks the stream once.
+ *   stream      host, table->stream_bytes bytes
+ *   gap         host, info->n_windows bytes (output)
+ *   out_start   host, info->n_tiles + 1 entries (output)
+ *   lut         host, info->lut_words words (output)
+ *   info        in: from dfw_plan_query; out: max_tile_symbols filled
+ * Errors: DFW_EINVAL, DFW_ECORRUPT (the stream does not hold exactly
+ * table->n codewords in table->total_bits bits).
+ */
+dfw_status dfw_plan(const uint8_t *stream, const dfw_table *table, uint8_t *gap,
+                    uint64_t *out_start, uint32_t *lut, dfw_plan_info *info);
+
+/*
+ * dfw_decode -- bit-exact bf16 reconstruction on the GPU, asynchronous on
+ * `cuda_stream` (a cudaStream_t; NULL = legacy default stream).
+ * Source: DFloat11 abstract (two-phase kernel, SRAM LUTs, bit-exact output).
+ *   d_stream     device, table->stream_bytes bytes
+ *   d_mant       device, dfw_mant_bytes(n) bytes
+ *   d_lut        device, info->lut_words words
+ *   d_gap        device, info->n_windows bytes
+ *   d_out_start  device, info->n_tiles + 1 entries
+ *   table, info  host structures from dfw_encode* and dfw_plan
+ *   d_out        device, n bf16 patterns (output)
+ * Errors: DFW_EINVAL, DFW_EALIGN, DFW_ECUDA; device-detected corruption
+ * through dfw_check.
+ */
+dfw_status dfw_decode(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                      const uint8_t *d_gap, const uint64_t *d_out_start, const dfw_table *table,
+                      const dfw_plan_info *info, uint16_t *d_out, void *cuda_stream);
+
+/*
+ * dfw_decode_block -- decodes the k tensors of one block (one shared table,
+ * encoded by dfw_encode_multi) in one launch into one scratch buffer
+ * (DFloat11 abstract point (iii)); tensor i lands at
+ * d_scratch + tensor_offsets[i].
+ *   tensor_offsets  host, k + 1 entries from dfw_encode_multi
+ *   d_scratch       device, scratch_elems >= table->n bf16 slots
+ * Other arguments and errors as dfw_decode.
+ */
+dfw_status dfw_decode_block(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                            const uint8_t *d_gap, const uint64_t *d_out_start,
+                            const dfw_table *table, const dfw_plan_info *info,
+                            const uint64_t *tensor_offsets, int k, uint16_t *d_scratch,
+                            uint64_t scratch_elems, void *cuda_stream);
+
+/*
+ * dfw_check -- waits for `cuda_stream`, then reads and clears this device's
+ * status word.  Returns DFW_ECORRUPT if any decode since the last check saw
+ * corrupt input, DFW_ECUDA if the stream reported a CUDA error, else DFW_OK.
+ * The word is shared by all streams of the device.
+ */
+dfw_status dfw_check(void *cuda_stream);
+
+/* Static English text for a status code. */
+const char *dfw_strerror(dfw_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DFW_H */

@@ -1,0 +1,212 @@
+"""Lossless entropy-coded bf16 weights, decoded on B200 (sm_100a).
+
+Thin Python binding over libdfw (include/dfw.h).  Every step of encoding,
+planning and decoding runs in the native library; this module only marshals
+torch tensors into pointers and sizes.  PyTorch provides host/device memory
+and CUDA streams.  There is no fallback path: if libdfw.so is missing, the
+first call raises ImportError.
+
+Typical use::
+
+    enc = encode(weights_bf16_cpu)            # host: split, code, pack
+    pl = plan(enc)                            # host: gap/out_start aux + LUT
+    dev = DeviceCompressed.upload(enc, pl)    # H2D (caller's memory: torch)
+    w = decode(dev)                           # GPU: bit-exact bf16 tensor
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, PlanInfo, Table,
+                   check as _check, lib)
+
+__all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
+           "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
+           "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
+
+
+def _ptr(t) -> int:
+    if isinstance(t, torch.Tensor):
+        return t.data_ptr()
+    return int(t.ctypes.data)
+
+
+def _as_u16_host(x) -> torch.Tensor:
+    if isinstance(x, np.ndarray):
+        x = torch.from_numpy(np.ascontiguousarray(x).view(np.int16))
+    if x.is_cuda:
+        raise ValueError("encode takes host tensors")
+    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected bf16 bit patterns, got {x.dtype}")
+    return x.contiguous().reshape(-1)
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def mant_bytes(n: int) -> int:
+    return int(lib().dfw_mant_bytes(n))
+
+
+def stream_bound(n: int) -> int:
+    return int(lib().dfw_stream_bound(n))
+
+
+@dataclass
+class Encoded:
+    """Host result of dfw_encode / dfw_encode_multi."""
+    stream: torch.Tensor  # uint8[table.stream_bytes]
+    mant: torch.Tensor  # uint8[mant_bytes(n)]
+    table: Table
+    tensor_offsets: np.ndarray | None = None  # uint64[k + 1] for a block
+
+    @property
+    def n(self) -> int:
+        return int(self.table.n)
+
+    @property
+    def total_bits(self) -> int:
+        return int(self.table.total_bits)
+
+    @property
+    def lengths(self) -> np.ndarray:
+        return np.frombuffer(bytes(self.table.len), dtype=np.uint8).copy()
+
+
+def _encode_call(fn, n, args_before, args_after, cap, n_threads, pin) -> tuple:
+    mant = torch.empty(mant_bytes(n), dtype=torch.uint8, pin_memory=pin)
+    table = Table()
+    cap_bytes = n + 4096  # enough for <= 8 bits/weight; retried with the exact size otherwise
+    stream = torch.empty(cap_bytes, dtype=torch.uint8, pin_memory=pin)
+    st = fn(*args_before, cap, _ptr(stream), cap_bytes, _ptr(mant), mant.numel(), ctypes.byref(table),
+            *args_after, n_threads)
+    if st == ENOMEM and table.stream_bytes > cap_bytes:
+        cap_bytes = int(table.stream_bytes)
+        stream = torch.empty(cap_bytes, dtype=torch.uint8, pin_memory=pin)
+        st = fn(*args_before, cap, _ptr(stream), cap_bytes, _ptr(mant), mant.numel(), ctypes.byref(table),
+                *args_after, n_threads)
+    _check(st, "dfw_encode")
+    used = int(table.stream_bytes)
+    if used < cap_bytes // 2:  # do not keep a mostly empty (possibly pinned) buffer alive
+        stream = torch.empty(used, dtype=torch.uint8, pin_memory=pin).copy_(stream[:used])
+    return stream[:used], mant, table
+
+
+def encode(bf16, cap: int = 32, n_threads: int = 0, pin: bool = False) -> Encoded:
+    """Encodes one host bf16 tensor (any shape; flattened)."""
+    u = _as_u16_host(bf16)
+    stream, mant, table = _encode_call(lib().dfw_encode, u.numel(), [_ptr(u), u.numel()], [], cap, n_threads, pin)
+    return Encoded(stream, mant, table)
+
+
+def encode_multi(tensors, cap: int = 32, n_threads: int = 0, pin: bool = False) -> Encoded:
+    """Encodes k host bf16 tensors with one shared code table (one block)."""
+    us = [_as_u16_host(t) for t in tensors]
+    k = len(us)
+    ptrs = (ctypes.c_void_p * k)(*[_ptr(u) for u in us])
+    sizes = (ctypes.c_uint64 * k)(*[u.numel() for u in us])
+    offs = np.zeros(k + 1, dtype=np.uint64)
+    n = int(sum(u.numel() for u in us))
+    stream, mant, table = _encode_call(lib().dfw_encode_multi, n, [ptrs, sizes, k], [_ptr(offs)], cap,
+                                       n_threads, pin)
+    return Encoded(stream, mant, table, offs)
+
+
+@dataclass
+class Plan:
+    """Host result of dfw_plan: aux arrays, LUT image and plan shape."""
+    gap: torch.Tensor  # uint8[n_windows]
+    out_start: torch.Tensor  # int64 view of uint64[n_tiles + 1]
+    lut: torch.Tensor  # int32 view of uint32[lut_words]
+    info: PlanInfo
+
+
+def plan(enc: Encoded, window_bytes: int = 8, tile_windows: int = 256, pin: bool = False) -> Plan:
+    info = PlanInfo()
+    _check(lib().dfw_plan_query(ctypes.byref(enc.table), window_bytes, tile_windows, ctypes.byref(info)),
+           "dfw_plan_query")
+    gap = torch.empty(int(info.n_windows), dtype=torch.uint8, pin_memory=pin)
+    out_start = torch.empty(int(info.n_tiles) + 1, dtype=torch.int64, pin_memory=pin)
+    lut = torch.empty(int(info.lut_words), dtype=torch.int32, pin_memory=pin)
+    _check(lib().dfw_plan(_ptr(enc.stream), ctypes.byref(enc.table), _ptr(gap), _ptr(out_start), _ptr(lut),
+                          ctypes.byref(info)), "dfw_plan")
+    return Plan(gap, out_start, lut, info)
+
+
+@dataclass
+class DeviceCompressed:
+    """A compressed tensor or block resident in device memory."""
+    stream: torch.Tensor
+    mant: torch.Tensor
+    lut: torch.Tensor
+    gap: torch.Tensor
+    out_start: torch.Tensor
+    table: Table
+    info: PlanInfo
+    tensor_offsets: np.ndarray | None = None
+
+    @staticmethod
+    def upload(enc: Encoded, pl: Plan, device="cuda", non_blocking: bool = False) -> "DeviceCompressed":
+        mv = lambda t: t.to(device, non_blocking=non_blocking)  # noqa: E731
+        return DeviceCompressed(mv(enc.stream), mv(enc.mant), mv(pl.lut), mv(pl.gap), mv(pl.out_start),
+                                enc.table, pl.info, enc.tensor_offsets)
+
+    @property
+    def n(self) -> int:
+        return int(self.table.n)
+
+    def compressed_bytes(self, with_aux: bool = True) -> int:
+        b = int(self.table.stream_bytes) + self.n + 256  # stream + raw bytes + length table
+        if with_aux:
+            b += self.gap.numel() + 8 * self.out_start.numel() + 4 * self.lut.numel()
+        return b
+
+    def algorithmic_bytes(self) -> int:
+        """Bytes a decode must move: coded stream + gap + out_start read,
+        one raw byte read and one bf16 written per weight."""
+        return (int(self.table.stream_bytes) + self.gap.numel() + 8 * self.out_start.numel()
+                + 4 * self.lut.numel() + self.n + 2 * self.n)
+
+
+def _decode_args(dc: DeviceCompressed):
+    return (_ptr(dc.stream), _ptr(dc.mant), _ptr(dc.lut), _ptr(dc.gap), _ptr(dc.out_start),
+            ctypes.byref(dc.table), ctypes.byref(dc.info))
+
+
+def decode(dc: DeviceCompressed, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decodes into ``out`` (bf16, n elements, on the device) asynchronously."""
+    if out is None:
+        out = torch.empty(dc.n, dtype=torch.bfloat16, device=dc.mant.device)
+    if out.numel() < dc.n or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor of at least n elements")
+    _check(lib().dfw_decode(*_decode_args(dc), _ptr(out), _stream_handle(stream)), "dfw_decode")
+    return out
+
+
+def decode_block(dc: DeviceCompressed, scratch: torch.Tensor | None = None, stream=None):
+    """Decodes a block (k tensors, one table) into one scratch buffer; returns
+    (scratch, [view of tensor i])."""
+    offs = dc.tensor_offsets if dc.tensor_offsets is not None else np.array([0, dc.n], np.uint64)
+    k = offs.size - 1
+    if scratch is None:
+        scratch = torch.empty(dc.n, dtype=torch.bfloat16, device=dc.mant.device)
+    _check(lib().dfw_decode_block(*_decode_args(dc), _ptr(offs), k, _ptr(scratch), scratch.numel(),
+                                  _stream_handle(stream)), "dfw_decode_block")
+    views = [scratch[int(offs[i]): int(offs[i + 1])] for i in range(k)]
+    return scratch, views
+
+
+def check(stream=None) -> None:
+    """Synchronises the stream and raises DfwError if a decode saw corruption."""
+    _check(lib().dfw_check(_stream_handle(stream)), "dfw_check")
+
+
+def check_status(stream=None) -> int:
+    return int(lib().dfw_check(_stream_handle(stream)))

@@ -1,0 +1,73 @@
+"""ctypes declarations of the libdfw C ABI (include/dfw.h)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdfw.so")
+
+OK, EINVAL, ECAP, ENOMEM, ECORRUPT, EALIGN, ECUDA = range(7)
+FORMAT_VERSION = 1
+MAX_CAP = 32
+
+
+class DfwError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = lib().dfw_strerror(status).decode() if _lib is not None else str(status)
+        super().__init__(f"{what}: {msg} (status {status})")
+
+
+class Table(ctypes.Structure):
+    _fields_ = [("version", ctypes.c_uint32), ("cap", ctypes.c_uint32), ("n", ctypes.c_uint64),
+                ("total_bits", ctypes.c_uint64), ("stream_bytes", ctypes.c_uint64),
+                ("n_symbols", ctypes.c_uint32), ("single_symbol", ctypes.c_uint32),
+                ("len", ctypes.c_uint8 * 256)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("window_bytes", ctypes.c_uint32), ("tile_windows", ctypes.c_uint32),
+                ("n_windows", ctypes.c_uint64), ("n_tiles", ctypes.c_uint64),
+                ("max_tile_symbols", ctypes.c_uint64), ("lut_words", ctypes.c_uint32),
+                ("lut_tables", ctypes.c_uint32)]
+
+
+_lib = None
+
+# name -> (restype, argtypes); the symbols include/dfw.h declares
+_vp, _u64, _i = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int
+_TP, _IP = ctypes.POINTER(Table), ctypes.POINTER(PlanInfo)
+SIGNATURES = {
+    "dfw_stream_bound": (_u64, [_u64]),
+    "dfw_mant_bytes": (_u64, [_u64]),
+    "dfw_encode": (_i, [_vp, _u64, _i, _vp, _u64, _vp, _u64, _TP, _i]),
+    "dfw_encode_multi": (_i, [_vp, _vp, _i, _i, _vp, _u64, _vp, _u64, _TP, _vp, _i]),
+    "dfw_plan_query": (_i, [_TP, ctypes.c_uint32, ctypes.c_uint32, _IP]),
+    "dfw_plan": (_i, [_vp, _TP, _vp, _vp, _vp, _IP]),
+    "dfw_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _IP, _vp, _vp]),
+    "dfw_decode_block": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _IP, _vp, _i, _vp, _u64, _vp]),
+    "dfw_check": (_i, [_vp]),
+    "dfw_strerror": (ctypes.c_char_p, [_i]),
+}
+
+
+def lib():
+    """Loads libdfw.so from the package directory; fails loudly if absent."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libdfw.so is not built ({LIB_PATH}); run "
+                              "`python -m lossless_entropy_coded_canonical_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def check(status: int, what: str):
+    if status != OK:
+        raise DfwError(status, what)

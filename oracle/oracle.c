@@ -338,46 +338,32 @@ int oracle_aux(const uint8_t *stream, uint64_t total_bits, const uint8_t len[256
         return OR_EINVAL;
     uint64_t nwin = oracle_n_windows(total_bits, W);
     uint64_t ntiles = (nwin + T - 1) / T;
-    uint64_t *starts = (uint64_t *)malloc((size_t)(n + 1) * sizeof(uint64_t));
-    if (!starts)
-        return OR_ENOMEM;
-    uint64_t nstarts = 0;
-    if (total_bits > 0) {
-        canon_dec d;
-        canon_init(len, &d);
-        uint64_t pos = 0;
-        while (pos < total_bits) {
-            if (nstarts >= n) {
-                free(starts);
-                return OR_ECORRUPT;
-            }
-            starts[nstarts++] = pos;
-            if (canon_read(&d, stream, total_bits, &pos) < 0) {
-                free(starts);
-                return OR_ECORRUPT;
-            }
+    uint64_t t = 0, b = 0, count = 0, pos = 0;
+    canon_dec d;
+    canon_init(len, &d);
+    /* visit the code starts in order; every window (tile) not yet given a
+     * value takes the first start at or after its own first bit */
+    while (pos < total_bits) {
+        while (t < nwin && 8 * W * t <= pos) {
+            gap[t] = (uint8_t)(pos - 8 * W * t);
+            t++;
         }
-        if (nstarts != n) {
-            free(starts);
+        while (b < ntiles && 8 * W * T * b <= pos) {
+            out_start[b] = count;
+            b++;
+        }
+        if (canon_read(&d, stream, total_bits, &pos) < 0)
             return OR_ECORRUPT;
-        }
+        count++;
+        if (count > n)
+            return OR_ECORRUPT;
     }
-    uint64_t j = 0;
-    for (uint64_t t = 0; t < nwin; t++) {
-        uint64_t wstart = 8 * W * t;
-        while (j < nstarts && starts[j] < wstart)
-            j++;
-        uint64_t s = j < nstarts ? starts[j] : total_bits;
-        gap[t] = (uint8_t)(s - wstart);
-    }
-    j = 0;
-    for (uint64_t b = 0; b < ntiles; b++) {
-        uint64_t tstart = 8 * W * T * b;
-        while (j < nstarts && starts[j] < tstart)
-            j++;
-        out_start[b] = j;
-    }
+    if (total_bits > 0 && count != n)
+        return OR_ECORRUPT;
+    for (; t < nwin; t++)
+        gap[t] = (uint8_t)(total_bits - 8 * W * t);
+    for (; b < ntiles; b++)
+        out_start[b] = n;
     out_start[ntiles] = n;
-    free(starts);
     return OR_OK;
 }
