@@ -40,10 +40,15 @@
  *     out_start[b] (u64) = number of codewords that start before bit 8WTb,
  *     i.e. the output index of the tile's first weight; out_start[n_tiles]
  *     = n.
- *   - lut is a hierarchy of 256-entry tables keyed by the next 8 code bits
- *     (DFloat11 abstract point (i)); table 0 resolves every codeword of at
- *     most 8 bits and points to a subtable for longer ones (at most four
- *     levels for 32-bit codes).
+ *   - lut (DFloat11 abstract point (i): compact tables in on-chip SRAM) holds
+ *     two parts.  First a fast table of 2^K 64-bit entries (K = fast_bits,
+ *     8..12) keyed by the next K stream bits at a codeword start: it lists up
+ *     to four whole codewords inside those K bits (their symbols, how many,
+ *     the bits they use and where each ends) or marks an escape when the
+ *     first codeword is longer than K bits.  Then a hierarchy of 256-entry
+ *     tables keyed by successive bytes of the code: table 0 resolves every
+ *     codeword of at most 8 bits and points to a subtable for longer ones (at
+ *     most four levels for 32-bit codes); escapes are resolved through it.
  *
  * MEMORY AND OWNERSHIP: the caller allocates every buffer (host or device).
  * libdfw keeps no pointer after a call returns.  Device pointers must be
@@ -98,11 +103,13 @@ typedef struct dfw_table {
 typedef struct dfw_plan_info {
     uint32_t window_bytes;     /* W: bytes of stream per window */
     uint32_t tile_windows;     /* T: windows per tile (one tile per CTA) */
-    uint64_t n_windows;        /* ceil(total_bits / 8W): length of gap[] */
+    uint64_t n_windows;        /* ceil(total_bits / 8W) windows; gap[] holds n_tiles * T bytes */
     uint64_t n_tiles;          /* ceil(n_windows / T): out_start[] has n_tiles + 1 */
     uint64_t max_tile_symbols; /* largest out_start[b+1] - out_start[b] (dfw_plan) */
-    uint32_t lut_words;        /* u32 words of the LUT image: 256 * lut_tables */
-    uint32_t lut_tables;       /* 256-entry tables in the LUT image */
+    uint32_t lut_words;        /* u32 words of the LUT image: 2 * 2^fast_bits + 256 * lut_tables */
+    uint32_t lut_tables;       /* 256-entry byte-keyed tables after the fast table */
+    uint32_t fast_bits;        /* K: key width of the fast table (dfw_plan_query sets 10) */
+    uint32_t reserved;         /* zero */
 } dfw_plan_info;
 
 /* Worst-case padded stream bytes for n weights (every code 32 bits long). */
@@ -144,8 +151,11 @@ dfw_status dfw_encode_multi(const uint16_t *const *tensors, const uint64_t *size
 
 /*
  * dfw_plan_query -- sizes of the plan arrays for a table and (W, T), before
- * allocation.  Supported: W in {8, 16}, T in {128, 256, 512}.  Fills every
- * field of info except max_tile_symbols.  Errors: DFW_EINVAL.
+ * allocation.  Supported: W in {8, 16}, T in {128, 256, 512}, W * T <= 4096
+ * (a tile's worst case must fit in shared memory).  Fills every
+ * field of info except max_tile_symbols, with fast_bits = 10; a caller may
+ * set fast_bits to another value in 8..12 and call again with it filled in
+ * (a nonzero info->fast_bits on entry is kept).  Errors: DFW_EINVAL.
  */
 dfw_status dfw_plan_query(const dfw_table *table, uint32_t window_bytes, uint32_t tile_windows,
                           dfw_plan_info *info);
@@ -154,7 +164,8 @@ dfw_status dfw_plan_query(const dfw_table *table, uint32_t window_bytes, uint32_
  * dfw_plan -- auxiliary arrays and LUT image for one stream (DFloat11
  * abstract points (i) and (ii)).  Host only; walks the stream once.
  *   stream      host, table->stream_bytes bytes
- *   gap         host, info->n_windows bytes (output)
+ *   gap         host, info->n_tiles * info->tile_windows bytes (output; the
+ *               first n_windows are the gaps, the rest zero padding)
  *   out_start   host, info->n_tiles + 1 entries (output)
  *   lut         host, info->lut_words words (output)
  *   info        in: from dfw_plan_query; out: max_tile_symbols filled
@@ -171,7 +182,7 @@ dfw_status dfw_plan(const uint8_t *stream, const dfw_table *table, uint8_t *gap,
  *   d_stream     device, table->stream_bytes bytes
  *   d_mant       device, dfw_mant_bytes(n) bytes
  *   d_lut        device, info->lut_words words
- *   d_gap        device, info->n_windows bytes
+ *   d_gap        device, info->n_tiles * info->tile_windows bytes
  *   d_out_start  device, info->n_tiles + 1 entries
  *   table, info  host structures from dfw_encode* and dfw_plan
  *   d_out        device, n bf16 patterns (output)

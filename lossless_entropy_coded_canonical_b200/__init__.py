@@ -122,17 +122,19 @@ def encode_multi(tensors, cap: int = 32, n_threads: int = 0, pin: bool = False) 
 @dataclass
 class Plan:
     """Host result of dfw_plan: aux arrays, LUT image and plan shape."""
-    gap: torch.Tensor  # uint8[n_windows]
+    gap: torch.Tensor  # uint8[n_tiles * tile_windows]: n_windows gaps, then zero padding
     out_start: torch.Tensor  # int64 view of uint64[n_tiles + 1]
     lut: torch.Tensor  # int32 view of uint32[lut_words]
     info: PlanInfo
 
 
-def plan(enc: Encoded, window_bytes: int = 8, tile_windows: int = 256, pin: bool = False) -> Plan:
+def plan(enc: Encoded, window_bytes: int = 8, tile_windows: int = 256, pin: bool = False,
+         fast_bits: int = 0) -> Plan:
     info = PlanInfo()
+    info.fast_bits = fast_bits  # 0 = library default
     _check(lib().dfw_plan_query(ctypes.byref(enc.table), window_bytes, tile_windows, ctypes.byref(info)),
            "dfw_plan_query")
-    gap = torch.empty(int(info.n_windows), dtype=torch.uint8, pin_memory=pin)
+    gap = torch.empty(int(info.n_tiles) * int(info.tile_windows), dtype=torch.uint8, pin_memory=pin)
     out_start = torch.empty(int(info.n_tiles) + 1, dtype=torch.int64, pin_memory=pin)
     lut = torch.empty(int(info.lut_words), dtype=torch.int32, pin_memory=pin)
     _check(lib().dfw_plan(_ptr(enc.stream), ctypes.byref(enc.table), _ptr(gap), _ptr(out_start), _ptr(lut),

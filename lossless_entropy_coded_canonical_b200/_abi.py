@@ -30,7 +30,7 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("window_bytes", ctypes.c_uint32), ("tile_windows", ctypes.c_uint32),
                 ("n_windows", ctypes.c_uint64), ("n_tiles", ctypes.c_uint64),
                 ("max_tile_symbols", ctypes.c_uint64), ("lut_words", ctypes.c_uint32),
-                ("lut_tables", ctypes.c_uint32)]
+                ("lut_tables", ctypes.c_uint32), ("fast_bits", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
 
 
 _lib = None

@@ -4,26 +4,34 @@
 // Compression for Efficient GPU Inference via Dynamic-Length Float"): compact
 // LUTs in GPU SRAM, a two-phase kernel that coordinates thread read/write
 // positions through lightweight auxiliary arrays, block-level decompression,
-// bit-exact output.  This kernel is written for B200 from that description:
+// bit-exact output.  This kernel is written for B200 from that description.
 //
-//   one CTA per tile of T windows of W stream bytes (one window per thread)
-//   phase 0  LUT table 0 -> shared memory (validated once per CTA);
-//            each thread loads its W (+4 guard) stream bytes and its gap
-//   phase 1  each thread walks the codewords that start in its window and
-//            counts them; whole codewords inside the next 8 bits are counted
-//            in one table lookup
-//   scan     warp shuffle scan + block scan of the counts; the tile's total
-//            must equal out_start[b+1] - out_start[b]
-//   phase 2  each thread walks its window again and writes the exponent
-//            symbols into a shared-memory buffer at its scanned offset
-//   phase 3  all threads turn (exponent, raw byte) pairs into bf16, 8 weights
-//            per thread per step: 64-bit shared and global loads, 128-bit
-//            coalesced global stores; ragged tile edges go element by element
+// Persistent CTAs (grid = SMs x resident CTAs) load the fast table into
+// shared memory once, then loop over tiles of T windows of W stream bytes
+// (one window per thread).  Tiles are double-buffered: while tile i is
+// decoded, one thread has already started TMA bulk copies (cp.async.bulk,
+// completion on an mbarrier, no multicast) of the next tile's stream bytes,
+// gap bytes and raw-byte range into the other buffer.  Per tile:
+//   phase 1  each thread decodes the codewords that start in its window; one
+//            fast-table lookup yields up to four whole codewords; symbols go
+//            through a 64-bit register accumulator into the thread's own
+//            word slots (interleaved by thread: conflict-free stores)
+//   scan     warp shuffle scan of the counts; one CTA barrier publishes the
+//            warp totals, and every warp scans those itself (no second
+//            barrier); the tile total must equal out_start[b+1] - out_start[b]
+//   phase 2  each thread copies its symbols a word at a time (funnel shift to
+//            the destination's byte alignment) into the tile's exponent buffer
+//   phase 3  each warp assembles bf16 for its own output range from the
+//            exponent buffer and the raw bytes already in shared memory, 16
+//            weights per thread-step, 128-bit coalesced stores, ragged ends
+//            element by element; warps need no barrier between phases 2 and 3
+//            (the exponent buffer alternates between two copies by tile)
 //
-// Bounds: every walk advances at least one bit per step and stops at its
-// window end (8W bits), so no loop depends on the data for termination; the
-// LUT is checked before use; tiles whose counts or ranges are inconsistent
-// write nothing and set a bit of the device status word.
+// Bounds: every lookup advances at least one bit and a walk stops at its
+// window end, so loops end whatever the data; tables are validated once per
+// CTA; waits on bulk copies give up after a time limit (status bit, early
+// return); a tile whose counts or ranges disagree writes nothing and sets a
+// bit of the device status word.  Nothing waits on another CTA.
 #include <cuda_runtime.h>
 
 #include "dfw_internal.h"
@@ -34,59 +42,146 @@ __device__ unsigned int g_status;
 
 namespace {
 
+constexpr uint32_t ESC_BAD = 0x40000000u;
+constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s, far above any copy
+
+// --------------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Orders this thread's earlier generic accesses to shared memory (made
+// visible to it by a barrier) before its later bulk-copy writes.
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// 1-D bulk copy global -> this CTA's shared memory; 16-byte aligned addresses
+// and a size that is a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0u;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for a phase of an mbarrier with a time and iteration limit; false if
+// it gave up.
+__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    for (uint32_t it = 0; it < (1u << 24); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+    }
+    return false;
+}
+
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
-// Walks subtables (global memory, read-only path) for a codeword longer than
-// 8 bits.  x holds the 32 stream bits starting at the codeword.
-__device__ __noinline__ uint32_t resolve_long(uint32_t x, uint32_t e, const uint32_t *__restrict__ g_lut,
-                                              uint32_t n_tables, uint32_t &err) {
+// --------------------------------------------------------------- decoding
+
+// A codeword longer than the fast table's key: walk the byte-keyed hierarchy
+// (global memory, read-only path).  x holds the 32 stream bits from the
+// codeword's first bit.  Returns a hierarchy leaf (symbol, total length), or
+// on a corrupt table ESC_BAD with length 1.
+__device__ __noinline__ uint32_t resolve_escape(uint32_t x, const uint32_t *__restrict__ g_hier,
+                                                uint32_t n_tables) {
+    uint32_t e = __ldg(g_hier + (x >> 24));
 #pragma unroll 1
-    for (int level = 1; level < 4; ++level) {
+    for (int level = 1; level < 4 && (e & LUT_PTR); ++level) {
         const uint32_t child = e & LUT_CHILD_MASK;
         if (child >= n_tables) break;
-        e = __ldg(g_lut + child * 256u + ((x >> (24 - 8 * level)) & 0xFFu));
+        e = __ldg(g_hier + child * 256u + ((x >> (24 - 8 * level)) & 0xFFu));
         if (!(e & LUT_PTR)) {
             const uint32_t l = (e >> LUT_LEN_SHIFT) & 63u;
             if (l > 8u * level && l <= 8u * level + 8u) return e;
             break;
         }
     }
-    err |= ST_LUT;
-    return 1u << LUT_LEN_SHIFT;  // length 1 keeps the walk finite
+    return ESC_BAD | (1u << LUT_LEN_SHIFT);  // length 1 keeps the walk finite
 }
 
-// Walks the codewords starting in [p, wend) of a window held as NSEG
-// big-endian words plus one guard word.  Counts them (EMIT = false) or also
-// writes their symbols to ebuf[o...] (EMIT = true), never past ebuf[lim].
-template <bool EMIT, int NSEG>
-__device__ __forceinline__ uint32_t walk(const uint32_t (&wd)[NSEG + 1], int p, const int wend,
-                                         const uint32_t *__restrict__ s_lut,
-                                         const uint32_t *__restrict__ g_lut, uint32_t n_tables,
-                                         uint8_t *__restrict__ ebuf, uint32_t o, uint32_t lim,
-                                         uint32_t &err) {
-    uint32_t cnt = 0;
+// Phase 1 for one window held as NSEG big-endian words plus a guard word:
+// decodes the codewords starting in [p, wend) and appends their symbols to
+// the thread's word slots wp[0], wp[NT], ...  Returns the codeword count.
+// A final lookup that crosses wend appends all its symbols but counts only
+// the codewords that start before wend (the extra bytes are never read).
+template <int NSEG, int NT>
+__device__ __forceinline__ uint32_t decode_window(const uint32_t (&wd)[NSEG + 1], int p, const int wend,
+                                                  const uint2 *__restrict__ s_fast, const uint32_t kshift,
+                                                  const uint32_t *__restrict__ g_hier, uint32_t n_tables,
+                                                  uint32_t *__restrict__ wp, uint32_t &err) {
+    uint32_t *const wp0 = wp;
+    uint32_t lo = 0u, hi = 0u, sh = 0u, extra = 0u;
 #pragma unroll
     for (int seg = 0; seg < NSEG; ++seg) {
-        const uint32_t hi = wd[seg], lo = wd[seg + 1];
+        const uint32_t a = wd[seg], b = wd[seg + 1];
         const int seg_end = min(32 * (seg + 1), wend);
         while (p < seg_end) {
-            const uint32_t x = __funnelshift_l(lo, hi, (uint32_t)p);  // bits [p, p + 32)
-            uint32_t e = s_lut[x >> 24];
-            if (!EMIT) {
-                const uint32_t c = (e >> LUT_CNT_SHIFT) & 15u;
-                if (c != 0u && p + 8 <= wend) {  // all c codewords start before wend
-                    cnt += c;
-                    p += (int)((e >> LUT_CBITS_SHIFT) & 15u);
-                    continue;
+            const uint32_t x = __funnelshift_l(b, a, (uint32_t)p);  // stream bits [p, p + 32)
+            const uint2 e = s_fast[x >> kshift];
+            uint32_t syms = e.x, c8 = __byte_perm(e.y, 0u, 0x4441);
+            int pn = p + (int)(e.y & 255u);
+            if (pn > wend) {
+                if (e.y & FAST_ESC) {
+                    const uint32_t f = resolve_escape(x, g_hier, n_tables);
+                    if (f & ESC_BAD) err |= ST_LUT;
+                    syms = f & 0xFFu;
+                    c8 = 8u;
+                    pn = p + (int)((f >> LUT_LEN_SHIFT) & 63u);
+                } else {
+                    // codeword 0 starts at p < wend; codeword k+1 starts where k
+                    // ends, so it counts if that end offset is below wend - p
+                    const uint32_t ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
+                    const uint32_t r = (uint32_t)(wend - p);
+                    const uint32_t t8 = min(c8, 8u + 8u * (uint32_t)__popc(ends & ((1u << (r - 1u)) - 1u)));
+                    extra = c8 - t8;
                 }
             }
-            if (e & LUT_PTR) e = resolve_long(x, e, g_lut, n_tables, err);
-            if (EMIT) ebuf[min(o + cnt, lim)] = (uint8_t)e;  // clamp only matters for a corrupt LUT
-            ++cnt;
-            p += (int)((e >> LUT_LEN_SHIFT) & 63u);
+            lo |= syms << sh;
+            hi |= __funnelshift_l(syms, 0u, sh);
+            sh += c8;
+            const bool full = sh >= 32u;
+            if (full) *wp = lo;
+            wp += full ? NT : 0;
+            lo = full ? hi : lo;
+            hi = full ? 0u : hi;
+            sh &= 31u;
+            p = pn;
         }
     }
-    return cnt;
+    if (sh) *wp = lo;
+    const uint32_t words = (uint32_t)(wp - wp0) / NT;  // full words flushed
+    return (32u * words + sh - extra) >> 3;
 }
 
 // Four (exponent, raw byte) pairs -> four bf16 patterns in two words.
@@ -101,132 +196,237 @@ __device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t m) {
     return (uint16_t)(((m & 0x80u) << 8) | (e << 7) | (m & 0x7Fu));
 }
 
-constexpr int SMEM_HEAD = 1024 + 128;  // LUT table 0 + per-warp scan slots
+struct Params {
+    const uint8_t *stream;
+    const uint8_t *mant;
+    const uint32_t *lut;
+    const uint8_t *gap;
+    const uint64_t *out_start;
+    uint16_t *out;
+    uint64_t total_bits, stream_bytes, n_windows, n_tiles, n;
+    uint32_t fast_bits, n_tables;
+    uint32_t ebuf_bytes;  // tile exponent buffer (>= max tile symbols + 16)
+    uint32_t mbuf_bytes;  // raw-byte buffer per slot (>= max tile symbols + 32)
+};
+
+// Shared memory: fast table | scan slots | 2 mbarriers | word slots |
+// 2 exponent buffers | 2 x (stream bytes | gap bytes | raw bytes).
+template <int W, int NT>
+struct Layout {
+    static constexpr uint32_t PRIV_WORDS = 2 * W + 1;  // 8W + 4 bytes: a window's worst case
+    static constexpr uint32_t SBUF = NT * W + 16;      // a tile's stream bytes + guard
+    uint32_t fast, scan, mbar, priv, ebuf, slot0, slot_bytes, total;
+    __host__ __device__ Layout(uint32_t fast_bits, uint32_t ebuf_bytes, uint32_t mbuf_bytes) {
+        fast = 0;
+        scan = 8u << fast_bits;
+        mbar = scan + 64 * 4;
+        priv = mbar + 16;
+        ebuf = priv + 4 * PRIV_WORDS * NT;
+        slot0 = ebuf + 2 * ebuf_bytes;
+        slot_bytes = SBUF + NT + mbuf_bytes;
+        total = slot0 + 2 * slot_bytes;
+    }
+};
 
 template <int W, int NT>
-__global__ void __launch_bounds__(NT) decode_tiles(
-    const uint8_t *__restrict__ stream, const uint8_t *__restrict__ mant,
-    const uint32_t *__restrict__ g_lut, uint32_t n_tables, const uint8_t *__restrict__ gap,
-    const uint64_t *__restrict__ out_start, uint64_t total_bits, uint64_t n_windows, uint64_t n,
-    uint32_t ebuf_syms, uint16_t *__restrict__ out) {
+__global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
     constexpr int NSEG = W / 4;
     constexpr int NWARP = NT / 32;
+    using L = Layout<W, NT>;
     static_assert(NWARP <= 32, "block scan assumes at most 32 warps");
     extern __shared__ __align__(16) uint8_t smem[];
-    uint32_t *s_lut = reinterpret_cast<uint32_t *>(smem);
-    uint32_t *s_warp = s_lut + 256;
-    uint8_t *ebuf = smem + SMEM_HEAD;
-
+    const L lay(prm.fast_bits, prm.ebuf_bytes, prm.mbuf_bytes);
+    const uint32_t n_fast = 1u << prm.fast_bits;
+    uint2 *s_fast = reinterpret_cast<uint2 *>(smem + lay.fast);
+    uint32_t *s_scan = reinterpret_cast<uint32_t *>(smem + lay.scan);
+    uint32_t *s_priv = reinterpret_cast<uint32_t *>(smem + lay.priv);
+    uint8_t *ebuf = smem + lay.ebuf;
+    const uint32_t bar0 = smem_u32(smem + lay.mbar);
+    const uint32_t *g_hier = prm.lut + 2u * n_fast;
+    const uint32_t kshift = 32u - prm.fast_bits;
+    const uint64_t tile_bytes = (uint64_t)NT * W;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const uint64_t tile = blockIdx.x;
-    const uint64_t os = out_start[tile], oe = out_start[tile + 1];
 
-    // phase 0: table 0 into shared memory, checked entry by entry
-    bool lut_bad = false;
-    for (int i = tid; i < 256; i += NT) {
-        const uint32_t e = __ldg(g_lut + i);
-        if (!(e & LUT_PTR)) {
-            const uint32_t l = (e >> LUT_LEN_SHIFT) & 63u, c = (e >> LUT_CNT_SHIFT) & 15u,
-                           cb = (e >> LUT_CBITS_SHIFT) & 15u;
-            lut_bad |= l == 0u || l > 8u || c == 0u || cb == 0u || cb > 8u;
-        }
-        s_lut[i] = e;
+    // Starts the copies of tile t's bytes into slot s (thread 0 only). A tile
+    // whose out_start range is out of bounds copies no raw bytes; the consumer
+    // rejects it by the same test.
+    auto issue = [&](uint64_t t, uint32_t s, uint64_t os, uint64_t oe) {
+        uint8_t *slot = smem + lay.slot0 + s * lay.slot_bytes;
+        const uint64_t sb0 = t * tile_bytes;
+        const uint32_t sbytes = (uint32_t)min((uint64_t)L::SBUF, prm.stream_bytes - sb0);
+        const bool ok = oe >= os && oe <= prm.n && oe - os + 32 <= prm.mbuf_bytes;
+        const uint64_t m0 = os & ~15ull, m1 = (oe + 15) & ~15ull;
+        const uint32_t mbytes = ok ? (uint32_t)(m1 - m0) : 0u;
+        fence_proxy_async();
+        mbar_expect_tx(bar0 + 8 * s, sbytes + NT + mbytes);
+        bulk_load(smem_u32(slot), prm.stream + sb0, sbytes, bar0 + 8 * s);
+        bulk_load(smem_u32(slot + L::SBUF), prm.gap + t * NT, NT, bar0 + 8 * s);
+        if (mbytes) bulk_load(smem_u32(slot + L::SBUF + NT), prm.mant + m0, mbytes, bar0 + 8 * s);
+    };
+
+    if (tid == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar0 + 8, 1);
+        fence_mbar_init();
     }
-    const uint64_t w = tile * NT + tid;
-    uint32_t wd[NSEG + 1];
-    int p = 0, wend = 0;
-    if (w < n_windows) {
-        const uint8_t *src = stream + w * W;
-        if constexpr (W == 8) {
-            const uint2 v = __ldg(reinterpret_cast<const uint2 *>(src));
-            wd[0] = bswap32(v.x);
-            wd[1] = bswap32(v.y);
+    // fast table into shared memory, each entry checked once per CTA
+    bool bad = false;
+    for (uint32_t i = tid; i < n_fast; i += NT) {
+        const uint2 e = __ldg(reinterpret_cast<const uint2 *>(prm.lut) + i);
+        if (e.y & FAST_ESC) {
+            bad |= e.y != FAST_ESC_WORD || e.x != 0u;
         } else {
-            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(src));
-            wd[0] = bswap32(v.x);
-            wd[1] = bswap32(v.y);
-            wd[2] = bswap32(v.z);
-            wd[3] = bswap32(v.w);
+            const uint32_t cb = e.y & 255u, c8 = (e.y >> FAST_C8_SHIFT) & 255u,
+                           ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
+            bad |= c8 == 0u || (c8 & 7u) || c8 > 8u * FAST_MAX_SYMS || cb == 0u || cb > prm.fast_bits ||
+                   8u * cb < c8 || (uint32_t)__popc(ends) * 8u != c8 || (ends >> (cb - 1u)) != 1u ||
+                   (e.y & 0x70000000u) || (c8 < 32u && (e.x >> c8) != 0u);
         }
-        wd[NSEG] = bswap32(__ldg(reinterpret_cast<const uint32_t *>(src + W)));
-        p = __ldg(gap + w);
-        const uint64_t rem = total_bits - w * (8ull * W);
-        wend = rem < 8ull * W ? (int)rem : 8 * W;
-    } else {
-#pragma unroll
-        for (int i = 0; i <= NSEG; ++i) wd[i] = 0u;
+        s_fast[i] = e;
     }
-    if (__syncthreads_or(lut_bad)) {
+    uint64_t tile = blockIdx.x;
+    uint64_t os = 0, oe = 0;
+    if (tile < prm.n_tiles) {
+        os = __ldg(prm.out_start + tile);
+        oe = __ldg(prm.out_start + tile + 1);
+    }
+    if (__syncthreads_or(bad)) {
         if (tid == 0) atomicOr(&g_status, ST_LUT);
         return;
     }
-    if (oe < os || oe > n || oe - os > ebuf_syms) {
-        if (tid == 0) atomicOr(&g_status, ST_RANGE);
-        return;
-    }
+    if (tid == 0 && tile < prm.n_tiles) issue(tile, 0, os, oe);
 
-    // phase 1: count the codewords that start in this thread's window
-    uint32_t err = 0;
-    const uint32_t cnt = walk<false, NSEG>(wd, p, wend, s_lut, g_lut, n_tables, nullptr, 0, 0, err);
+    for (uint32_t k = 0; tile < prm.n_tiles; ++k) {
+        const uint32_t s = k & 1u;
+        const uint8_t *slot = smem + lay.slot0 + s * lay.slot_bytes;
+        const uint64_t next = tile + gridDim.x;
+        uint64_t nos = 0, noe = 0;
+        if (next < prm.n_tiles) {  // next tile's output range, needed after the first barrier
+            nos = __ldg(prm.out_start + next);
+            noe = __ldg(prm.out_start + next + 1);
+        }
+        const bool waited = mbar_wait_bounded(bar0 + 8 * s, (k >> 1) & 1u);
+        const bool valid = oe >= os && oe <= prm.n && oe - os + 32 <= prm.mbuf_bytes &&
+                           oe - os + 16 <= prm.ebuf_bytes;  // uniform across the CTA
 
-    // scan: warp shuffles, then one warp scans the warp totals
-    uint32_t incl = cnt;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d) incl += y;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t v = lane < NWARP ? s_warp[lane] : 0u;
+        // phase 1: decode this thread's window into its word slots
+        const uint64_t w = tile * NT + tid;
+        uint32_t cnt = 0, err = 0;
+        if (valid && waited && w < prm.n_windows) {
+            uint32_t wd[NSEG + 1];
+            const uint8_t *src = slot + tid * W;
+            if constexpr (W == 8) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(src);
+                wd[0] = bswap32(v.x);
+                wd[1] = bswap32(v.y);
+            } else {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src);
+                wd[0] = bswap32(v.x);
+                wd[1] = bswap32(v.y);
+                wd[2] = bswap32(v.z);
+                wd[3] = bswap32(v.w);
+            }
+            wd[NSEG] = bswap32(*reinterpret_cast<const uint32_t *>(src + W));
+            const int p = slot[L::SBUF + tid];
+            const uint64_t rem = prm.total_bits - w * (8ull * W);
+            const int wend = rem < 8ull * W ? (int)rem : 8 * W;
+            cnt = decode_window<NSEG, NT>(wd, p, wend, s_fast, kshift, g_hier, prm.n_tables, s_priv + tid, err);
+            if (err) atomicOr(&g_status, err);
+        }
+
+        // scan: warp shuffles; the warp totals go through shared memory
+        uint32_t *scan = s_scan + (s ? 32 : 0);
+        uint32_t incl = cnt;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        if (lane == 31) scan[warp] = incl;
+        if (!__syncthreads_and(waited)) {  // a bulk copy never completed: give up
+            if (tid == 0) {
+                atomicOr(&g_status, ST_TIMEOUT);
+                mbar_wait_bounded(bar0 + 8 * s, (k >> 1) & 1u);  // let an in-flight copy land first
+            }
+            return;
+        }
+        // every thread is past the previous tile: its slot can take the next one
+        if (tid == 0 && next < prm.n_tiles) issue(next, s ^ 1u, nos, noe);
+        // each warp scans the warp totals itself
+        uint32_t v = lane < NWARP ? scan[lane] : 0u;
+#pragma unroll
+        for (int d = 1; d < NWARP; d <<= 1) {
             const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, v, d);
             if (lane >= d) v += y;
         }
-        if (lane < NWARP) s_warp[lane] = v;
-    }
-    __syncthreads();
-    const uint32_t total = s_warp[NWARP - 1];
-    const uint32_t excl = (warp ? s_warp[warp - 1] : 0u) + incl - cnt;
-    if (total != (uint32_t)(oe - os)) {
-        if (tid == 0) atomicOr(&g_status, ST_COUNT);
-        return;
-    }
-
-    // phase 2: symbols into the tile buffer; ebuf[j - (os & ~15)] holds weight j
-    const uint32_t cnt2 = walk<true, NSEG>(wd, p, wend, s_lut, g_lut, n_tables, ebuf,
-                                           (uint32_t)(os & 15u) + excl, ebuf_syms + 15u, err);
-    if (err) atomicOr(&g_status, err);
-    // both walks must agree (they can only differ if the LUT's counts contradict its lengths)
-    if (__syncthreads_or(cnt2 != cnt)) {
-        if (tid == 0) atomicOr(&g_status, ST_COUNT);
-        return;
-    }
-
-    // phase 3: bf16 assembly, 8 weights per thread per step
-    const uint64_t base = os & ~15ull;
-    const uint64_t c0 = os >> 3, c1 = (oe + 7) >> 3;
-    for (uint64_t c = c0 + tid; c < c1; c += NT) {
-        const uint64_t j0 = c << 3;
-        if (j0 >= os && j0 + 8 <= oe) {
-            const uint2 m = __ldcs(reinterpret_cast<const uint2 *>(mant + j0));
-            const uint2 e = *reinterpret_cast<const uint2 *>(ebuf + (j0 - base));
-            uint4 r;
-            join4(e.x, m.x, r.x, r.y);
-            join4(e.y, m.y, r.z, r.w);
-            __stcs(reinterpret_cast<uint4 *>(out + j0), r);
+        const uint32_t total = __shfl_sync(0xFFFFFFFFu, v, NWARP - 1);
+        const uint32_t wbase = warp ? __shfl_sync(0xFFFFFFFFu, v, (warp - 1) & 31) : 0u;
+        const uint32_t wcount = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const uint32_t excl = wbase + incl - cnt;
+        const uint32_t count = (uint32_t)(oe - os);
+        if (!valid || total != count) {  // the same decision in every warp
+            if (tid == 0) atomicOr(&g_status, valid ? ST_COUNT : ST_RANGE);
         } else {
-            const uint64_t lo = j0 > os ? j0 : os, hi = j0 + 8 < oe ? j0 + 8 : oe;
-            for (uint64_t j = lo; j < hi; ++j) out[j] = join1(ebuf[j - base], mant[j]);
+            // phase 2: word copy into the exponent buffer; eb[j - (os & ~15)] holds weight j
+            uint8_t *eb = ebuf + s * prm.ebuf_bytes;
+            const uint32_t b16 = (uint32_t)(os & 15u);
+            if (cnt) {
+                const uint32_t d = b16 + excl;
+                const uint32_t *src = s_priv + tid;
+                const uint32_t h = min((4u - (d & 3u)) & 3u, cnt);
+                uint32_t cur = src[0];
+                if (h > 0u) eb[d] = (uint8_t)cur;
+                if (h > 1u) eb[d + 1] = (uint8_t)(cur >> 8);
+                if (h > 2u) eb[d + 2] = (uint8_t)(cur >> 16);
+                const uint32_t nbody = (cnt - h) >> 2;
+                uint32_t *dst = reinterpret_cast<uint32_t *>(eb + d + h);
+                const uint32_t s8 = 8u * h;
+                for (uint32_t j = 0; j < nbody; ++j) {
+                    const uint32_t nxt = src[(j + 1) * NT];
+                    dst[j] = __funnelshift_r(cur, nxt, s8);
+                    cur = nxt;
+                }
+                const uint32_t rem = cnt - h - 4u * nbody;  // 0..3 bytes left
+                if (rem) {
+                    const uint32_t t = __funnelshift_r(cur, src[(nbody + 1) * NT], s8);
+                    uint8_t *tb = eb + d + h + 4u * nbody;
+                    tb[0] = (uint8_t)t;
+                    if (rem > 1u) tb[1] = (uint8_t)(t >> 8);
+                    if (rem > 2u) tb[2] = (uint8_t)(t >> 16);
+                }
+            }
+            __syncwarp();
+
+            // phase 3: this warp's weights, local index i <-> weight (os & ~15) + i
+            const uint8_t *mb = slot + L::SBUF + NT;
+            uint16_t *ot = prm.out + (os & ~15ull);
+            const uint32_t lo_i = b16 + wbase, hi_i = lo_i + wcount;
+            const uint32_t q0 = (lo_i + 15u) >> 4, q1 = hi_i >> 4;
+            for (uint32_t q = q0 + lane; q < q1; q += 32) {
+                const uint4 e = *reinterpret_cast<const uint4 *>(eb + 16 * q);
+                const uint4 m = *reinterpret_cast<const uint4 *>(mb + 16 * q);
+                uint4 r0, r1;
+                join4(e.x, m.x, r0.x, r0.y);
+                join4(e.y, m.y, r0.z, r0.w);
+                join4(e.z, m.z, r1.x, r1.y);
+                join4(e.w, m.w, r1.z, r1.w);
+                __stcs(reinterpret_cast<uint4 *>(ot + 16 * q), r0);
+                __stcs(reinterpret_cast<uint4 *>(ot + 16 * q + 8), r1);
+            }
+            // ragged ends of the warp's range: [lo_i, min(16 q0, hi_i)) and [max(16 q1, 16 q0), hi_i)
+            const uint32_t i = lane < 16 ? lo_i + lane : 16u * max(q1, q0) + (lane - 16);
+            const bool edge = lane < 16 ? i < min(16u * q0, hi_i) : i < hi_i;
+            if (edge) ot[i] = join1(eb[i], mb[i]);
         }
+        os = nos;
+        oe = noe;
+        tile = next;
     }
 }
 
 // One distinct exponent: every weight is (sym, raw byte).
 __global__ void fill_single(const uint8_t *__restrict__ mant, uint32_t sym, uint64_t n,
-                           uint16_t *__restrict__ out) {
+                            uint16_t *__restrict__ out) {
     const uint32_t E = sym * 0x01010101u;
     const uint64_t nfull = n >> 3;
     for (uint64_t c = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; c < nfull;
@@ -243,22 +443,38 @@ __global__ void fill_single(const uint8_t *__restrict__ mant, uint32_t sym, uint
     }
 }
 
-typedef void (*decode_fn)(const uint8_t *, const uint8_t *, const uint32_t *, uint32_t, const uint8_t *,
-                          const uint64_t *, uint64_t, uint64_t, uint64_t, uint32_t, uint16_t *);
+typedef void (*decode_fn)(const Params);
 
 struct Variant {
     uint32_t W, T;
     decode_fn fn;
-    int smem_set[16];  // dynamic shared memory opted in per device
+    int smem_set[16];  // dynamic shared memory opted in, per device
 };
 
 Variant g_variants[] = {
     {8, 128, decode_tiles<8, 128>, {0}},   {8, 256, decode_tiles<8, 256>, {0}},
     {8, 512, decode_tiles<8, 512>, {0}},   {16, 128, decode_tiles<16, 128>, {0}},
-    {16, 256, decode_tiles<16, 256>, {0}}, {16, 512, decode_tiles<16, 512>, {0}},
+    {16, 256, decode_tiles<16, 256>, {0}},
 };
 
+int g_sms[16];
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int W, int NT>
+uint32_t smem_bytes(uint32_t fb, uint32_t ebuf, uint32_t mbuf) {
+    return Layout<W, NT>(fb, ebuf, mbuf).total;
+}
+
+uint32_t variant_smem(const Variant &v, uint32_t fb, uint32_t ebuf, uint32_t mbuf) {
+    switch (v.W * 1000 + v.T) {
+        case 8128: return smem_bytes<8, 128>(fb, ebuf, mbuf);
+        case 8256: return smem_bytes<8, 256>(fb, ebuf, mbuf);
+        case 8512: return smem_bytes<8, 512>(fb, ebuf, mbuf);
+        case 16128: return smem_bytes<16, 128>(fb, ebuf, mbuf);
+        default: return smem_bytes<16, 256>(fb, ebuf, mbuf);
+    }
+}
 
 }  // namespace
 
@@ -276,37 +492,58 @@ dfw_status launch_decode(const uint8_t *d_stream, const uint8_t *d_mant, const u
     if (n == 0) return DFW_OK;
     if (!d_mant || !d_out) return DFW_EINVAL;
     if (!aligned16(d_mant) || !aligned16(d_out)) return DFW_EALIGN;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
+    if (!g_sms[dev] && cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFW_ECUDA;
     if (table->total_bits == 0) {
-        int dev = 0, sms = 148;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const uint64_t chunks = (n >> 3) + 1;
-        const uint64_t want = (chunks + 255) / 256;
-        const unsigned grid = (unsigned)(want < (uint64_t)sms * 8 ? want : (uint64_t)sms * 8);
-        fill_single<<<grid, 256, 0, s>>>(d_mant, table->single_symbol, n, d_out);
+        const uint64_t want = ((n >> 3) + 256) / 256;
+        const uint64_t cap = (uint64_t)g_sms[dev] * 8;
+        fill_single<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(d_mant, table->single_symbol, n, d_out);
         return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
     }
     if (!d_stream || !d_lut || !d_gap || !d_out_start) return DFW_EINVAL;
-    if (!aligned16(d_stream) || !aligned16(d_lut) || !aligned16(d_out_start)) return DFW_EALIGN;
-    if (info->lut_tables < 1 || info->lut_words != 256u * info->lut_tables) return DFW_EINVAL;
+    if (!aligned16(d_stream) || !aligned16(d_lut) || !aligned16(d_out_start) || !aligned16(d_gap))
+        return DFW_EALIGN;
+    const uint32_t fb = info->fast_bits;
+    if (fb < (uint32_t)FAST_BITS_MIN || fb > (uint32_t)FAST_BITS_MAX || info->lut_tables < 1 ||
+        info->lut_words != (2u << fb) + 256u * info->lut_tables)
+        return DFW_EINVAL;
     if (info->max_tile_symbols > 8ull * info->window_bytes * info->tile_windows) return DFW_EINVAL;
-    if (info->n_tiles > 0x7FFFFFFFull) return DFW_EINVAL;
+    if (table->stream_bytes & 15u) return DFW_EINVAL;
     Variant *v = nullptr;
     for (auto &x : g_variants)
         if (x.W == info->window_bytes && x.T == info->tile_windows) v = &x;
     if (!v) return DFW_EINVAL;
-    const uint32_t ebuf_bytes = (uint32_t)((info->max_tile_symbols + 16 + 15) & ~15ull);
-    const size_t smem = SMEM_HEAD + ebuf_bytes;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return DFW_ECUDA;
-    if (smem > 48 * 1024 && dev < 16 && !v->smem_set[dev]) {
-        if (cudaFuncSetAttribute(v->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) != cudaSuccess)
+    Params prm;
+    prm.stream = d_stream;
+    prm.mant = d_mant;
+    prm.lut = d_lut;
+    prm.gap = d_gap;
+    prm.out_start = d_out_start;
+    prm.out = d_out;
+    prm.total_bits = table->total_bits;
+    prm.stream_bytes = table->stream_bytes;
+    prm.n_windows = info->n_windows;
+    prm.n_tiles = info->n_tiles;
+    prm.n = n;
+    prm.fast_bits = fb;
+    prm.n_tables = info->lut_tables;
+    prm.ebuf_bytes = (uint32_t)((info->max_tile_symbols + 16 + 15) & ~15ull);
+    prm.mbuf_bytes = (uint32_t)((info->max_tile_symbols + 32 + 15) & ~15ull);
+    const uint32_t smem = variant_smem(*v, fb, prm.ebuf_bytes, prm.mbuf_bytes);
+    if (!v->smem_set[dev]) {
+        if (cudaFuncSetAttribute(v->fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
             return DFW_ECUDA;
         v->smem_set[dev] = 1;
     }
-    v->fn<<<(unsigned)info->n_tiles, v->T, smem, s>>>(d_stream, d_mant, d_lut, info->lut_tables, d_gap,
-                                                      d_out_start, table->total_bits, info->n_windows, n,
-                                                      ebuf_bytes - 16, d_out);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v->fn, (int)v->T, smem) != cudaSuccess)
+        return DFW_ECUDA;
+    if (per_sm < 1) return DFW_EINVAL;
+    const uint64_t slots = (uint64_t)per_sm * g_sms[dev];
+    const unsigned grid = (unsigned)(info->n_tiles < slots ? info->n_tiles : slots);
+    v->fn<<<grid, v->T, smem, s>>>(prm);
     return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
 }
 

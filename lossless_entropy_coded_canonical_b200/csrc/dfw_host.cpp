@@ -325,8 +325,58 @@ dfw_status build_lut(const dfw_table *table, std::vector<uint32_t> &lut) {
     return DFW_OK;
 }
 
+// One codeword from the hierarchy: x holds the next 32 bits, left-aligned.
+// Returns false if the tables do not resolve it within four levels.
+static bool hier_decode(const std::vector<uint32_t> &lut, uint32_t x, int &sym, int &len) {
+    size_t tab = 0;
+    for (int level = 0; level < 4; ++level) {
+        const uint32_t e = lut[tab * 256 + ((x >> (24 - 8 * level)) & 0xFF)];
+        if (!(e & LUT_PTR)) {
+            sym = (int)(e & 0xFF);
+            len = (int)((e >> LUT_LEN_SHIFT) & 63);
+            return len > 0;
+        }
+        tab = e & LUT_CHILD_MASK;
+        if (tab * 256 >= lut.size()) return false;
+    }
+    return false;
+}
+
+// Fast table: for every K-bit key, the whole codewords (at most four) that
+// start at the key's first bit and end within its K bits.
+dfw_status build_fast(const std::vector<uint32_t> &lut, int fast_bits, std::vector<uint32_t> &fast) {
+    if (fast_bits < FAST_BITS_MIN || fast_bits > FAST_BITS_MAX) return DFW_EINVAL;
+    const uint32_t entries = 1u << fast_bits;
+    fast.assign(2 * (size_t)entries, 0);
+    for (uint32_t key = 0; key < entries; ++key) {
+        const uint32_t x = key << (32 - fast_bits);
+        int pos = 0, cnt = 0;
+        uint32_t syms = 0, ends = 0;
+        while (cnt < FAST_MAX_SYMS) {
+            int sym = 0, len = 0;
+            if (!hier_decode(lut, x << pos, sym, len)) break;
+            if (pos + len > fast_bits) break;
+            syms |= (uint32_t)sym << (8 * cnt);
+            pos += len;
+            ends |= 1u << (pos - 1);
+            ++cnt;
+            if (pos == 32) break;
+        }
+        if (cnt == 0) {
+            fast[2 * key] = 0;
+            fast[2 * key + 1] = FAST_ESC_WORD;
+        } else {
+            fast[2 * key] = syms;
+            fast[2 * key + 1] = (uint32_t)pos | ((uint32_t)(8 * cnt) << FAST_C8_SHIFT) | (ends << FAST_ENDS_SHIFT);
+        }
+    }
+    return DFW_OK;
+}
+
+// W * T <= 4096 keeps a tile's worst case (one codeword per stream bit) within
+// shared memory: about 174 KB with a 12-bit fast table.
 bool plan_shape_supported(uint32_t W, uint32_t T) {
-    return (W == 8 || W == 16) && (T == 128 || T == 256 || T == 512);
+    return (W == 8 || W == 16) && (T == 128 || T == 256 || T == 512) && W * T <= 4096;
 }
 
 }  // namespace dfw
@@ -386,7 +436,10 @@ extern "C" dfw_status dfw_plan_query(const dfw_table *table, uint32_t window_byt
     if (!info || !plan_shape_supported(window_bytes, tile_windows)) return DFW_EINVAL;
     dfw_status st = validate_table(table);
     if (st != DFW_OK) return st;
+    const uint32_t fb = info->fast_bits ? info->fast_bits : (uint32_t)FAST_BITS_DEFAULT;
+    if (fb < (uint32_t)FAST_BITS_MIN || fb > (uint32_t)FAST_BITS_MAX) return DFW_EINVAL;
     std::memset(info, 0, sizeof(*info));
+    info->fast_bits = fb;
     info->window_bytes = window_bytes;
     info->tile_windows = tile_windows;
     const uint64_t wbits = 8ull * window_bytes;
@@ -395,8 +448,8 @@ extern "C" dfw_status dfw_plan_query(const dfw_table *table, uint32_t window_byt
     std::vector<uint32_t> lut;
     st = build_lut(table, lut);
     if (st != DFW_OK) return st;
-    info->lut_words = (uint32_t)lut.size();
     info->lut_tables = (uint32_t)(lut.size() / 256);
+    info->lut_words = (2u << fb) + (uint32_t)lut.size();
     return DFW_OK;
 }
 
@@ -404,14 +457,18 @@ extern "C" dfw_status dfw_plan(const uint8_t *stream, const dfw_table *table, ui
                                uint64_t *out_start, uint32_t *lut, dfw_plan_info *info) {
     if (!info || !out_start || !lut) return DFW_EINVAL;
     dfw_plan_info q;
+    q.fast_bits = info->fast_bits;
     dfw_status st = dfw_plan_query(table, info->window_bytes, info->tile_windows, &q);
     if (st != DFW_OK) return st;
     if (q.n_windows != info->n_windows || q.n_tiles != info->n_tiles || q.lut_words != info->lut_words)
         return DFW_EINVAL;
     if (q.n_windows && (!gap || !stream)) return DFW_EINVAL;
-    std::vector<uint32_t> img;
+    std::vector<uint32_t> img, fast;
     build_lut(table, img);
-    std::memcpy(lut, img.data(), img.size() * sizeof(uint32_t));
+    st = build_fast(img, (int)q.fast_bits, fast);
+    if (st != DFW_OK) return st;
+    std::memcpy(lut, fast.data(), fast.size() * sizeof(uint32_t));
+    std::memcpy(lut + fast.size(), img.data(), img.size() * sizeof(uint32_t));
     const uint64_t n = table->n, tb = table->total_bits;
     const uint64_t wbits = 8ull * q.window_bytes, tbits = wbits * q.tile_windows;
     if (tb == 0) {
@@ -471,6 +528,7 @@ extern "C" dfw_status dfw_plan(const uint8_t *stream, const dfw_table *table, ui
         if (g >= 32) return DFW_ECORRUPT;
         gap[t_next++] = (uint8_t)g;
     }
+    std::memset(gap + nwin, 0, (size_t)(q.n_tiles * q.tile_windows - nwin));  // pad to whole tiles
     while (b_next < ntiles) out_start[b_next++] = n;
     out_start[ntiles] = n;
     uint64_t mx = 0;

@@ -18,16 +18,33 @@ constexpr int LUT_LEN_SHIFT = 8;
 constexpr int LUT_CNT_SHIFT = 14;
 constexpr int LUT_CBITS_SHIFT = 18;
 
+// Fast table: 2^K entries of two u32 words.  Word 0: the symbols of up to
+// four whole codewords inside the K key bits (first in the low byte, absent
+// ones zero).  Word 1: byte 0 = bits those codewords use, byte 1 = 8 * their
+// count, bits 16..27 = end mask (bit j-1 set when one of them ends at key
+// offset j), bit 31 = escape (first codeword longer than K bits; its bits
+// byte is 255 so any bounds test sends it to the slow path).
+constexpr int FAST_BITS_DEFAULT = 10;
+constexpr int FAST_BITS_MIN = 8;
+constexpr int FAST_BITS_MAX = 12;
+constexpr int FAST_MAX_SYMS = 4;
+constexpr int FAST_C8_SHIFT = 8;
+constexpr int FAST_ENDS_SHIFT = 16;
+constexpr uint32_t FAST_ESC = 0x80000000u;
+constexpr uint32_t FAST_ESC_WORD = FAST_ESC | 255u;
+
 // Bits of the device status word.
 constexpr uint32_t ST_COUNT = 1u;   // a tile decoded a different number of codes than out_start says
 constexpr uint32_t ST_LUT = 2u;     // a LUT pointer left the table or a code ran past four levels
 constexpr uint32_t ST_RANGE = 4u;   // out_start out of order or beyond n, or tile too large
+constexpr uint32_t ST_TIMEOUT = 8u; // a wait for a bulk copy gave up (the kernel returned early)
 
 dfw_status code_lengths(const uint64_t hist[256], int cap, uint8_t len[256]);
 void canonical_codes(const uint8_t len[256], uint32_t code[256]);
 bool kraft_complete(const uint8_t len[256], int cap);
 uint64_t stream_bytes_for(uint64_t total_bits);
 dfw_status build_lut(const dfw_table *table, std::vector<uint32_t> &lut);
+dfw_status build_fast(const std::vector<uint32_t> &lut, int fast_bits, std::vector<uint32_t> &fast);
 bool plan_shape_supported(uint32_t W, uint32_t T);
 dfw_status validate_table(const dfw_table *t);
 

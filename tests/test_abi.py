@@ -44,4 +44,4 @@ def test_strerror_covers_every_status():
 def test_struct_layouts_match_header():
     import ctypes
     assert ctypes.sizeof(dfw.Table) == 4 + 4 + 8 + 8 + 8 + 4 + 4 + 256
-    assert ctypes.sizeof(dfw.PlanInfo) == 4 + 4 + 8 + 8 + 8 + 4 + 4
+    assert ctypes.sizeof(dfw.PlanInfo) == 4 + 4 + 8 + 8 + 8 + 4 + 4 + 4 + 4

@@ -17,7 +17,7 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 BENCH_SHAPE = (8, 256)
-SHAPES = [(8, 128), (8, 256), (8, 512), (16, 128), (16, 256), (16, 512)]
+SHAPES = [(8, 128), (8, 256), (8, 512), (16, 128), (16, 256)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -116,7 +116,7 @@ def test_cap_binding_tables(oracle, cap):
     with caps that bind, so every LUT level is exercised."""
     u = _u16(workloads.c4("b", 1_500_001))
     oracle_parity(oracle, u, 8, 256, cap)
-    oracle_parity(oracle, u, 16, 512, cap)
+    oracle_parity(oracle, u, 16, 256, cap)
 
 
 def test_codes_straddle_tiles(oracle):

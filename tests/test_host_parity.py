@@ -108,14 +108,16 @@ def test_encode_multi_with_empty_tensor(oracle):
 
 
 @pytest.mark.parametrize("name", ["c1", "c2", "c4a", "c4b", "c4c", "tiny", "single"])
-@pytest.mark.parametrize("W,T", [(8, 128), (8, 256), (16, 256), (16, 512)])
+@pytest.mark.parametrize("W,T", [(8, 128), (8, 256), (8, 512), (16, 256)])
 def test_plan_matches_oracle(oracle, name, W, T):
     u = CASES[name]()
     enc = dfw.encode(u, 32, n_threads=2)
     oenc = oracle.encode(u, 32)
     pl = dfw.plan(enc, W, T)
     gap, out_start = oracle.aux(oenc, W, T)
-    assert np.array_equal(pl.gap.numpy(), gap)
+    assert pl.gap.numel() == pl.info.n_tiles * T
+    assert np.array_equal(pl.gap.numpy()[: gap.size], gap)
+    assert not pl.gap.numpy()[gap.size:].any()
     assert np.array_equal(pl.out_start.numpy().view(np.uint64), out_start)
     st = out_start.astype(np.int64)
     mx = int(np.max(np.diff(st))) if st.size > 1 else 0
@@ -125,7 +127,7 @@ def test_plan_matches_oracle(oracle, name, W, T):
 
 def test_plan_rejects_bad_shapes():
     enc = dfw.encode(CASES["c1"](), 32)
-    for W, T in ((4, 256), (8, 100), (32, 256), (8, 1024)):
+    for W, T in ((4, 256), (8, 100), (32, 256), (8, 1024), (16, 512)):
         with pytest.raises(dfw.DfwError) as ei:
             dfw.plan(enc, W, T)
         assert ei.value.status == dfw.EINVAL
@@ -169,35 +171,98 @@ def _lut_walk(lut, stream_u8, total_bits):
     return syms
 
 
-@pytest.mark.parametrize("name", ["c1", "c4b", "c4c", "tiny"])
-def test_lut_image_decodes_like_oracle(oracle, name):
-    u = CASES[name]()[:40_000]
+def _split_lut(pl):
+    img = pl.lut.numpy().view(np.uint32)
+    nf = 1 << pl.info.fast_bits
+    assert pl.info.lut_words == img.size == 2 * nf + 256 * pl.info.lut_tables
+    return img[: 2 * nf].reshape(nf, 2), img[2 * nf:]
+
+
+def _fast_window_walk(fast, hier, K, stream_u8, total_bits, W):
+    """Emulates the device's phase 1 on every window: fast lookups of K bits,
+    escapes through the byte hierarchy, and the window-end rule (a lookup that
+    crosses the end keeps only codewords starting before it).  Returns the
+    per-window symbol lists."""
+    bits = np.concatenate([np.unpackbits(stream_u8), np.zeros(64, np.uint8)])
+    wbits = 8 * W
+    nwin = -(-total_bits // wbits)
+    out = []
+    # first codeword start per window, by a plain walk with the hierarchy
+    starts, pos = [], 0
+
+    def hier_one(pos):
+        tab, level = 0, 0
+        while True:
+            key = int(np.packbits(bits[pos + 8 * level: pos + 8 * level + 8])[0])
+            e = int(hier[tab * 256 + key])
+            if e & 0x80000000:
+                tab, level = e & 0x3FFF, level + 1
+                continue
+            return e & 0xFF, (e >> 8) & 63
+
+    while pos < total_bits:
+        starts.append(pos)
+        pos += hier_one(pos)[1]
+    starts = np.array(starts)
+    for t in range(nwin):
+        lo = wbits * t
+        wend = min(wbits, total_bits - lo)
+        after = starts[starts >= lo]
+        p = int(after[0]) - lo if after.size else wend
+        syms = []
+        while p < wend:
+            key = int(np.packbits(np.concatenate([bits[lo + p: lo + p + K], np.zeros(16 - K, np.uint8)])).view(">u2")[0]) >> (16 - K)
+            e0, e1 = int(fast[key, 0]), int(fast[key, 1])
+            if e1 & 0x80000000:
+                s_, l_ = hier_one(lo + p)
+                syms.append(s_)
+                p += l_
+                continue
+            c = ((e1 >> 8) & 255) // 8
+            cb = e1 & 255
+            ends = (e1 >> 16) & 0xFFF
+            take = c
+            if p + cb > wend:
+                r = wend - p
+                take = min(c, 1 + bin(ends & ((1 << (r - 1)) - 1)).count("1"))
+            syms += [(e0 >> (8 * i)) & 0xFF for i in range(take)]
+            p += cb
+        out.append(syms)
+    return out
+
+
+@pytest.mark.parametrize("name", ["c1", "c4a", "c4b", "c4c", "tiny"])
+@pytest.mark.parametrize("K", [8, 11, 12])
+def test_lut_image_decodes_like_oracle(oracle, name, K):
+    u = CASES[name]()[:20_000]
     enc = dfw.encode(u, 32 if name != "c4b" else 14)
-    pl = dfw.plan(enc)
-    lut = pl.lut.numpy().view(np.uint32)
-    assert pl.info.lut_words == lut.size == 256 * pl.info.lut_tables
-    syms = _lut_walk(lut, enc.stream.numpy(), enc.total_bits)
+    pl = dfw.plan(enc, 8, 128, fast_bits=K)
+    assert pl.info.fast_bits == K
+    fast, hier = _split_lut(pl)
+    # the hierarchy alone decodes the stream
+    syms = _lut_walk(hier, enc.stream.numpy(), enc.total_bits)
     e, _ = oracle.split(u)
     assert syms == list(e)
-    # table 0: whole-codeword count and their bits within the 8 key bits
-    ln = enc.lengths
-    codes = oracle.canonical_codes(ln)
-    words = {(int(ln[s]), int(codes[s])): s for s in range(256) if ln[s]}
-    for key in range(256):
-        ent = int(lut[key])
-        if ent & 0x80000000:
-            assert (ent >> 14) & 0xFF == 0
+    # every fast entry satisfies what the kernel checks before use
+    for key in range(1 << K):
+        e0, e1 = int(fast[key, 0]), int(fast[key, 1])
+        if e1 & 0x80000000:
+            assert e1 == 0x80000000 | 255 and e0 == 0
             continue
-        pos, cnt = 0, 0
-        while True:
-            for l in range(1, 9 - pos):
-                if (l, (key >> (8 - pos - l)) & ((1 << l) - 1)) in words:
-                    pos += l
-                    cnt += 1
-                    break
-            else:
-                break
-        assert ((ent >> 14) & 15, (ent >> 18) & 15) == (cnt, pos)
+        cb, c8, ends = e1 & 255, (e1 >> 8) & 255, (e1 >> 16) & 0xFFF
+        assert c8 in (8, 16, 24, 32) and 1 <= cb <= K and 8 * cb >= c8
+        assert bin(ends).count("1") * 8 == c8 and ends >> (cb - 1) == 1
+        assert (e1 >> 28) & 7 == 0
+        assert e0 >> c8 == 0 if c8 < 32 else True
+    # the per-window walk the kernel performs gives the oracle's symbols in order
+    W = 8
+    wins = _fast_window_walk(fast, hier, K, enc.stream.numpy(), enc.total_bits, W)
+    flat = [s for w in wins for s in w]
+    assert flat == list(e)
+    gap, out_start = oracle.aux(oracle.encode(u, 32 if name != "c4b" else 14), W, 128)
+    counts = np.array([len(w) for w in wins])
+    assert np.array_equal(np.concatenate([[0], np.cumsum(counts)])[::128][: out_start.size - 1],
+                          out_start[:-1].astype(np.int64))
 
 
 def test_plan_tables_for_cap_binding_case(oracle):
@@ -227,10 +292,13 @@ def test_plan_tables_for_cap_binding_case(oracle):
     enc = dfw.Encoded(torch.from_numpy(stream), torch.zeros((e.size + 15) // 16 * 16, dtype=torch.uint8), t)
     pl = dfw.plan(enc, 8, 256)
     assert pl.info.lut_tables > 4
-    assert _lut_walk(pl.lut.numpy().view(np.uint32), stream, t.total_bits) == list(e)
+    fast, hier = _split_lut(pl)
+    assert _lut_walk(hier, stream, t.total_bits) == list(e)
+    wins = _fast_window_walk(fast, hier, pl.info.fast_bits, stream, t.total_bits, 8)
+    assert [s for w in wins for s in w] == list(e)
     oenc = oracle.Encoded(stream, np.zeros(e.size, np.uint8), ln, t.total_bits, e.size, -1)
     gap, out_start = oracle.aux(oenc, 8, 256)
-    assert np.array_equal(pl.gap.numpy(), gap)
+    assert np.array_equal(pl.gap.numpy()[: gap.size], gap)
     assert np.array_equal(pl.out_start.numpy().view(np.uint64), out_start)
 
 
