@@ -19,13 +19,15 @@
 //   scan     warp shuffle scan of the counts; one CTA barrier publishes the
 //            warp totals, and every warp scans those itself (no second
 //            barrier); the tile total must equal out_start[b+1] - out_start[b]
-//   phase 2  each thread copies its symbols a word at a time (funnel shift to
-//            the destination's byte alignment) into the tile's exponent buffer
-//   phase 3  each warp assembles bf16 for its own output range from the
-//            exponent buffer and the raw bytes already in shared memory, 16
-//            weights per thread-step, 128-bit coalesced stores, ragged ends
-//            element by element; warps need no barrier between phases 2 and 3
-//            (the exponent buffer alternates between two copies by tile)
+//   phase 2  each thread joins its symbols with their raw bytes (both read a
+//            word at a time, funnel-shifted to the output's alignment) into
+//            bf16 in a shared staging buffer in output order
+//   store    each warp bulk-stores its output range from the staging buffer
+//            with one TMA store (cp.async.bulk shared -> global); the <= 7
+//            weights at either unaligned end are stored one by one.  Before
+//            the next tile writes the staging buffer, each warp waits until
+//            its store has read it (bulk wait_group.read), then the CTA
+//            barrier orders all warps.
 //
 // Bounds: every lookup advances at least one bit and a walk stops at its
 // window end, so loops end whatever the data; tables are validated once per
@@ -76,6 +78,19 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
                  "l"(src), "r"(bytes), "r"(bar)
                  : "memory");
 }
+
+// 1-D bulk copy this CTA's shared memory -> global, tracked in a bulk group.
+__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+
+// Waits until this thread's bulk stores have read their shared memory.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Waits until this thread's bulk stores have completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
@@ -205,12 +220,12 @@ struct Params {
     uint16_t *out;
     uint64_t total_bits, stream_bytes, n_windows, n_tiles, n;
     uint32_t fast_bits, n_tables;
-    uint32_t ebuf_bytes;  // tile exponent buffer (>= max tile symbols + 16)
+    uint32_t ebuf_bytes;  // staging entries (>= max tile symbols + 16); 2 bytes each
     uint32_t mbuf_bytes;  // raw-byte buffer per slot (>= max tile symbols + 32)
 };
 
 // Shared memory: fast table | scan slots | 2 mbarriers | word slots |
-// 2 exponent buffers | 2 x (stream bytes | gap bytes | raw bytes).
+// bf16 staging | 2 x (stream bytes | gap bytes | raw bytes).
 template <int W, int NT>
 struct Layout {
     static constexpr uint32_t PRIV_WORDS = 2 * W + 1;  // 8W + 4 bytes: a window's worst case
@@ -222,7 +237,7 @@ struct Layout {
         mbar = scan + 64 * 4;
         priv = mbar + 16;
         ebuf = priv + 4 * PRIV_WORDS * NT;
-        slot0 = ebuf + 2 * ebuf_bytes;
+        slot0 = ebuf + 2 * ebuf_bytes;  // staging: 2 bytes per tile-buffer entry
         slot_bytes = SBUF + NT + mbuf_bytes;
         total = slot0 + 2 * slot_bytes;
     }
@@ -306,6 +321,7 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
             noe = __ldg(prm.out_start + next + 1);
         }
         const bool waited = mbar_wait_bounded(bar0 + 8 * s, (k >> 1) & 1u);
+        if (lane == 0) bulk_wait_read();  // this warp's last store has read the staging buffer
         const bool valid = oe >= os && oe <= prm.n && oe - os + 32 <= prm.mbuf_bytes &&
                            oe - os + 16 <= prm.ebuf_bytes;  // uniform across the CTA
 
@@ -348,6 +364,7 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
                 atomicOr(&g_status, ST_TIMEOUT);
                 mbar_wait_bounded(bar0 + 8 * s, (k >> 1) & 1u);  // let an in-flight copy land first
             }
+            if (lane == 0) bulk_wait_all();
             return;
         }
         // every thread is past the previous tile: its slot can take the next one
@@ -367,61 +384,56 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
         if (!valid || total != count) {  // the same decision in every warp
             if (tid == 0) atomicOr(&g_status, valid ? ST_COUNT : ST_RANGE);
         } else {
-            // phase 2: word copy into the exponent buffer; eb[j - (os & ~15)] holds weight j
-            uint8_t *eb = ebuf + s * prm.ebuf_bytes;
+            // phase 2: join into the staging buffer; st[i] holds weight (os & ~15) + i
+            uint16_t *st = reinterpret_cast<uint16_t *>(ebuf);
+            const uint8_t *mb = slot + L::SBUF + NT;
             const uint32_t b16 = (uint32_t)(os & 15u);
             if (cnt) {
                 const uint32_t d = b16 + excl;
                 const uint32_t *src = s_priv + tid;
                 const uint32_t h = min((4u - (d & 3u)) & 3u, cnt);
                 uint32_t cur = src[0];
-                if (h > 0u) eb[d] = (uint8_t)cur;
-                if (h > 1u) eb[d + 1] = (uint8_t)(cur >> 8);
-                if (h > 2u) eb[d + 2] = (uint8_t)(cur >> 16);
+                for (uint32_t i = 0; i < h; ++i) st[d + i] = join1((cur >> (8u * i)) & 0xFFu, mb[d + i]);
                 const uint32_t nbody = (cnt - h) >> 2;
-                uint32_t *dst = reinterpret_cast<uint32_t *>(eb + d + h);
                 const uint32_t s8 = 8u * h;
+                const uint32_t q0 = d + h;  // multiple of 4
                 for (uint32_t j = 0; j < nbody; ++j) {
                     const uint32_t nxt = src[(j + 1) * NT];
-                    dst[j] = __funnelshift_r(cur, nxt, s8);
+                    const uint32_t E = __funnelshift_r(cur, nxt, s8);
+                    const uint32_t M = *reinterpret_cast<const uint32_t *>(mb + q0 + 4u * j);
+                    uint2 r;
+                    join4(E, M, r.x, r.y);
+                    *reinterpret_cast<uint2 *>(st + q0 + 4u * j) = r;
                     cur = nxt;
                 }
-                const uint32_t rem = cnt - h - 4u * nbody;  // 0..3 bytes left
+                const uint32_t rem = cnt - h - 4u * nbody;  // 0..3 weights left
                 if (rem) {
                     const uint32_t t = __funnelshift_r(cur, src[(nbody + 1) * NT], s8);
-                    uint8_t *tb = eb + d + h + 4u * nbody;
-                    tb[0] = (uint8_t)t;
-                    if (rem > 1u) tb[1] = (uint8_t)(t >> 8);
-                    if (rem > 2u) tb[2] = (uint8_t)(t >> 16);
+                    const uint32_t i0 = q0 + 4u * nbody;
+                    for (uint32_t i = 0; i < rem; ++i) st[i0 + i] = join1((t >> (8u * i)) & 0xFFu, mb[i0 + i]);
                 }
             }
+            fence_proxy_async();  // these writes before the warp's bulk store reads them
             __syncwarp();
 
-            // phase 3: this warp's weights, local index i <-> weight (os & ~15) + i
-            const uint8_t *mb = slot + L::SBUF + NT;
+            // store: the warp's range [lo_i, hi_i) of local indices; ot[i] is weight (os & ~15) + i
             uint16_t *ot = prm.out + (os & ~15ull);
             const uint32_t lo_i = b16 + wbase, hi_i = lo_i + wcount;
-            const uint32_t q0 = (lo_i + 15u) >> 4, q1 = hi_i >> 4;
-            for (uint32_t q = q0 + lane; q < q1; q += 32) {
-                const uint4 e = *reinterpret_cast<const uint4 *>(eb + 16 * q);
-                const uint4 m = *reinterpret_cast<const uint4 *>(mb + 16 * q);
-                uint4 r0, r1;
-                join4(e.x, m.x, r0.x, r0.y);
-                join4(e.y, m.y, r0.z, r0.w);
-                join4(e.z, m.z, r1.x, r1.y);
-                join4(e.w, m.w, r1.z, r1.w);
-                __stcs(reinterpret_cast<uint4 *>(ot + 16 * q), r0);
-                __stcs(reinterpret_cast<uint4 *>(ot + 16 * q + 8), r1);
+            const uint32_t A = (lo_i + 7u) & ~7u, B = hi_i & ~7u;  // 16-byte aligned interior
+            if (lane == 0 && B > A) bulk_store(ot + A, smem_u32(st + A), 2u * (B - A));
+            if (lane < 8) {
+                const uint32_t i = lo_i + lane;
+                if (i < min(A, hi_i)) ot[i] = st[i];
+            } else if (lane < 16) {
+                const uint32_t i = max(B, A) + (lane - 8);
+                if (i < hi_i) ot[i] = st[i];
             }
-            // ragged ends of the warp's range: [lo_i, min(16 q0, hi_i)) and [max(16 q1, 16 q0), hi_i)
-            const uint32_t i = lane < 16 ? lo_i + lane : 16u * max(q1, q0) + (lane - 16);
-            const bool edge = lane < 16 ? i < min(16u * q0, hi_i) : i < hi_i;
-            if (edge) ot[i] = join1(eb[i], mb[i]);
         }
         os = nos;
         oe = noe;
         tile = next;
     }
+    if (lane == 0) bulk_wait_all();
 }
 
 // One distinct exponent: every weight is (sym, raw byte).
