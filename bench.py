@@ -157,7 +157,7 @@ def barrier():
 
 # ------------------------------------------------------------------ setup
 
-def prepare(blocks, device, window, tile, threads):
+def prepare(blocks, device, window, tile, threads, variant="window"):
     """Generates each block on the GPU, encodes and plans it on the host,
     uploads it; returns the device-resident blocks and host copies (pinned)."""
     import lossless_entropy_coded_canonical_b200 as dfw
@@ -167,7 +167,7 @@ def prepare(blocks, device, window, tile, threads):
 
     def host_side(i, tensors):
         enc = dfw.encode_multi(tensors, 32, n_threads=enc_threads, pin=True)
-        pl = dfw.plan(enc, window, tile, pin=True)
+        pl = dfw.plan_lanes(enc, pin=True) if variant == "lanes" else dfw.plan(enc, window, tile, pin=True)
         return i, enc, pl
 
     futs = []
@@ -181,21 +181,33 @@ def prepare(blocks, device, window, tile, threads):
         i, enc, pl = f.result()
         res[i] = (enc, pl)
     pool.shutdown()
-    devs = [dfw.DeviceCompressed.upload(enc, pl, device) for enc, pl in res]
+    up = dfw.DeviceLanes.upload if variant == "lanes" else dfw.DeviceCompressed.upload
+    devs = [up(enc, pl, device) for enc, pl in res]
     torch.cuda.synchronize(device)
     torch.cuda.empty_cache()  # drop the generator's temporaries before timing
     return devs, res
+
+
+def decode_one(d, scratch, stream=None):
+    """One decode launch of a block into the scratch buffer (either plan)."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    if isinstance(d, dfw.DeviceLanes):
+        dfw.decode_lanes(d, scratch, stream=stream)
+    else:
+        dfw.decode_block(d, scratch, stream=stream)
 
 
 def verify(blocks, devs, scratch, device):
     """Decodes each block once more and compares with the regenerated input."""
     import lossless_entropy_coded_canonical_b200 as dfw
     for b, d in zip(blocks, devs):
-        _, views = dfw.decode_block(d, scratch)
+        decode_one(d, scratch)
         dfw.check()
-        for v, t in zip(views, workloads.generate_block(b, device)):
-            if not torch.equal(v.view(torch.int16), t.view(torch.int16)):
+        off = 0
+        for t in workloads.generate_block(b, device):
+            if not torch.equal(scratch[off: off + t.numel()].view(torch.int16), t.view(torch.int16)):
                 return False
+            off += t.numel()
     return True
 
 
@@ -205,7 +217,7 @@ def run_device(devs, scratch, steps, warmup, stream):
     import lossless_entropy_coded_canonical_b200 as dfw
     for _ in range(warmup):
         for d in devs:
-            dfw.decode_block(d, scratch, stream=stream)
+            decode_one(d, scratch, stream)
     dfw.check(stream)
     ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in devs]
           for _ in range(steps)]
@@ -216,7 +228,7 @@ def run_device(devs, scratch, steps, warmup, stream):
     for s in range(steps):
         for j, d in enumerate(devs):
             ev[s][j][0].record(stream)
-            dfw.decode_block(d, scratch, stream=stream)
+            decode_one(d, scratch, stream)
             ev[s][j][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -233,21 +245,22 @@ def run_e2e(results, devs, device, steps, stream):
     on their own streams, double-buffered so they overlap the decode."""
     import lossless_entropy_coded_canonical_b200 as dfw
     nmax = max(d.n for d in devs)
+    lanes = isinstance(results[0][1], dfw.LanesPlan)
+    aux_names = ("chunk_bits", "group_start", "lut") if lanes else ("gap", "out_start", "lut")
     h2d_s, d2h_s = torch.cuda.Stream(device), torch.cuda.Stream(device)
     slots = []
     for _ in range(2):
-        slots.append({
-            "stream": torch.empty(max(int(e.table.stream_bytes) for e, _ in results), dtype=torch.uint8, device=device),
-            "mant": torch.empty(max(e.mant.numel() for e, _ in results), dtype=torch.uint8, device=device),
-            "gap": torch.empty(max(p.gap.numel() for _, p in results) + 1, dtype=torch.uint8, device=device),
-            "out_start": torch.empty(max(p.out_start.numel() for _, p in results), dtype=torch.int64, device=device),
-            "lut": torch.empty(max(p.lut.numel() for _, p in results), dtype=torch.int32, device=device),
-            "scratch": torch.empty(nmax, dtype=torch.bfloat16, device=device),
-            "host_out": torch.empty(nmax, dtype=torch.bfloat16, pin_memory=True),
-            "loaded": torch.cuda.Event(), "decoded": torch.cuda.Event(), "drained": torch.cuda.Event(),
-        })
-    h2d = sum(int(e.table.stream_bytes) + e.mant.numel() + p.gap.numel() + 8 * p.out_start.numel()
-              + 4 * p.lut.numel() for e, p in results)
+        sl = {"stream": torch.empty(max(int(e.table.stream_bytes) for e, _ in results), dtype=torch.uint8, device=device),
+              "mant": torch.empty(max(e.mant.numel() for e, _ in results), dtype=torch.uint8, device=device),
+              "scratch": torch.empty(nmax, dtype=torch.bfloat16, device=device),
+              "host_out": torch.empty(nmax, dtype=torch.bfloat16, pin_memory=True),
+              "loaded": torch.cuda.Event(), "decoded": torch.cuda.Event(), "drained": torch.cuda.Event()}
+        for a in aux_names:
+            t0 = getattr(results[0][1], a)
+            sl[a] = torch.empty(max(getattr(p, a).numel() for _, p in results), dtype=t0.dtype, device=device)
+        slots.append(sl)
+    h2d = sum(int(e.table.stream_bytes) + e.mant.numel() + sum(getattr(p, a).numel() * getattr(p, a).element_size()
+                                                                for a in aux_names) for e, p in results)
     d2h = sum(2 * e.n for e, _ in results)
 
     def one_step():
@@ -260,15 +273,19 @@ def run_e2e(results, devs, device, steps, stream):
             with torch.cuda.stream(h2d_s):
                 sl["stream"][: enc.stream.numel()].copy_(enc.stream, non_blocking=True)
                 sl["mant"][: enc.mant.numel()].copy_(enc.mant, non_blocking=True)
-                sl["gap"][: pl.gap.numel()].copy_(pl.gap, non_blocking=True)
-                sl["out_start"][: pl.out_start.numel()].copy_(pl.out_start, non_blocking=True)
-                sl["lut"][: pl.lut.numel()].copy_(pl.lut, non_blocking=True)
+                for a in aux_names:
+                    src = getattr(pl, a)
+                    sl[a][: src.numel()].copy_(src, non_blocking=True)
                 sl["loaded"].record(h2d_s)
             stream.wait_event(sl["loaded"])
             stream.wait_event(sl["drained"])
-            dc = dfw.DeviceCompressed(sl["stream"], sl["mant"], sl["lut"], sl["gap"], sl["out_start"], enc.table,
-                                      pl.info, enc.tensor_offsets)
-            dfw.decode_block(dc, sl["scratch"], stream=stream)
+            if lanes:
+                dc = dfw.DeviceLanes(sl["stream"], sl["mant"], sl["lut"], sl["chunk_bits"], sl["group_start"],
+                                     enc.table, pl.info, enc.tensor_offsets)
+            else:
+                dc = dfw.DeviceCompressed(sl["stream"], sl["mant"], sl["lut"], sl["gap"], sl["out_start"], enc.table,
+                                          pl.info, enc.tensor_offsets)
+            decode_one(dc, sl["scratch"], stream)
             sl["decoded"].record(stream)
             d2h_s.wait_event(sl["decoded"])
             with torch.cuda.stream(d2h_s):
@@ -327,6 +344,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="c5")
     ap.add_argument("--window", type=int, default=8)
     ap.add_argument("--tile", type=int, default=256)
+    ap.add_argument("--variant", default="window", choices=["window", "lanes"],
+                    help="window: gap/out_start plan (count phase + scan); lanes: known-start chunks")
     ap.add_argument("--threads", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
@@ -356,7 +375,7 @@ def main(argv=None):
     dfw.lib()
     dfw.check()
 
-    devs, results = prepare(blocks, device, args.window, args.tile, args.threads)
+    devs, results = prepare(blocks, device, args.window, args.tile, args.threads, args.variant)
     nmax = max(d.n for d in devs)
     scratch = torch.empty(nmax, dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream(device)
@@ -400,8 +419,9 @@ def main(argv=None):
         "metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
-        "config": {"workload": wdesc, "weights": n_total, "code_tables": len(devs),
-                   "window_bytes": args.window, "tile_windows": args.tile,
+        "config": {"workload": wdesc, "weights": n_total, "code_tables": len(devs), "plan": args.variant,
+                   "window_bytes": args.window if args.variant == "window" else None,
+                   "tile_windows": args.tile if args.variant == "window" else None,
                    "l2": "inputs larger than L2 (each step reads every block's compressed form and writes "
                          "every block's bf16; no reuse between steps)",
                    "parallelism": f"replica{world}" if world > 1 else "single GPU"},
@@ -410,7 +430,8 @@ def main(argv=None):
         "bits_per_weight": 8 * comp / n_total,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "decode_tiles", "algorithmic_bytes_per_step": alg_bytes,
+                     "kernel": "decode_lanes" if args.variant == "lanes" else "decode_tiles",
+                     "algorithmic_bytes_per_step": alg_bytes,
                      "mean_launch_ms": float(mean_launch_ms.mean())},
         "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": args.steps * len(devs),
         "verified_bit_exact": bool(ok),

@@ -216,6 +216,56 @@ dfw_status dfw_decode_block(const uint8_t *d_stream, const uint8_t *d_mant, cons
  */
 dfw_status dfw_check(void *cuda_stream);
 
+/*
+ * KNOWN-START CHUNKS (a second decode plan over the same stream; the
+ * "interleaved lanes" design of the LazyWeights write-up, Verified Facts
+ * and body, realised with per-chunk bit offsets instead of separate lane
+ * streams).  The codewords are cut into chunks of 64 (the last may be
+ * shorter); chunk_bits[c] (u16) is the number of stream bits chunk c uses,
+ * and group_start[g] (u64) is the first bit of chunk 32g, with
+ * group_start[n_groups] = total_bits.  A warp decodes one group of 32
+ * chunks: each lane finds its chunk's first bit by a warp prefix sum over
+ * chunk_bits and decodes exactly its 64 codewords, so no count phase, no
+ * block scan and no realignment of outputs are needed.
+ */
+typedef struct dfw_lanes_info {
+    uint64_t n_chunks;        /* ceil(n / 64) */
+    uint64_t n_groups;        /* ceil(n_chunks / 32); chunk_bits[] holds 32 * n_groups entries */
+    uint32_t chunk_symbols;   /* 64 */
+    uint32_t group_chunks;    /* 32 */
+    uint32_t max_group_bytes; /* largest stream span a group reads, 16-byte aligned with guard (dfw_plan_lanes) */
+    uint32_t lut_words;       /* as dfw_plan_info */
+    uint32_t lut_tables;      /* as dfw_plan_info */
+    uint32_t fast_bits;       /* as dfw_plan_info (dfw_plan_lanes_query sets 12 unless set) */
+} dfw_lanes_info;
+
+/* Sizes of the known-start plan arrays.  A nonzero info->fast_bits on entry
+ * (8..12) is kept.  Errors: DFW_EINVAL. */
+dfw_status dfw_plan_lanes_query(const dfw_table *table, dfw_lanes_info *info);
+
+/*
+ * dfw_plan_lanes -- chunk_bits (host, 32 * n_groups u16; padding zero),
+ * group_start (host, n_groups + 1 u64) and the LUT image (host, lut_words
+ * u32) for one stream; fills info->max_group_bytes.  Host only.
+ * Errors: DFW_EINVAL, DFW_ECORRUPT (stream inconsistent with the table).
+ */
+dfw_status dfw_plan_lanes(const uint8_t *stream, const dfw_table *table, uint16_t *chunk_bits,
+                          uint64_t *group_start, uint32_t *lut, dfw_lanes_info *info);
+
+/*
+ * dfw_decode_lanes -- bit-exact bf16 reconstruction from the known-start
+ * plan, asynchronous on cuda_stream.  Device buffers: d_stream
+ * (table->stream_bytes), d_mant (dfw_mant_bytes(n)), d_lut (lut_words),
+ * d_chunk_bits (32 * n_groups u16), d_group_start (n_groups + 1 u64), d_out
+ * (n bf16).  Errors as dfw_decode; a group whose chunk bits disagree with
+ * group_start, or whose codewords do not end where chunk_bits says, writes
+ * nothing / is flagged through dfw_check.
+ */
+dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                            const uint16_t *d_chunk_bits, const uint64_t *d_group_start,
+                            const dfw_table *table, const dfw_lanes_info *info, uint16_t *d_out,
+                            void *cuda_stream);
+
 /* Static English text for a status code. */
 const char *dfw_strerror(dfw_status status);
 

@@ -21,10 +21,11 @@ from dataclasses import dataclass
 import numpy as np
 import torch
 
-from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, PlanInfo, Table,
+from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, LanesInfo, PlanInfo, Table,
                    check as _check, lib)
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
+           "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "LanesInfo",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
            "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
 
@@ -203,6 +204,74 @@ def decode_block(dc: DeviceCompressed, scratch: torch.Tensor | None = None, stre
                                   _stream_handle(stream)), "dfw_decode_block")
     views = [scratch[int(offs[i]): int(offs[i + 1])] for i in range(k)]
     return scratch, views
+
+
+@dataclass
+class LanesPlan:
+    """Host result of dfw_plan_lanes (known-start chunks)."""
+    chunk_bits: torch.Tensor  # int16 view of uint16[32 * n_groups]
+    group_start: torch.Tensor  # int64 view of uint64[n_groups + 1]
+    lut: torch.Tensor  # int32 view of uint32[lut_words]
+    info: LanesInfo
+
+
+def plan_lanes(enc: Encoded, pin: bool = False, fast_bits: int = 0) -> LanesPlan:
+    info = LanesInfo()
+    info.fast_bits = fast_bits
+    _check(lib().dfw_plan_lanes_query(ctypes.byref(enc.table), ctypes.byref(info)), "dfw_plan_lanes_query")
+    cb = torch.empty(max(32 * int(info.n_groups), 1), dtype=torch.int16, pin_memory=pin)
+    gs = torch.empty(int(info.n_groups) + 1, dtype=torch.int64, pin_memory=pin)
+    lut = torch.empty(int(info.lut_words), dtype=torch.int32, pin_memory=pin)
+    _check(lib().dfw_plan_lanes(_ptr(enc.stream), ctypes.byref(enc.table), _ptr(cb), _ptr(gs), _ptr(lut),
+                                ctypes.byref(info)), "dfw_plan_lanes")
+    return LanesPlan(cb, gs, lut, info)
+
+
+@dataclass
+class DeviceLanes:
+    """A compressed tensor or block resident in device memory, known-start plan."""
+    stream: torch.Tensor
+    mant: torch.Tensor
+    lut: torch.Tensor
+    chunk_bits: torch.Tensor
+    group_start: torch.Tensor
+    table: Table
+    info: LanesInfo
+    tensor_offsets: np.ndarray | None = None
+
+    @staticmethod
+    def upload(enc: Encoded, pl: LanesPlan, device="cuda", non_blocking: bool = False) -> "DeviceLanes":
+        mv = lambda t: t.to(device, non_blocking=non_blocking)  # noqa: E731
+        return DeviceLanes(mv(enc.stream), mv(enc.mant), mv(pl.lut), mv(pl.chunk_bits), mv(pl.group_start),
+                           enc.table, pl.info, enc.tensor_offsets)
+
+    @property
+    def n(self) -> int:
+        return int(self.table.n)
+
+    def compressed_bytes(self, with_aux: bool = True) -> int:
+        b = int(self.table.stream_bytes) + self.n + 256
+        if with_aux:
+            b += 2 * self.chunk_bits.numel() + 8 * self.group_start.numel() + 4 * self.lut.numel()
+        return b
+
+    def algorithmic_bytes(self) -> int:
+        """Stream + chunk_bits + group_start + LUT read, one raw byte read and
+        one bf16 written per weight."""
+        return (int(self.table.stream_bytes) + 2 * self.chunk_bits.numel() + 8 * self.group_start.numel()
+                + 4 * self.lut.numel() + self.n + 2 * self.n)
+
+
+def decode_lanes(dl: DeviceLanes, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Decodes with the known-start plan into ``out`` (bf16, n elements)."""
+    if out is None:
+        out = torch.empty(dl.n, dtype=torch.bfloat16, device=dl.mant.device)
+    if out.numel() < dl.n or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor of at least n elements")
+    _check(lib().dfw_decode_lanes(_ptr(dl.stream), _ptr(dl.mant), _ptr(dl.lut), _ptr(dl.chunk_bits),
+                                  _ptr(dl.group_start), ctypes.byref(dl.table), ctypes.byref(dl.info), _ptr(out),
+                                  _stream_handle(stream)), "dfw_decode_lanes")
+    return out
 
 
 def check(stream=None) -> None:

@@ -33,11 +33,17 @@ class PlanInfo(ctypes.Structure):
                 ("lut_tables", ctypes.c_uint32), ("fast_bits", ctypes.c_uint32), ("reserved", ctypes.c_uint32)]
 
 
+class LanesInfo(ctypes.Structure):
+    _fields_ = [("n_chunks", ctypes.c_uint64), ("n_groups", ctypes.c_uint64), ("chunk_symbols", ctypes.c_uint32),
+                ("group_chunks", ctypes.c_uint32), ("max_group_bytes", ctypes.c_uint32), ("lut_words", ctypes.c_uint32),
+                ("lut_tables", ctypes.c_uint32), ("fast_bits", ctypes.c_uint32)]
+
+
 _lib = None
 
 # name -> (restype, argtypes); the symbols include/dfw.h declares
 _vp, _u64, _i = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int
-_TP, _IP = ctypes.POINTER(Table), ctypes.POINTER(PlanInfo)
+_TP, _IP, _LP = ctypes.POINTER(Table), ctypes.POINTER(PlanInfo), ctypes.POINTER(LanesInfo)
 SIGNATURES = {
     "dfw_stream_bound": (_u64, [_u64]),
     "dfw_mant_bytes": (_u64, [_u64]),
@@ -47,6 +53,9 @@ SIGNATURES = {
     "dfw_plan": (_i, [_vp, _TP, _vp, _vp, _vp, _IP]),
     "dfw_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _IP, _vp, _vp]),
     "dfw_decode_block": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _IP, _vp, _i, _vp, _u64, _vp]),
+    "dfw_plan_lanes_query": (_i, [_TP, _LP]),
+    "dfw_plan_lanes": (_i, [_vp, _TP, _vp, _vp, _vp, _LP]),
+    "dfw_decode_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _vp, _vp]),
     "dfw_check": (_i, [_vp]),
     "dfw_strerror": (ctypes.c_char_p, [_i]),
 }

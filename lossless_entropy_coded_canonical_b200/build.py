@@ -16,7 +16,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdfw.so")
 SOURCES = ["dfw_host.cpp", "dfw_decode.cu"]
-HEADERS = ["dfw_internal.h", os.path.join("..", "..", "include", "dfw.h")]
+HEADERS = ["dfw_internal.h", "dfw_device.cuh", "dfw_lanes.cuh", os.path.join("..", "..", "include", "dfw.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

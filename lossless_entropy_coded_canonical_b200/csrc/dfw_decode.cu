@@ -39,111 +39,14 @@
 #include "dfw_internal.h"
 
 namespace dfw {
+__device__ unsigned int g_status;  // device status word (sticky error bits)
+}
 
-__device__ unsigned int g_status;
+#include "dfw_device.cuh"
+#include "dfw_lanes.cuh"
 
+namespace dfw {
 namespace {
-
-constexpr uint32_t ESC_BAD = 0x40000000u;
-constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s, far above any copy
-
-// --------------------------------------------------------------- PTX helpers
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void fence_mbar_init() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-// Orders this thread's earlier generic accesses to shared memory (made
-// visible to it by a barrier) before its later bulk-copy writes.
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
-}
-
-// 1-D bulk copy global -> this CTA's shared memory; 16-byte aligned addresses
-// and a size that is a multiple of 16.
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
-                 : "memory");
-}
-
-// 1-D bulk copy this CTA's shared memory -> global, tracked in a bulk group.
-__device__ __forceinline__ void bulk_store(void *dst, uint32_t src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(src), "r"(bytes)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-
-// Waits until this thread's bulk stores have read their shared memory.
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-// Waits until this thread's bulk stores have completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0u;
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-// Waits for a phase of an mbarrier with a time and iteration limit; false if
-// it gave up.
-__device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    for (uint32_t it = 0; it < (1u << 24); ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > WAIT_LIMIT_NS) break;
-    }
-    return false;
-}
-
-__device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
-
-// --------------------------------------------------------------- decoding
-
-// A codeword longer than the fast table's key: walk the byte-keyed hierarchy
-// (global memory, read-only path).  x holds the 32 stream bits from the
-// codeword's first bit.  Returns a hierarchy leaf (symbol, total length), or
-// on a corrupt table ESC_BAD with length 1.
-__device__ __noinline__ uint32_t resolve_escape(uint32_t x, const uint32_t *__restrict__ g_hier,
-                                                uint32_t n_tables) {
-    uint32_t e = __ldg(g_hier + (x >> 24));
-#pragma unroll 1
-    for (int level = 1; level < 4 && (e & LUT_PTR); ++level) {
-        const uint32_t child = e & LUT_CHILD_MASK;
-        if (child >= n_tables) break;
-        e = __ldg(g_hier + child * 256u + ((x >> (24 - 8 * level)) & 0xFFu));
-        if (!(e & LUT_PTR)) {
-            const uint32_t l = (e >> LUT_LEN_SHIFT) & 63u;
-            if (l > 8u * level && l <= 8u * level + 8u) return e;
-            break;
-        }
-    }
-    return ESC_BAD | (1u << LUT_LEN_SHIFT);  // length 1 keeps the walk finite
-}
 
 // Phase 1 for one window held as NSEG big-endian words plus a guard word:
 // decodes the codewords starting in [p, wend) and appends their symbols to
@@ -197,18 +100,6 @@ __device__ __forceinline__ uint32_t decode_window(const uint32_t (&wd)[NSEG + 1]
     if (sh) *wp = lo;
     const uint32_t words = (uint32_t)(wp - wp0) / NT;  // full words flushed
     return (32u * words + sh - extra) >> 3;
-}
-
-// Four (exponent, raw byte) pairs -> four bf16 patterns in two words.
-__device__ __forceinline__ void join4(uint32_t E, uint32_t M, uint32_t &w0, uint32_t &w1) {
-    const uint32_t hi = (M & 0x80808080u) | ((E >> 1) & 0x7F7F7F7Fu);  // sign | exp[7:1]
-    const uint32_t lo = ((E << 7) & 0x80808080u) | (M & 0x7F7F7F7Fu);  // exp[0] | mant
-    w0 = __byte_perm(lo, hi, 0x5140);
-    w1 = __byte_perm(lo, hi, 0x7362);
-}
-
-__device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t m) {
-    return (uint16_t)(((m & 0x80u) << 8) | (e << 7) | (m & 0x7Fu));
 }
 
 struct Params {
@@ -436,25 +327,6 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
     if (lane == 0) bulk_wait_all();
 }
 
-// One distinct exponent: every weight is (sym, raw byte).
-__global__ void fill_single(const uint8_t *__restrict__ mant, uint32_t sym, uint64_t n,
-                            uint16_t *__restrict__ out) {
-    const uint32_t E = sym * 0x01010101u;
-    const uint64_t nfull = n >> 3;
-    for (uint64_t c = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; c < nfull;
-         c += (uint64_t)gridDim.x * blockDim.x) {
-        const uint2 m = __ldcs(reinterpret_cast<const uint2 *>(mant + (c << 3)));
-        uint4 r;
-        join4(E, m.x, r.x, r.y);
-        join4(E, m.y, r.z, r.w);
-        __stcs(reinterpret_cast<uint4 *>(out + (c << 3)), r);
-    }
-    if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
-        const uint64_t j = (nfull << 3) + threadIdx.x;
-        out[j] = join1(sym, mant[j]);
-    }
-}
-
 typedef void (*decode_fn)(const Params);
 
 struct Variant {
@@ -582,6 +454,30 @@ extern "C" dfw_status dfw_decode_block(const uint8_t *d_stream, const uint8_t *d
     if (scratch_elems < table->n) return DFW_ENOMEM;
     return launch_decode(d_stream, d_mant, d_lut, d_gap, d_out_start, table, info, d_scratch,
                          static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                                       const uint16_t *d_chunk_bits, const uint64_t *d_group_start,
+                                       const dfw_table *table, const dfw_lanes_info *info, uint16_t *d_out,
+                                       void *cuda_stream) {
+    dfw_status st = validate_table(table);
+    if (st != DFW_OK) return st;
+    if (!info) return DFW_EINVAL;
+    const uint64_t n = table->n;
+    if (n == 0) return DFW_OK;
+    if (!d_mant || !d_out) return DFW_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(d_mant) | reinterpret_cast<uintptr_t>(d_out)) & 15u) return DFW_EALIGN;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFW_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (table->total_bits == 0) {
+        const uint64_t want = ((n >> 3) + 256) / 256, cap = (uint64_t)sms * 8;
+        fill_single<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(d_mant, table->single_symbol, n, d_out);
+        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+    }
+    return launch_decode_lanes(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, d_out, s, sms);
 }
 
 extern "C" dfw_status dfw_check(void *cuda_stream) {

@@ -537,6 +537,117 @@ extern "C" dfw_status dfw_plan(const uint8_t *stream, const dfw_table *table, ui
     return DFW_OK;
 }
 
+// Stream bytes a group reads: from the 16-byte boundary at or below its first
+// bit to 8 guard bytes past its last bit, rounded up to 16.
+uint32_t dfw::group_span_bytes(uint64_t start_bit, uint64_t end_bit) {
+    const uint64_t b0 = (start_bit >> 3) & ~15ull;
+    const uint64_t b1 = (((end_bit + 7) >> 3) + 8 + 15) & ~15ull;
+    return (uint32_t)(b1 - b0);
+}
+
+namespace {
+// Codeword lengths at successive stream positions, from the canonical limits
+// (a 12-bit table for short codes).
+struct LengthWalker {
+    uint64_t limit[34] = {0};
+    std::vector<uint8_t> len12;
+    explicit LengthWalker(const uint8_t len[256]) : len12(4096, 0) {
+        uint64_t cnt[34] = {0};
+        for (int s = 0; s < 256; ++s)
+            if (len[s]) cnt[len[s]]++;
+        uint64_t first = 0;
+        for (int l = 1; l <= 32; ++l) {
+            first = (first + cnt[l - 1]) << 1;
+            limit[l] = first + cnt[l];
+        }
+        for (uint32_t x = 0; x < 4096; ++x)
+            for (int l = 1; l <= 12; ++l)
+                if ((x >> (12 - l)) < limit[l]) {
+                    len12[x] = (uint8_t)l;
+                    break;
+                }
+    }
+    // Length of the codeword at bit pos (the stream has >= 16 guard bytes), 0 if none.
+    int at(const uint8_t *stream, uint64_t pos) const {
+        const uint8_t *p = stream + (pos >> 3);
+        uint64_t v = 0;
+        for (int i = 0; i < 5; ++i) v = (v << 8) | p[i];
+        const uint32_t x = (uint32_t)(v >> (8 - (pos & 7)));
+        int l = len12[x >> 20];
+        if (!l) {
+            for (l = 13; l <= 32; ++l)
+                if ((uint64_t)(x >> (32 - l)) < limit[l]) break;
+            if (l > 32) return 0;
+        }
+        return l;
+    }
+};
+}  // namespace
+
+extern "C" dfw_status dfw_plan_lanes_query(const dfw_table *table, dfw_lanes_info *info) {
+    if (!info) return DFW_EINVAL;
+    dfw_status st = validate_table(table);
+    if (st != DFW_OK) return st;
+    const uint32_t fb = info->fast_bits ? info->fast_bits : (uint32_t)FAST_BITS_DEFAULT_LANES;
+    if (fb < (uint32_t)FAST_BITS_MIN || fb > (uint32_t)FAST_BITS_MAX) return DFW_EINVAL;
+    std::memset(info, 0, sizeof(*info));
+    info->fast_bits = fb;
+    info->chunk_symbols = LANE_SYMS;
+    info->group_chunks = GROUP_CHUNKS;
+    info->n_chunks = (table->n + LANE_SYMS - 1) / LANE_SYMS;
+    info->n_groups = (info->n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+    std::vector<uint32_t> lut;
+    st = build_lut(table, lut);
+    if (st != DFW_OK) return st;
+    info->lut_tables = (uint32_t)(lut.size() / 256);
+    info->lut_words = (2u << fb) + (uint32_t)lut.size();
+    return DFW_OK;
+}
+
+extern "C" dfw_status dfw_plan_lanes(const uint8_t *stream, const dfw_table *table, uint16_t *chunk_bits,
+                                     uint64_t *group_start, uint32_t *lut, dfw_lanes_info *info) {
+    if (!info || !group_start || !lut) return DFW_EINVAL;
+    dfw_lanes_info q;
+    q.fast_bits = info->fast_bits;
+    dfw_status st = dfw_plan_lanes_query(table, &q);
+    if (st != DFW_OK) return st;
+    if (q.n_groups != info->n_groups || q.lut_words != info->lut_words) return DFW_EINVAL;
+    if (q.n_groups && !chunk_bits) return DFW_EINVAL;
+    std::vector<uint32_t> img, fast;
+    build_lut(table, img);
+    st = build_fast(img, (int)q.fast_bits, fast);
+    if (st != DFW_OK) return st;
+    std::memcpy(lut, fast.data(), fast.size() * sizeof(uint32_t));
+    std::memcpy(lut + fast.size(), img.data(), img.size() * sizeof(uint32_t));
+    const uint64_t n = table->n, tb = table->total_bits;
+    std::memset(chunk_bits, 0, (size_t)(q.n_groups * GROUP_CHUNKS) * sizeof(uint16_t));
+    if (tb == 0) {  // one symbol: no bits anywhere
+        for (uint64_t g = 0; g <= q.n_groups; ++g) group_start[g] = 0;
+        info->max_group_bytes = 16;
+        return DFW_OK;
+    }
+    if (!stream) return DFW_EINVAL;
+    LengthWalker walk(table->len);
+    uint64_t pos = 0, cstart = 0;
+    for (uint64_t i = 0; i < n; ++i) {
+        if (i % LANE_SYMS == 0) {
+            cstart = pos;
+            if (i % ((uint64_t)LANE_SYMS * GROUP_CHUNKS) == 0) group_start[i / ((uint64_t)LANE_SYMS * GROUP_CHUNKS)] = pos;
+        }
+        if (pos >= tb) return DFW_ECORRUPT;
+        const int l = walk.at(stream, pos);
+        if (!l) return DFW_ECORRUPT;
+        pos += (uint64_t)l;
+        if ((i + 1) % LANE_SYMS == 0 || i + 1 == n) chunk_bits[i / LANE_SYMS] = (uint16_t)(pos - cstart);
+    }
+    if (pos != tb) return DFW_ECORRUPT;
+    group_start[q.n_groups] = tb;
+    uint32_t mx = 16;
+    for (uint64_t g = 0; g < q.n_groups; ++g) mx = std::max(mx, group_span_bytes(group_start[g], group_start[g + 1]));
+    info->max_group_bytes = mx;
+    return DFW_OK;
+}
+
 extern "C" const char *dfw_strerror(dfw_status s) {
     switch (s) {
         case DFW_OK: return "ok";

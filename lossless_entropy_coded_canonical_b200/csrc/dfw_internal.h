@@ -24,7 +24,8 @@ constexpr int LUT_CBITS_SHIFT = 18;
 // count, bits 16..27 = end mask (bit j-1 set when one of them ends at key
 // offset j), bit 31 = escape (first codeword longer than K bits; its bits
 // byte is 255 so any bounds test sends it to the slow path).
-constexpr int FAST_BITS_DEFAULT = 10;
+constexpr int FAST_BITS_DEFAULT = 10;        // windowed plan
+constexpr int FAST_BITS_DEFAULT_LANES = 12;  // known-start plan
 constexpr int FAST_BITS_MIN = 8;
 constexpr int FAST_BITS_MAX = 12;
 constexpr int FAST_MAX_SYMS = 4;
@@ -32,6 +33,10 @@ constexpr int FAST_C8_SHIFT = 8;
 constexpr int FAST_ENDS_SHIFT = 16;
 constexpr uint32_t FAST_ESC = 0x80000000u;
 constexpr uint32_t FAST_ESC_WORD = FAST_ESC | 255u;
+
+// Known-start chunks: codewords per chunk, chunks per group (one warp).
+constexpr uint32_t LANE_SYMS = 64;
+constexpr uint32_t GROUP_CHUNKS = 32;
 
 // Bits of the device status word.
 constexpr uint32_t ST_COUNT = 1u;   // a tile decoded a different number of codes than out_start says
@@ -47,5 +52,6 @@ dfw_status build_lut(const dfw_table *table, std::vector<uint32_t> &lut);
 dfw_status build_fast(const std::vector<uint32_t> &lut, int fast_bits, std::vector<uint32_t> &fast);
 bool plan_shape_supported(uint32_t W, uint32_t T);
 dfw_status validate_table(const dfw_table *t);
+uint32_t group_span_bytes(uint64_t start_bit, uint64_t end_bit);
 
 }  // namespace dfw

@@ -1,0 +1,433 @@
+// dfw_lanes.cuh -- the known-start decode kernel (included by dfw_decode.cu).
+//
+// Same stream and tables as the windowed kernel; the plan differs: codewords
+// are cut into chunks of 64, chunk_bits[c] says how many stream bits chunk c
+// uses and group_start[g] where group g (32 chunks) begins (the LazyWeights
+// write-up's interleaved lanes with known starts, body and Verified Facts).
+// One warp decodes one group at a time, persistently.  All bulk copies are
+// issued by lane 0, one per buffer (copy instructions take warp-uniform
+// operands, so per-lane copies would be serialised lane by lane):
+//   - the group's chunk_bits and stream span arrive in one of the warp's two
+//     stream slots (started one group ahead), its 2048 raw bytes in the
+//     warp's raw-byte buffer (started as soon as the previous group's join
+//     has read that buffer);
+//   - each lane finds its chunk's first bit with a warp prefix sum of
+//     chunk_bits and decodes exactly its 64 codewords with the fast table
+//     (up to four codewords per lookup) into its own word slots, interleaved
+//     by lane so stores never conflict;
+//   - each lane joins exponents and raw bytes into bf16, 16 at a time in a
+//     lane-rotated order (which spreads the 128-bit shared accesses over the
+//     banks), into the warp's staging buffer in output order; lane 0 then
+//     writes the group's 4 KB with one TMA bulk store.
+// No count phase, no block scan, no CTA barrier after the table load, and no
+// realignment: every chunk's output is 64-weight aligned.
+//
+// Bounds: a lane makes at most 64 lookups per chunk (each yields >= 1
+// codeword); stream reads are clamped to the slot; a group whose chunk_bits
+// do not add up to its group_start span, or whose lanes do not end exactly
+// where chunk_bits says, writes nothing and sets a status bit; waits on bulk
+// copies are bounded.
+#pragma once
+
+#include "dfw_device.cuh"
+
+namespace dfw {
+namespace {
+
+constexpr uint32_t EXP_WORDS = 17;        // a chunk's 64 exponent bytes + up to 3 more from the last lookup
+constexpr uint32_t GROUP_SYMS = LANE_SYMS * GROUP_CHUNKS;  // 2048 weights per warp group
+
+struct LanesParams {
+    const uint8_t *stream;
+    const uint8_t *mant;
+    const uint32_t *lut;
+    const uint16_t *chunk_bits;
+    const uint64_t *group_start;
+    uint16_t *out;
+    uint64_t n, n_chunks, n_groups, stream_bytes, mant_bytes;
+    uint32_t fast_bits, n_tables, sbuf_bytes;
+};
+
+__device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_bit) {
+    const uint64_t b0 = (start_bit >> 3) & ~15ull;
+    const uint64_t b1 = (((end_bit + 7) >> 3) + 8 + 15) & ~15ull;
+    return (uint32_t)(b1 - b0);
+}
+
+// Decodes `left8 / 8` codewords starting at bit r of the stream words held in
+// shared memory at sw (32-bit shared address), n_words of them, and appends
+// their symbols to this lane's word slots ep, ep + 128, ... (slots of the 32
+// lanes interleave; a last lookup may append up to three more symbols, which
+// are never read).  fast is the shared address of the
+// fast table.  Returns the stream bit position (relative to sw) after the
+// last codeword decoded.
+//
+// The inner loop is straight-line code: it always loads the word after the
+// current pair and selects it in when the position crosses a word, and it
+// always stores the accumulator's low word and advances by select.  Only an
+// escape or the chunk's last lookup leaves it, for one step of the general
+// path.
+__device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t n_words, uint32_t r, int left8,
+                                                 uint32_t fast, uint32_t kshift,
+                                                 const uint32_t *__restrict__ g_hier, uint32_t n_tables,
+                                                 uint32_t ep, uint32_t &err) {
+    const uint32_t w_end = sw + 4u * (n_words - 1u);  // last readable word
+    uint32_t wa = min(sw + 4u * (r >> 5), w_end);
+    uint32_t a = bswap32(lds32(wa));
+    wa = min(wa + 4u, w_end);
+    uint32_t b = bswap32(lds32(wa));
+    wa = min(wa + 4u, w_end);  // the next word to shift in
+    uint32_t p = r & 31u, words = 0;  // bit position = 32 * ((r >> 5) + words) + p
+    uint32_t lo = 0u, hi = 0u, sh = 0u;
+    while (left8 > 0) {
+        uint32_t x, syms, c8, cb, ey;
+        // straight-line loop in PTX; it exits on an escape (bits byte 255)
+        // or on the lookup that completes the chunk (8 * count >= left8)
+        asm volatile(
+            "{\n\t"
+            ".reg .pred pe, pl, pa, pf;\n\t"
+            ".reg .b32 t0, t1, ex, nx, ad;\n"
+            "LANES_LOOP:\n\t"
+            "shf.l.wrap.b32 %0, %10, %9, %11;\n\t"  // x = stream bits [p, p + 32)
+            "shr.b32 t0, %0, %19;\n\t"
+            "mad.lo.u32 ad, t0, 8, %18;\n\t"
+            "ld.shared.v2.u32 {ex, %4}, [ad];\n\t"
+            "ld.shared.u32 nx, [%12];\n\t"  // the word after b
+            "and.b32 %3, %4, 255;\n\t"
+            "prmt.b32 %2, %4, 0, 0x4441;\n\t"
+            "setp.eq.u32 pe, %3, 255;\n\t"
+            "setp.ge.s32 pl, %2, %17;\n\t"
+            "or.pred pe, pe, pl;\n\t"
+            "@pe bra LANES_EXIT;\n\t"
+            "add.u32 %11, %11, %3;\n\t"  // p += bits used
+            "setp.ge.u32 pa, %11, 32;\n\t"
+            "prmt.b32 nx, nx, 0, 0x0123;\n\t"
+            "selp.b32 %9, %10, %9, pa;\n\t"  // a = b
+            "selp.b32 %10, nx, %10, pa;\n\t"  // b = next word
+            "@pa add.u32 %12, %12, 4;\n\t"
+            "min.u32 %12, %12, %20;\n\t"
+            "@pa add.u32 %13, %13, 1;\n\t"
+            "and.b32 %11, %11, 31;\n\t"
+            "shl.b32 t0, ex, %16;\n\t"  // append symbols at byte offset sh / 8
+            "or.b32 %14, %14, t0;\n\t"
+            "shf.l.wrap.b32 t1, ex, 0, %16;\n\t"
+            "or.b32 %15, %15, t1;\n\t"
+            "add.u32 %16, %16, %2;\n\t"
+            "st.shared.u32 [%8], %14;\n\t"
+            "setp.ge.u32 pf, %16, 32;\n\t"
+            "@pf add.u32 %8, %8, 128;\n\t"  // next word slot of this lane
+            "selp.b32 %14, %15, %14, pf;\n\t"
+            "selp.b32 %15, 0, %15, pf;\n\t"
+            "and.b32 %16, %16, 31;\n\t"
+            "sub.s32 %17, %17, %2;\n\t"
+            "bra LANES_LOOP;\n"
+            "LANES_EXIT:\n\t"
+            "mov.b32 %1, ex;\n\t"
+            "}"
+            : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(err), "+r"(n_words), "+r"(r),
+              "+r"(ep), "+r"(a), "+r"(b), "+r"(p), "+r"(wa), "+r"(words), "+r"(lo), "+r"(hi), "+r"(sh),
+              "+r"(left8)
+            : "r"(fast), "r"(kshift), "r"(w_end)
+            : "memory");
+        if (cb != 255u) {
+            // the chunk's last lookup: later codewords belong to the next
+            // chunk, so advance only to the end of codeword left8/8 - 1
+            uint32_t ends = (ey >> FAST_ENDS_SHIFT) & 0xFFFu;
+            for (int i = 8; i < left8; i += 8) ends &= ends - 1u;
+            cb = (uint32_t)__ffs(ends);
+            c8 = (uint32_t)left8;
+        }
+        // one general step: an escape (codeword longer than the fast key) or
+        // the chunk's last lookup
+        if (cb == 255u) {
+            const uint32_t f = resolve_escape(x, g_hier, n_tables);
+            if (f & ESC_BAD) err |= ST_LUT;
+            syms = f & 0xFFu;
+            c8 = 8u;
+            cb = (f >> LUT_LEN_SHIFT) & 63u;  // <= 32: at most one word to shift in
+        }
+        p += cb;
+        if (p >= 32u) {
+            a = b;
+            b = bswap32(lds32(wa));
+            wa = min(wa + 4u, w_end);
+            ++words;
+            p -= 32u;
+        }
+        lo |= syms << sh;
+        hi |= __funnelshift_l(syms, 0u, sh);
+        sh += c8;
+        if (sh >= 32u) {
+            sts32(ep, lo);
+            ep += 128u;
+            lo = hi;
+            hi = 0u;
+            sh -= 32u;
+        }
+        left8 -= (int)c8;
+    }
+    if (sh) sts32(ep, lo);
+    return 32u * ((r >> 5) + words) + p;
+}
+
+// Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes) | 2 x
+// (chunk_bits | stream span) | raw bytes (2048) | bf16 staging (4096) |
+// exponent word slots (EXP_WORDS x 32).
+__host__ __device__ constexpr uint32_t warp_smem_bytes(uint32_t sbuf_bytes) {
+    return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + 2u * GROUP_SYMS + 4u * EXP_WORDS * 32u;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
+    constexpr int NWARP = NT / 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    const uint32_t n_fast = 1u << prm.fast_bits;
+    uint2 *s_fast = reinterpret_cast<uint2 *>(smem);
+    const uint32_t wbytes = warp_smem_bytes(prm.sbuf_bytes);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t *wbase = smem + (8u << prm.fast_bits) + warp * wbytes;
+    const uint32_t bar_s0 = smem_u32(wbase), bar_m = bar_s0 + 16u;
+    uint8_t *wslots = wbase + 32;
+    const uint32_t slot_bytes = 64u + prm.sbuf_bytes;
+    uint8_t *mbuf = wslots + 2u * slot_bytes;
+    uint8_t *stage = mbuf + GROUP_SYMS;
+    const uint32_t exps = smem_u32(stage + 2u * GROUP_SYMS) + 4u * lane;  // word k at exps + 128 k
+    const uint32_t *g_hier = prm.lut + 2u * n_fast;
+    const uint32_t kshift = 32u - prm.fast_bits;
+
+    if (lane == 0) {
+        mbar_init(bar_s0, 1);
+        mbar_init(bar_s0 + 8u, 1);
+        mbar_init(bar_m, 1);
+        fence_mbar_init();
+    }
+    bool bad = false;
+    for (uint32_t i = tid; i < n_fast; i += NT) {
+        const uint2 e = __ldg(reinterpret_cast<const uint2 *>(prm.lut) + i);
+        if (e.y & FAST_ESC) {
+            bad |= e.y != FAST_ESC_WORD || e.x != 0u;
+        } else {
+            const uint32_t cb = e.y & 255u, c8 = (e.y >> FAST_C8_SHIFT) & 255u,
+                           ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
+            bad |= c8 == 0u || (c8 & 7u) || c8 > 8u * FAST_MAX_SYMS || cb == 0u || cb > prm.fast_bits ||
+                   8u * cb < c8 || (uint32_t)__popc(ends) * 8u != c8 || (ends >> (cb - 1u)) != 1u ||
+                   (e.y & 0x70000000u) || (c8 < 32u && (e.x >> c8) != 0u);
+        }
+        s_fast[i] = e;
+    }
+    if (__syncthreads_or(bad)) {
+        if (tid == 0) atomicOr(&g_status, ST_LUT);
+        return;
+    }
+
+    const uint64_t gstride = (uint64_t)gridDim.x * NWARP;
+    uint64_t g = (uint64_t)blockIdx.x * NWARP + warp;
+    if (g >= prm.n_groups) return;  // no CTA barrier follows
+
+    // lane 0: chunk_bits and stream span of group gg into slot s
+    auto issue_stream = [&](uint64_t gg, uint32_t s, uint64_t s0, uint64_t s1) {
+        uint8_t *slot = wslots + s * slot_bytes;
+        const uint32_t bar = bar_s0 + 8u * s;
+        const uint64_t sb0 = (s0 >> 3) & ~15ull;
+        uint32_t sbytes = 0;
+        if (s1 >= s0 && sb0 < prm.stream_bytes) {
+            sbytes = min(span_bytes(s0, s1), prm.sbuf_bytes);
+            sbytes = (uint32_t)min((uint64_t)sbytes, prm.stream_bytes - sb0);
+        }
+        fence_proxy_async();
+        mbar_expect_tx(bar, 64u + sbytes);
+        bulk_load(smem_u32(slot), prm.chunk_bits + gg * GROUP_CHUNKS, 64u, bar);
+        if (sbytes) bulk_load(smem_u32(slot + 64), prm.stream + sb0, sbytes, bar);
+    };
+    // lane 0: the group's raw bytes into the warp buffer
+    auto issue_mant = [&](uint64_t gg) {
+        const uint64_t m0 = gg * (uint64_t)GROUP_SYMS;
+        const uint32_t bytes = (uint32_t)min((uint64_t)GROUP_SYMS, prm.mant_bytes - m0);
+        fence_proxy_async();
+        mbar_expect_tx(bar_m, bytes);
+        bulk_load(smem_u32(mbuf), prm.mant + m0, bytes, bar_m);
+    };
+
+    uint64_t gs0 = __ldg(prm.group_start + g), gs1 = __ldg(prm.group_start + g + 1);
+    uint64_t g1 = g + gstride, ns0 = 0, ns1 = 0;
+    if (g1 < prm.n_groups) {
+        ns0 = __ldg(prm.group_start + g1);
+        ns1 = __ldg(prm.group_start + g1 + 1);
+    }
+    if (lane == 0) {
+        issue_stream(g, 0, gs0, gs1);
+        issue_mant(g);
+    }
+
+    for (uint32_t k = 0;; ++k) {
+        const uint32_t s = k & 1u;
+        const uint8_t *slot = wslots + s * slot_bytes;
+        const bool has_next = g1 < prm.n_groups;
+        const uint64_t g2 = g1 + gstride;
+        uint64_t ms0 = 0, ms1 = 0;
+        if (g2 < prm.n_groups) {  // starts two groups ahead, for the copy issued next round
+            ms0 = __ldg(prm.group_start + g2);
+            ms1 = __ldg(prm.group_start + g2 + 1);
+        }
+        __syncwarp();  // every lane is done with the other slot
+        if (has_next && lane == 0) issue_stream(g1, s ^ 1u, ns0, ns1);
+
+        bool ok = mbar_wait_bounded(bar_s0 + 8u * s, (k >> 1) & 1u);
+        const uint32_t cbits = reinterpret_cast<const uint16_t *>(slot)[lane];
+        uint32_t incl = cbits;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        const uint32_t excl = incl - cbits, gbits = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const uint64_t c = g * GROUP_CHUNKS + lane;
+        const uint32_t t = c < prm.n_chunks ? (uint32_t)min((uint64_t)LANE_SYMS, prm.n - LANE_SYMS * c) : 0u;
+        const uint64_t sb0 = (gs0 >> 3) & ~15ull;
+        const bool valid = __all_sync(0xFFFFFFFFu, gs1 >= gs0 && gs1 - gs0 == gbits && cbits <= 32u * LANE_SYMS &&
+                                                       span_bytes(gs0, gs1) <= prm.sbuf_bytes &&
+                                                       sb0 + span_bytes(gs0, gs1) <= prm.stream_bytes &&
+                                                       (t != 0u || cbits == 0u));
+        uint32_t err = 0;
+        if (ok && valid && t) {
+            const uint32_t r = (uint32_t)(gs0 - 8ull * sb0) + excl;
+            const uint32_t end = decode_chunk(smem_u32(slot + 64), prm.sbuf_bytes / 4u, r, (int)(8u * t),
+                                              smem_u32(s_fast), kshift, g_hier, prm.n_tables, exps, err);
+            if (end != r + cbits) err |= ST_COUNT;
+        }
+        ok = mbar_wait_bounded(bar_m, k & 1u) && ok;
+        if (lane == 0) bulk_wait_read();  // the previous group's store has read the staging buffer
+        if (!__all_sync(0xFFFFFFFFu, ok)) {  // a bulk copy never completed: give up
+            if (lane == 0) {
+                atomicOr(&g_status, ST_TIMEOUT);
+                if (has_next) mbar_wait_bounded(bar_s0 + 8u * (s ^ 1u), ((k + 1) >> 1) & 1u);
+                bulk_wait_all();
+            }
+            return;
+        }
+        const bool good = valid && !__any_sync(0xFFFFFFFFu, err != 0u);
+        if (!valid) {
+            if (lane == 0) atomicOr(&g_status, ST_RANGE);
+        } else if (!good) {
+            if (err) atomicOr(&g_status, err);
+        } else {
+            // join: piece q (16 weights) of this lane's chunk, in the order
+            // (j + lane / 2) mod 4 so lanes spread over the banks
+            const uint32_t mrow = smem_u32(mbuf) + 64u * lane, orow = smem_u32(stage) + 128u * lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
+                const uint4 m = lds128(mrow + 16u * q);
+                const uint32_t e0 = lds32(exps + 512u * q), e1 = lds32(exps + 512u * q + 128u),
+                               e2 = lds32(exps + 512u * q + 256u), e3 = lds32(exps + 512u * q + 384u);
+                uint4 r0, r1;
+                join4(e0, m.x, r0.x, r0.y);
+                join4(e1, m.y, r0.z, r0.w);
+                join4(e2, m.z, r1.x, r1.y);
+                join4(e3, m.w, r1.z, r1.w);
+                sts128(orow + 32u * q, r0);
+                sts128(orow + 32u * q + 16u, r1);
+            }
+            fence_proxy_async();
+            __syncwarp();
+            const uint64_t w0 = g * (uint64_t)GROUP_SYMS;
+            const uint32_t gw = (uint32_t)min((uint64_t)GROUP_SYMS, prm.n - w0);  // weights in this group
+            const uint32_t body = gw & ~7u;
+            if (lane == 0 && body) bulk_store(prm.out + w0, smem_u32(stage), 2u * body);
+            if (lane < (int)(gw - body)) {
+                const uint32_t i = body + lane;
+                prm.out[w0 + i] = reinterpret_cast<const uint16_t *>(stage)[i];
+            }
+        }
+        if (!has_next) break;
+        __syncwarp();  // all lanes have read the raw bytes
+        if (lane == 0) issue_mant(g1);
+        g = g1;
+        g1 = g2;
+        gs0 = ns0;
+        gs1 = ns1;
+        ns0 = ms0;
+        ns1 = ms1;
+    }
+    if (lane == 0) bulk_wait_all();
+}
+
+template <int NT>
+uint32_t lanes_smem(uint32_t fast_bits, uint32_t sbuf_bytes) {
+    return (8u << fast_bits) + (NT / 32) * warp_smem_bytes(sbuf_bytes);
+}
+
+typedef void (*lanes_fn)(const LanesParams);
+struct LanesVariant {
+    int nt;
+    lanes_fn fn;
+    uint32_t (*smem)(uint32_t, uint32_t);
+    int smem_set[16];  // dynamic shared memory opted in, per device
+};
+// Largest CTA first: a larger CTA shares one copy of the fast table among
+// more warps; data with long codes needs bigger stream slots and falls back
+// to a smaller CTA.
+LanesVariant g_lanes[] = {
+    {512, decode_lanes<512>, lanes_smem<512>, {0}},
+    {256, decode_lanes<256>, lanes_smem<256>, {0}},
+    {128, decode_lanes<128>, lanes_smem<128>, {0}},
+};
+
+}  // namespace
+
+dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                               const uint16_t *d_chunk_bits, const uint64_t *d_group_start, const dfw_table *table,
+                               const dfw_lanes_info *info, uint16_t *d_out, cudaStream_t s, int sms) {
+    const uint64_t n = table->n;
+    if (info->chunk_symbols != LANE_SYMS || info->group_chunks != GROUP_CHUNKS ||
+        info->n_chunks != (n + LANE_SYMS - 1) / LANE_SYMS ||
+        info->n_groups != (info->n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS)
+        return DFW_EINVAL;
+    const uint32_t fb = info->fast_bits;
+    if (fb < (uint32_t)FAST_BITS_MIN || fb > (uint32_t)FAST_BITS_MAX || info->lut_tables < 1 ||
+        info->lut_words != (2u << fb) + 256u * info->lut_tables)
+        return DFW_EINVAL;
+    if (!d_stream || !d_lut || !d_chunk_bits || !d_group_start) return DFW_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(d_stream) | reinterpret_cast<uintptr_t>(d_lut) |
+         reinterpret_cast<uintptr_t>(d_chunk_bits) | reinterpret_cast<uintptr_t>(d_group_start)) & 15u)
+        return DFW_EALIGN;
+    if (info->max_group_bytes < 16 || (info->max_group_bytes & 15u) || info->max_group_bytes > 64u * 1024u)
+        return DFW_EINVAL;
+    LanesParams prm;
+    prm.stream = d_stream;
+    prm.mant = d_mant;
+    prm.lut = d_lut;
+    prm.chunk_bits = d_chunk_bits;
+    prm.group_start = d_group_start;
+    prm.out = d_out;
+    prm.n = n;
+    prm.n_chunks = info->n_chunks;
+    prm.n_groups = info->n_groups;
+    prm.stream_bytes = table->stream_bytes;
+    prm.mant_bytes = (n + 15) & ~15ull;
+    prm.fast_bits = fb;
+    prm.n_tables = info->lut_tables;
+    prm.sbuf_bytes = info->max_group_bytes;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
+    for (LanesVariant &v : g_lanes) {
+        const uint32_t smem = v.smem(fb, prm.sbuf_bytes);
+        if (smem > 227u * 1024u) continue;
+        if (!v.smem_set[dev]) {
+            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+                return DFW_ECUDA;
+            v.smem_set[dev] = 1;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess) return DFW_ECUDA;
+        if (per_sm < 1) continue;
+        const uint64_t wpc = (uint64_t)v.nt / 32;
+        const uint64_t warps = (uint64_t)per_sm * sms * wpc;
+        const uint64_t want = info->n_groups < warps ? info->n_groups : warps;
+        v.fn<<<(unsigned)((want + wpc - 1) / wpc), v.nt, smem, s>>>(prm);
+        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+    }
+    return DFW_EINVAL;  // even the smallest CTA does not fit
+}
+
+}  // namespace dfw

@@ -72,6 +72,8 @@ def _load():
         lib.oracle_n_windows.restype = u64
         lib.oracle_aux.argtypes = [u8p, u64, u8p, u64, u64, u64, u8p, u64p]
         lib.oracle_aux.restype = ctypes.c_int
+        lib.oracle_chunk_aux.argtypes = [u8p, u64, u8p, u64, u64, u64, u32p, u64p]
+        lib.oracle_chunk_aux.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -217,3 +219,17 @@ def aux(enc: Encoded, W: int, T: int) -> tuple[np.ndarray, np.ndarray]:
     _check(_load().oracle_aux(_p(stream, ctypes.c_uint8), enc.total_bits, _p(ln, ctypes.c_uint8), enc.n, W, T,
                               _p(gap, ctypes.c_uint8), _p(out_start, ctypes.c_uint64)), "aux")
     return gap[:nwin], out_start
+
+
+def chunk_aux(enc: Encoded, M: int = 64, G: int = 32) -> tuple[np.ndarray, np.ndarray]:
+    """(chunk_bits[n_groups * G] u32, group_start[n_groups + 1] u64) for
+    chunks of M codewords and groups of G chunks (reading R7)."""
+    n_chunks = (enc.n + M - 1) // M
+    n_groups = (n_chunks + G - 1) // G
+    bits = np.zeros(max(n_groups * G, 1), np.uint32)
+    starts = np.zeros(n_groups + 1, np.uint64)
+    stream = np.ascontiguousarray(enc.stream if enc.stream.size else np.zeros(1, np.uint8), dtype=np.uint8)
+    ln = np.ascontiguousarray(enc.lengths, dtype=np.uint8)
+    _check(_load().oracle_chunk_aux(_p(stream, ctypes.c_uint8), enc.total_bits, _p(ln, ctypes.c_uint8), enc.n, M, G,
+                                    _p(bits, ctypes.c_uint32), _p(starts, ctypes.c_uint64)), "chunk_aux")
+    return bits[: n_groups * G], starts

@@ -31,6 +31,9 @@
  *      it (or to total_bits when no code starts there); for a tile of T
  *      windows, out_start[b] counts the code starts before bit 8*W*T*b, and
  *      out_start[n_tiles] = n.
+ *   R7 known-start chunks (the per-chunk bit offsets of a second decode
+ *      plan): chunk_bits[c] = bits of codewords Mc .. M(c+1)-1, and
+ *      group_start[g] = first bit of codeword MGg.
  * Parity: every function here is pinned by tests in tests/test_oracle_*.py
  * (round trip, Kraft equality, entropy bounds, brute-force optimality,
  * closed forms, independent recounts).  The tie rule of R2 is this
@@ -365,5 +368,39 @@ int oracle_aux(const uint8_t *stream, uint64_t total_bits, const uint8_t len[256
     for (; b < ntiles; b++)
         out_start[b] = n;
     out_start[ntiles] = n;
+    return OR_OK;
+}
+
+/* ---- R7 (known-start chunks): codeword i starts at bit start(i), with
+ * start(n) = total_bits.  For chunks of M codewords, chunk_bits[c] =
+ * start(min(M(c+1), n)) - start(Mc); for groups of G chunks,
+ * group_start[g] = start(MGg) and group_start[n_groups] = total_bits.
+ * chunk_bits has n_groups * G entries; the ones past the last chunk are 0. */
+int oracle_chunk_aux(const uint8_t *stream, uint64_t total_bits, const uint8_t len[256], uint64_t n,
+                     uint64_t M, uint64_t G, uint32_t *chunk_bits, uint64_t *group_start)
+{
+    if (M == 0 || G == 0)
+        return OR_EINVAL;
+    uint64_t n_chunks = (n + M - 1) / M;
+    uint64_t n_groups = (n_chunks + G - 1) / G;
+    for (uint64_t c = 0; c < n_groups * G; c++)
+        chunk_bits[c] = 0;
+    canon_dec d;
+    canon_init(len, &d);
+    uint64_t pos = 0, chunk_start = 0;
+    for (uint64_t i = 0; i < n; i++) {
+        if (i % M == 0) {
+            chunk_start = pos;
+            if (i % (M * G) == 0)
+                group_start[i / (M * G)] = pos;
+        }
+        if (total_bits > 0 && canon_read(&d, stream, total_bits, &pos) < 0)
+            return OR_ECORRUPT;
+        if ((i + 1) % M == 0 || i + 1 == n)
+            chunk_bits[i / M] = (uint32_t)(pos - chunk_start);
+    }
+    if (pos != total_bits)
+        return OR_ECORRUPT;
+    group_start[n_groups] = total_bits;
     return OR_OK;
 }

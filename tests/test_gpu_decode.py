@@ -17,7 +17,7 @@ import workloads
 pytestmark = pytest.mark.gpu
 
 BENCH_SHAPE = (8, 256)
-SHAPES = [(8, 128), (8, 256), (8, 512), (16, 128), (16, 256)]
+SHAPES = [(8, 128), (8, 256), (8, 512), (16, 128), (16, 256), (0, 0)]  # (0, 0): known-start plan
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -53,10 +53,20 @@ def gpu_decode(enc: dfw.Encoded, W: int, T: int) -> np.ndarray:
     return workloads.as_u16_numpy(out)
 
 
+def gpu_decode_lanes(enc: dfw.Encoded) -> np.ndarray:
+    pl = dfw.plan_lanes(enc)
+    dl = dfw.DeviceLanes.upload(enc, pl)
+    out = dfw.decode_lanes(dl)
+    dfw.check()
+    return workloads.as_u16_numpy(out)
+
+
 def oracle_parity(oracle, u: np.ndarray, W: int, T: int, cap: int = 32):
+    """Windowed plan with shape (W, T), and (W == 0) the known-start plan."""
     oenc = oracle.encode(u, cap)
     expect = oracle.decode(oenc)
-    got = gpu_decode(encoded_from_oracle(oenc), W, T)
+    enc = encoded_from_oracle(oenc)
+    got = gpu_decode_lanes(enc) if W == 0 else gpu_decode(enc, W, T)
     assert got.shape == expect.shape
     bad = np.nonzero(got != expect)[0]
     assert bad.size == 0, f"{bad.size} mismatches, first at {bad[:5]}"
@@ -88,10 +98,12 @@ def test_parity_edge_sizes(oracle, n):
     rng = np.random.default_rng(n)
     u = rng.integers(0, 65536, size=n, dtype=np.uint64).astype(np.uint16)
     oracle_parity(oracle, u, *BENCH_SHAPE)
+    oracle_parity(oracle, u, 0, 0)
     # five exponents only: short codes, many codewords per window
     u2 = ((rng.integers(0, 2, n) << 15) | ((120 + rng.integers(0, 5, n)) << 7)
           | rng.integers(0, 128, n)).astype(np.uint16)
     oracle_parity(oracle, u2, 8, 128)
+    oracle_parity(oracle, u2, 0, 0)
 
 
 @pytest.mark.parametrize("n", [1, 7, 8, 9, 1000, 100_003])
@@ -99,6 +111,7 @@ def test_single_symbol(oracle, n):
     rng = np.random.default_rng(n)
     u = ((rng.integers(0, 2, n) << 15) | (119 << 7) | rng.integers(0, 128, n)).astype(np.uint16)
     oracle_parity(oracle, u, *BENCH_SHAPE)
+    oracle_parity(oracle, u, 0, 0)
 
 
 def test_empty():
@@ -117,6 +130,7 @@ def test_cap_binding_tables(oracle, cap):
     u = _u16(workloads.c4("b", 1_500_001))
     oracle_parity(oracle, u, 8, 256, cap)
     oracle_parity(oracle, u, 16, 256, cap)
+    oracle_parity(oracle, u, 0, 0, cap)
 
 
 def test_codes_straddle_tiles(oracle):
@@ -128,6 +142,7 @@ def test_codes_straddle_tiles(oracle):
     u = ((e.astype(np.uint16) << 7) | rng.integers(0, 128, e.size).astype(np.uint16)).astype(np.uint16)
     oracle_parity(oracle, u, 8, 128, 32)
     oracle_parity(oracle, u[:-3], 16, 128, 12)
+    oracle_parity(oracle, u[:-5], 0, 0, 32)
 
 
 def test_product_encoder_roundtrip_on_gpu(oracle):
@@ -193,6 +208,15 @@ def _full_parity(oracle, tensors, block=False, samples=6):
     return enc
 
 
+def _full_lanes(tensors):
+    """Known-start plan at full size: every weight compared with the input."""
+    enc = dfw.encode_multi(tensors, 32)
+    dl = dfw.DeviceLanes.upload(enc, dfw.plan_lanes(enc))
+    out = dfw.decode_lanes(dl)
+    dfw.check()
+    assert torch.equal(out.view(torch.int16), torch.cat(tensors).to("cuda").view(torch.int16))
+
+
 @pytest.mark.parametrize("name", ["c1", "c2", "c4a", "c4b", "c4bp", "c4c"])
 def test_full_size_tensor_configs(oracle, name):
     block = {"c1": workloads.c1(), "c2": workloads.c2(), "c4a": workloads.c4("a"), "c4b": workloads.c4("b"),
@@ -203,11 +227,13 @@ def test_full_size_tensor_configs(oracle, name):
         assert int(enc.lengths.max()) == 32  # the cap binds
     if name == "c4c":
         assert np.all(enc.lengths == 8)
+    _full_lanes([t.cpu() for t in ts])
 
 
 def test_full_size_block_c3(oracle):
     ts = [t.cpu() for t in workloads.generate_block(workloads.c3(), "cuda")]
     _full_parity(oracle, ts, block=True)
+    _full_lanes(ts)
 
 
 def test_full_size_c5_blocks(oracle):
@@ -216,6 +242,7 @@ def test_full_size_c5_blocks(oracle):
     for blk in (blocks[1], blocks[0]):
         ts = [t.cpu() for t in workloads.generate_block(blk, "cuda")]
         _full_parity(oracle, ts, block=True, samples=4)
+        _full_lanes(ts)
 
 
 # ------------------------------------------------------------ corruption
@@ -263,3 +290,32 @@ def test_bad_device_arguments_rejected_before_launch():
     with pytest.raises(dfw.DfwError) as ei:
         dfw.decode(dev, out=out[1:])  # 2-byte offset: not 16-byte aligned
     assert ei.value.status == dfw.EALIGN
+
+
+def test_lanes_corrupt_aux_and_stream_detected():
+    u = SMALL["c1"]()
+    enc = dfw.encode(u)
+    pl = dfw.plan_lanes(enc)
+    dl = dfw.DeviceLanes.upload(enc, pl)
+
+    def status():
+        out = torch.zeros(dl.n, dtype=torch.bfloat16, device="cuda")
+        dfw.decode_lanes(dl, out)
+        return dfw.check_status(), out
+
+    assert status()[0] == dfw.OK
+    dl.chunk_bits[40] += 3  # chunk bits no longer add up to the group span
+    assert status()[0] == dfw.ECORRUPT
+    dl.chunk_bits.copy_(pl.chunk_bits.to("cuda"))
+    dl.group_start[3] += 1  # group starts one bit late: its lanes end in the wrong place
+    assert status()[0] == dfw.ECORRUPT
+    dl.group_start.copy_(pl.group_start.to("cuda"))
+    dl.lut[9] = 0  # a fast-table entry with no codewords and no escape mark
+    assert status()[0] == dfw.ECORRUPT
+    dl.lut.copy_(pl.lut.to("cuda"))
+    half = dl.stream.numel() // 2
+    dl.stream[half: half + 64] = 0  # zero bits: lanes end before their chunk bits say
+    assert status()[0] == dfw.ECORRUPT
+    dl.stream.copy_(enc.stream.to("cuda"))
+    st, out = status()
+    assert st == dfw.OK and np.array_equal(workloads.as_u16_numpy(out), u)

@@ -332,3 +332,30 @@ def test_decode_host_validation_without_gpu():
     st = L.dfw_decode_block(None, None, None, None, None, ctypes.byref(enc.table), ctypes.byref(pl.info),
                             offs.ctypes.data, 1, None, enc.n - 1, None)
     assert st == dfw.ENOMEM
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c4a", "c4b", "c4c", "tiny", "single"])
+def test_plan_lanes_matches_oracle(oracle, name):
+    u = CASES[name]()
+    enc = dfw.encode(u, 32, n_threads=2)
+    oenc = oracle.encode(u, 32)
+    pl = dfw.plan_lanes(enc)
+    bits, starts = oracle.chunk_aux(oenc, 64, 32)
+    assert pl.info.n_chunks == -(-u.size // 64) and pl.info.n_groups == starts.size - 1
+    got_bits = pl.chunk_bits.numpy().view(np.uint16)[: bits.size]
+    assert np.array_equal(got_bits.astype(np.uint32), bits)
+    assert np.array_equal(pl.group_start.numpy().view(np.uint64), starts)
+    spans = [((((int(starts[g + 1]) + 7) >> 3) + 8 + 15) & ~15) - ((int(starts[g]) >> 3) & ~15)
+             for g in range(starts.size - 1)]
+    if enc.total_bits:
+        assert pl.info.max_group_bytes == max(spans + [16])
+    fast, hier = _split_lut(dfw.Plan(pl.chunk_bits, pl.group_start, pl.lut, pl.info))
+
+
+def test_plan_lanes_detects_corrupt_stream():
+    enc = dfw.encode(CASES["c1"](), 32)
+    bad = dfw.Encoded(enc.stream, enc.mant, dfw.Table.from_buffer_copy(enc.table))
+    bad.table.n = enc.table.n + 1  # one codeword more than the stream holds
+    with pytest.raises(dfw.DfwError) as ei:
+        dfw.plan_lanes(bad)
+    assert ei.value.status in (dfw.ECORRUPT, dfw.EINVAL)

@@ -491,3 +491,32 @@ def test_aux_window_without_code_start(oracle):
     assert list(gap) == [0, 1]
     assert list(out_start) == [0, 31, 31]
     assert np.array_equal(oracle.decode(enc), u)
+
+
+@pytest.mark.parametrize("M,G", [(64, 32), (4, 3), (1, 1), (7, 5)])
+@pytest.mark.parametrize("kind", ["c1", "c4b", "single"])
+def test_chunk_aux_against_independent_walk(oracle, M, G, kind):
+    if kind == "single":
+        u = ((np.arange(999) % 2) << 15 | (121 << 7)).astype(np.uint16)
+    else:
+        block = workloads.scaled(workloads.c1() if kind == "c1" else workloads.c4("b"), 10_007)
+        u = workloads.as_u16_numpy(workloads.generate(block.tensors[0]))
+    enc = oracle.encode(u)
+    bits, starts = oracle.chunk_aux(enc, M, G)
+    if enc.total_bits:
+        st, _ = walk_code_starts(enc.stream, enc.total_bits, enc.lengths)
+    else:
+        st = [0] * u.size
+    st = list(st) + [enc.total_bits]
+    n_chunks = -(-u.size // M)
+    n_groups = -(-n_chunks // G)
+    assert bits.size == n_groups * G and starts.size == n_groups + 1
+    for c in range(n_groups * G):
+        if c < n_chunks:
+            assert bits[c] == st[min(M * (c + 1), u.size)] - st[M * c]
+        else:
+            assert bits[c] == 0
+    for g in range(n_groups):
+        assert starts[g] == st[M * G * g]
+    assert starts[-1] == enc.total_bits
+    assert int(bits.sum()) == enc.total_bits
