@@ -16,9 +16,11 @@
 //     (up to four codewords per lookup) into its own word slots, interleaved
 //     by lane so stores never conflict;
 //   - each lane joins exponents and raw bytes into bf16, 16 at a time in a
-//     lane-rotated order (which spreads the 128-bit shared accesses over the
-//     banks), into the warp's staging buffer in output order; lane 0 then
-//     writes the group's 4 KB with one TMA bulk store.
+//     lane-rotated order (which spreads the 128-bit shared reads over the
+//     banks), and stores its chunk's 128 output bytes straight from
+//     registers with 128-bit stores (each lane's bytes are contiguous, so L2
+//     receives whole sectors); no staging buffer is needed, which leaves
+//     shared memory for up to 32 warps per SM.
 // No count phase, no block scan, no CTA barrier after the table load, and no
 // realignment: every chunk's output is 64-weight aligned.
 //
@@ -55,7 +57,7 @@ __device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_
 }
 
 // Decodes `left8 / 8` codewords starting at bit r of the stream words held in
-// shared memory at sw (32-bit shared address), n_words of them, and appends
+// shared memory at sw (32-bit shared address) and appends
 // their symbols to this lane's word slots ep, ep + 128, ... (slots of the 32
 // lanes interleave; a last lookup may append up to three more symbols, which
 // are never read).  fast is the shared address of the
@@ -67,67 +69,65 @@ __device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_
 // always stores the accumulator's low word and advances by select.  Only an
 // escape or the chunk's last lookup leaves it, for one step of the general
 // path.
-__device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t n_words, uint32_t r, int left8,
-                                                 uint32_t fast, uint32_t kshift,
-                                                 const uint32_t *__restrict__ g_hier, uint32_t n_tables,
-                                                 uint32_t ep, uint32_t &err) {
-    const uint32_t w_end = sw + 4u * (n_words - 1u);  // last readable word
-    uint32_t wa = min(sw + 4u * (r >> 5), w_end);
+__device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int left8, uint32_t fast,
+                                                 uint32_t kshift, const uint32_t *__restrict__ g_hier,
+                                                 uint32_t n_tables, uint32_t ep, uint32_t &err) {
+    // The bit position is 8 * (wa - sw) - 64 + p: a and b hold the words just
+    // below wa.  Reads past the slot (only a corrupt stream causes them) stay
+    // inside this warp's shared area, and the caller's end check rejects it.
+    uint32_t wa = sw + 4u * (r >> 5);
     uint32_t a = bswap32(lds32(wa));
-    wa = min(wa + 4u, w_end);
-    uint32_t b = bswap32(lds32(wa));
-    wa = min(wa + 4u, w_end);  // the next word to shift in
-    uint32_t p = r & 31u, words = 0;  // bit position = 32 * ((r >> 5) + words) + p
-    uint32_t lo = 0u, hi = 0u, sh = 0u;
+    uint32_t b = bswap32(lds32(wa + 4u));
+    wa += 8u;
+    uint32_t p = r & 31u;
+    uint32_t lo = 0u, sh = 0u;
+    const uint32_t kmul = 1u << (32u - kshift);  // x >> kshift == mulhi(x, 2^(32 - kshift))
     while (left8 > 0) {
         uint32_t x, syms, c8, cb, ey;
         // straight-line loop in PTX; it exits on an escape (bits byte 255)
-        // or on the lookup that completes the chunk (8 * count >= left8)
+        // or on the lookup that completes the chunk (8 * count >= left8).
+        // Symbols are appended by multiplication (m = 2^sh: lo += syms * m,
+        // spill = mulhi(syms, m)) to keep work off the integer-logic pipe.
         asm volatile(
             "{\n\t"
             ".reg .pred pe, pl, pa, pf;\n\t"
-            ".reg .b32 t0, t1, ex, nx, ad;\n"
+            ".reg .b32 t0, t1, sp, ex, nx, ad;\n"
             "LANES_LOOP:\n\t"
-            "shf.l.wrap.b32 %0, %10, %9, %11;\n\t"  // x = stream bits [p, p + 32)
-            "shr.b32 t0, %0, %19;\n\t"
-            "mad.lo.u32 ad, t0, 8, %18;\n\t"
+            "shf.l.wrap.b32 %0, %9, %8, %10;\n\t"  // x = stream bits [p, p + 32)
+            "mul.hi.u32 t0, %0, %16;\n\t"          // fast-table key
+            "mad.lo.u32 ad, t0, 8, %15;\n\t"
             "ld.shared.v2.u32 {ex, %4}, [ad];\n\t"
-            "ld.shared.u32 nx, [%12];\n\t"  // the word after b
+            "ld.shared.u32 nx, [%11];\n\t"  // the word after b
             "and.b32 %3, %4, 255;\n\t"
             "prmt.b32 %2, %4, 0, 0x4441;\n\t"
             "setp.eq.u32 pe, %3, 255;\n\t"
-            "setp.ge.s32 pl, %2, %17;\n\t"
+            "setp.ge.s32 pl, %2, %14;\n\t"
             "or.pred pe, pe, pl;\n\t"
             "@pe bra LANES_EXIT;\n\t"
-            "add.u32 %11, %11, %3;\n\t"  // p += bits used
-            "setp.ge.u32 pa, %11, 32;\n\t"
+            "mad.lo.u32 %10, %3, 1, %10;\n\t"  // p += bits used
+            "setp.ge.u32 pa, %10, 32;\n\t"
             "prmt.b32 nx, nx, 0, 0x0123;\n\t"
-            "selp.b32 %9, %10, %9, pa;\n\t"  // a = b
-            "selp.b32 %10, nx, %10, pa;\n\t"  // b = next word
-            "@pa add.u32 %12, %12, 4;\n\t"
-            "min.u32 %12, %12, %20;\n\t"
-            "@pa add.u32 %13, %13, 1;\n\t"
-            "and.b32 %11, %11, 31;\n\t"
-            "shl.b32 t0, ex, %16;\n\t"  // append symbols at byte offset sh / 8
-            "or.b32 %14, %14, t0;\n\t"
-            "shf.l.wrap.b32 t1, ex, 0, %16;\n\t"
-            "or.b32 %15, %15, t1;\n\t"
-            "add.u32 %16, %16, %2;\n\t"
-            "st.shared.u32 [%8], %14;\n\t"
-            "setp.ge.u32 pf, %16, 32;\n\t"
-            "@pf add.u32 %8, %8, 128;\n\t"  // next word slot of this lane
-            "selp.b32 %14, %15, %14, pf;\n\t"
-            "selp.b32 %15, 0, %15, pf;\n\t"
-            "and.b32 %16, %16, 31;\n\t"
-            "sub.s32 %17, %17, %2;\n\t"
+            "selp.b32 %8, %9, %8, pa;\n\t"  // a = b
+            "selp.b32 %9, nx, %9, pa;\n\t"  // b = next word
+            "@pa add.u32 %11, %11, 4;\n\t"
+            "and.b32 %10, %10, 31;\n\t"
+            "shl.b32 t1, 1, %13;\n\t"  // m = 2^sh
+            "mad.lo.u32 %12, ex, t1, %12;\n\t"
+            "mul.hi.u32 sp, ex, t1;\n\t"
+            "mad.lo.u32 %13, %2, 1, %13;\n\t"  // sh += 8 * count
+            "st.shared.u32 [%7], %12;\n\t"
+            "setp.ge.u32 pf, %13, 32;\n\t"
+            "@pf add.u32 %7, %7, 128;\n\t"  // next word slot of this lane
+            "selp.b32 %12, sp, %12, pf;\n\t"
+            "and.b32 %13, %13, 31;\n\t"
+            "sub.s32 %14, %14, %2;\n\t"
             "bra LANES_LOOP;\n"
             "LANES_EXIT:\n\t"
             "mov.b32 %1, ex;\n\t"
             "}"
-            : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(err), "+r"(n_words), "+r"(r),
-              "+r"(ep), "+r"(a), "+r"(b), "+r"(p), "+r"(wa), "+r"(words), "+r"(lo), "+r"(hi), "+r"(sh),
-              "+r"(left8)
-            : "r"(fast), "r"(kshift), "r"(w_end)
+            : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(err), "+r"(r), "+r"(ep), "+r"(a), "+r"(b),
+              "+r"(p), "+r"(wa), "+r"(lo), "+r"(sh), "+r"(left8)
+            : "r"(fast), "r"(kmul)
             : "memory");
         if (cb != 255u) {
             // the chunk's last lookup: later codewords belong to the next
@@ -136,10 +136,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t n_words, 
             for (int i = 8; i < left8; i += 8) ends &= ends - 1u;
             cb = (uint32_t)__ffs(ends);
             c8 = (uint32_t)left8;
-        }
-        // one general step: an escape (codeword longer than the fast key) or
-        // the chunk's last lookup
-        if (cb == 255u) {
+        } else {  // first codeword longer than the fast key
             const uint32_t f = resolve_escape(x, g_hier, n_tables);
             if (f & ESC_BAD) err |= ST_LUT;
             syms = f & 0xFFu;
@@ -150,31 +147,29 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t n_words, 
         if (p >= 32u) {
             a = b;
             b = bswap32(lds32(wa));
-            wa = min(wa + 4u, w_end);
-            ++words;
+            wa += 4u;
             p -= 32u;
         }
+        const uint32_t hi = __funnelshift_l(syms, 0u, sh);
         lo |= syms << sh;
-        hi |= __funnelshift_l(syms, 0u, sh);
         sh += c8;
         if (sh >= 32u) {
             sts32(ep, lo);
             ep += 128u;
             lo = hi;
-            hi = 0u;
             sh -= 32u;
         }
         left8 -= (int)c8;
     }
     if (sh) sts32(ep, lo);
-    return 32u * ((r >> 5) + words) + p;
+    return 8u * (wa - sw) - 64u + p;
 }
 
 // Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes) | 2 x
-// (chunk_bits | stream span) | raw bytes (2048) | bf16 staging (4096) |
-// exponent word slots (EXP_WORDS x 32).
+// (chunk_bits | stream span) | raw bytes (2048) | exponent word slots
+// (EXP_WORDS x 32).
 __host__ __device__ constexpr uint32_t warp_smem_bytes(uint32_t sbuf_bytes) {
-    return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + 2u * GROUP_SYMS + 4u * EXP_WORDS * 32u;
+    return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + 4u * EXP_WORDS * 32u;
 }
 
 template <int NT>
@@ -190,8 +185,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
     uint8_t *wslots = wbase + 32;
     const uint32_t slot_bytes = 64u + prm.sbuf_bytes;
     uint8_t *mbuf = wslots + 2u * slot_bytes;
-    uint8_t *stage = mbuf + GROUP_SYMS;
-    const uint32_t exps = smem_u32(stage + 2u * GROUP_SYMS) + 4u * lane;  // word k at exps + 128 k
+    const uint32_t exps = smem_u32(mbuf + GROUP_SYMS) + 4u * lane;  // word k at exps + 128 k
     const uint32_t *g_hier = prm.lut + 2u * n_fast;
     const uint32_t kshift = 32u - prm.fast_bits;
 
@@ -291,17 +285,15 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         uint32_t err = 0;
         if (ok && valid && t) {
             const uint32_t r = (uint32_t)(gs0 - 8ull * sb0) + excl;
-            const uint32_t end = decode_chunk(smem_u32(slot + 64), prm.sbuf_bytes / 4u, r, (int)(8u * t),
-                                              smem_u32(s_fast), kshift, g_hier, prm.n_tables, exps, err);
+            const uint32_t end = decode_chunk(smem_u32(slot + 64), r, (int)(8u * t), smem_u32(s_fast), kshift,
+                                              g_hier, prm.n_tables, exps, err);
             if (end != r + cbits) err |= ST_COUNT;
         }
         ok = mbar_wait_bounded(bar_m, k & 1u) && ok;
-        if (lane == 0) bulk_wait_read();  // the previous group's store has read the staging buffer
         if (!__all_sync(0xFFFFFFFFu, ok)) {  // a bulk copy never completed: give up
             if (lane == 0) {
                 atomicOr(&g_status, ST_TIMEOUT);
                 if (has_next) mbar_wait_bounded(bar_s0 + 8u * (s ^ 1u), ((k + 1) >> 1) & 1u);
-                bulk_wait_all();
             }
             return;
         }
@@ -313,7 +305,8 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         } else {
             // join: piece q (16 weights) of this lane's chunk, in the order
             // (j + lane / 2) mod 4 so lanes spread over the banks
-            const uint32_t mrow = smem_u32(mbuf) + 64u * lane, orow = smem_u32(stage) + 128u * lane;
+            const uint32_t mrow = smem_u32(mbuf) + 64u * lane;
+            uint16_t *dst = prm.out + LANE_SYMS * c;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
@@ -325,18 +318,16 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
                 join4(e1, m.y, r0.z, r0.w);
                 join4(e2, m.z, r1.x, r1.y);
                 join4(e3, m.w, r1.z, r1.w);
-                sts128(orow + 32u * q, r0);
-                sts128(orow + 32u * q + 16u, r1);
-            }
-            fence_proxy_async();
-            __syncwarp();
-            const uint64_t w0 = g * (uint64_t)GROUP_SYMS;
-            const uint32_t gw = (uint32_t)min((uint64_t)GROUP_SYMS, prm.n - w0);  // weights in this group
-            const uint32_t body = gw & ~7u;
-            if (lane == 0 && body) bulk_store(prm.out + w0, smem_u32(stage), 2u * body);
-            if (lane < (int)(gw - body)) {
-                const uint32_t i = body + lane;
-                prm.out[w0 + i] = reinterpret_cast<const uint16_t *>(stage)[i];
+                if (16u * q + 16u <= t) {
+                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q), r0);
+                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q + 8u), r1);
+                } else {  // the last, partial chunk of the tensor: one weight at a time
+                    for (uint32_t i = 16u * q; i < t; ++i) {
+                        const uint32_t e = (lds32(exps + 128u * (i >> 2)) >> (8u * (i & 3u))) & 0xFFu;
+                        const uint32_t mb = (lds32(mrow + (i & ~3u)) >> (8u * (i & 3u))) & 0xFFu;
+                        dst[i] = join1(e, mb);
+                    }
+                }
             }
         }
         if (!has_next) break;
@@ -349,7 +340,6 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         ns0 = ms0;
         ns1 = ms1;
     }
-    if (lane == 0) bulk_wait_all();
 }
 
 template <int NT>
@@ -368,6 +358,8 @@ struct LanesVariant {
 // more warps; data with long codes needs bigger stream slots and falls back
 // to a smaller CTA.
 LanesVariant g_lanes[] = {
+    {1024, decode_lanes<1024>, lanes_smem<1024>, {0}},
+    {768, decode_lanes<768>, lanes_smem<768>, {0}},
     {512, decode_lanes<512>, lanes_smem<512>, {0}},
     {256, decode_lanes<256>, lanes_smem<256>, {0}},
     {128, decode_lanes<128>, lanes_smem<128>, {0}},
