@@ -40,6 +40,8 @@ import workloads  # noqa: E402
 METRIC = "decoded bf16 weights/sec & effective GB/s as % of HBM roofline; compression ratio"
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["lossless_entropy_coded_canonical_b200/csrc/dfw_decode.cu",
+                  "lossless_entropy_coded_canonical_b200/csrc/dfw_lanes.cuh",
+                  "lossless_entropy_coded_canonical_b200/csrc/dfw_device.cuh",
                   "lossless_entropy_coded_canonical_b200/csrc/dfw_internal.h"]
 
 
@@ -71,10 +73,10 @@ def measured_peak_hbm():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def committed_traffic(workload: str):
+def committed_traffic(kernel: str):
     """Per-weight DRAM traffic of the decode kernel from a committed ncu
     summary, used only if it was taken on the current kernel source."""
-    p = os.path.join(ROOT, "profiles", f"decode_tiles_{workload}_traffic.txt")
+    p = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     if not os.path.exists(p):
         return None
     kv = {}
@@ -344,7 +346,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="c5")
     ap.add_argument("--window", type=int, default=8)
     ap.add_argument("--tile", type=int, default=256)
-    ap.add_argument("--variant", default="window", choices=["window", "lanes"],
+    ap.add_argument("--variant", default="lanes", choices=["window", "lanes"],
                     help="window: gap/out_start plan (count phase + scan); lanes: known-start chunks")
     ap.add_argument("--threads", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
@@ -395,7 +397,8 @@ def main(argv=None):
     mean_launch_ms = launch_ms.mean(axis=0)
     achieved = alg_bytes / (mean_launch_ms.sum() * 1e-3) / 1e9
     peak, peak_kind = measured_peak_hbm()
-    tpw = committed_traffic(args.workload)
+    kernel = "decode_lanes" if args.variant == "lanes" else "decode_tiles"
+    tpw = committed_traffic(kernel)
     traffic = None if tpw is None else tpw * n_total / len(devs)
 
     e2e = None
@@ -430,7 +433,7 @@ def main(argv=None):
         "bits_per_weight": 8 * comp / n_total,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "peak_source": peak_kind,
-                     "kernel": "decode_lanes" if args.variant == "lanes" else "decode_tiles",
+                     "kernel": kernel,
                      "algorithmic_bytes_per_step": alg_bytes,
                      "mean_launch_ms": float(mean_launch_ms.mean())},
         "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": args.steps * len(devs),

@@ -110,6 +110,14 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
     asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 
+// 32-byte streaming store (sm_100 256-bit vector store): one whole L2 sector
+// per thread; the address must be 32-byte aligned.
+__device__ __forceinline__ void stg256_cs(void *p, uint4 a, uint4 b) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y),
+                 "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+
 // --------------------------------------------------------------- decoding
 
 // A codeword longer than the fast table's key: walk the byte-keyed hierarchy

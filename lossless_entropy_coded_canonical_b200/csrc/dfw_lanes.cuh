@@ -18,9 +18,9 @@
 //   - each lane joins exponents and raw bytes into bf16, 16 at a time in a
 //     lane-rotated order (which spreads the 128-bit shared reads over the
 //     banks), and stores its chunk's 128 output bytes straight from
-//     registers with 128-bit stores (each lane's bytes are contiguous, so L2
-//     receives whole sectors); no staging buffer is needed, which leaves
-//     shared memory for up to 32 warps per SM.
+//     registers, one whole 32-byte sector per 256-bit store (two 128-bit
+//     stores when the output is only 16-byte aligned); no staging buffer is
+//     needed, which leaves shared memory for up to 32 warps per SM.
 // No count phase, no block scan, no CTA barrier after the table load, and no
 // realignment: every chunk's output is 64-weight aligned.
 //
@@ -48,6 +48,7 @@ struct LanesParams {
     uint16_t *out;
     uint64_t n, n_chunks, n_groups, stream_bytes, mant_bytes;
     uint32_t fast_bits, n_tables, sbuf_bytes;
+    uint32_t out32;  // out is 32-byte aligned: one 256-bit store per 16 weights
 };
 
 __device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_bit) {
@@ -319,8 +320,12 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
                 join4(e2, m.z, r1.x, r1.y);
                 join4(e3, m.w, r1.z, r1.w);
                 if (16u * q + 16u <= t) {
-                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q), r0);
-                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q + 8u), r1);
+                    if (prm.out32) {
+                        stg256_cs(dst + 16u * q, r0, r1);  // a whole sector per lane
+                    } else {
+                        __stcs(reinterpret_cast<uint4 *>(dst + 16u * q), r0);
+                        __stcs(reinterpret_cast<uint4 *>(dst + 16u * q + 8u), r1);
+                    }
                 } else {  // the last, partial chunk of the tensor: one weight at a time
                     for (uint32_t i = 16u * q; i < t; ++i) {
                         const uint32_t e = (lds32(exps + 128u * (i >> 2)) >> (8u * (i & 3u))) & 0xFFu;
@@ -400,6 +405,7 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     prm.fast_bits = fb;
     prm.n_tables = info->lut_tables;
     prm.sbuf_bytes = info->max_group_bytes;
+    prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
     for (LanesVariant &v : g_lanes) {

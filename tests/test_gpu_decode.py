@@ -319,3 +319,22 @@ def test_lanes_corrupt_aux_and_stream_detected():
     dl.stream.copy_(enc.stream.to("cuda"))
     st, out = status()
     assert st == dfw.OK and np.array_equal(workloads.as_u16_numpy(out), u)
+
+
+@pytest.mark.parametrize("offset", [0, 8, 16, 24])
+def test_lanes_output_alignment(oracle, offset):
+    """Known-start plan into an output that starts 0, 16, 32 or 48 bytes into
+    a buffer: 32-byte aligned outputs take one 256-bit store per 16 weights,
+    16-byte aligned ones two 128-bit stores; both must give the same bits
+    and leave the bytes around the output untouched."""
+    u = SMALL["c2"]()
+    oenc = oracle.encode(u, 32)
+    enc = encoded_from_oracle(oenc)
+    dl = dfw.DeviceLanes.upload(enc, dfw.plan_lanes(enc))
+    buf = torch.zeros(enc.n + 64, dtype=torch.bfloat16, device="cuda")
+    out = buf[offset: offset + enc.n]
+    dfw.decode_lanes(dl, out)
+    dfw.check()
+    assert np.array_equal(workloads.as_u16_numpy(out), oracle.decode(oenc))
+    whole = workloads.as_u16_numpy(buf)
+    assert not whole[:offset].any() and not whole[offset + enc.n:].any()
