@@ -65,69 +65,74 @@ __device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_
 // fast table.  Returns the stream bit position (relative to sw) after the
 // last codeword decoded.
 //
-// The inner loop is straight-line code: it always loads the word after the
-// current pair and selects it in when the position crosses a word, and it
-// always stores the accumulator's low word and advances by select.  Only an
-// escape or the chunk's last lookup leaves it, for one step of the general
-// path.
+// The inner loop is straight-line code: it keeps the word after the current
+// pair in a register, selects it in when the position crosses a word (and
+// only then loads the next one), and it always stores the accumulator's low
+// word and advances by select.  Only an escape or the chunk's last lookup
+// leaves it, for one step of the general path.
 __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int left8, uint32_t fast,
                                                  uint32_t kshift, const uint32_t *__restrict__ g_hier,
                                                  uint32_t n_tables, uint32_t ep, uint32_t &err) {
-    // The bit position is 8 * (wa - sw) - 64 + p: a and b hold the words just
-    // below wa.  Reads past the slot (only a corrupt stream causes them) stay
-    // inside this warp's shared area, and the caller's end check rejects it.
+    // a and b hold the two stream words the window [p, p + 32) lies in, c
+    // the word after them (not yet byte-swapped), wa the address of the word
+    // after c: the bit position is 8 * (wa - sw) - 96 + p.  Reads past the
+    // slot (only a corrupt stream causes them) stay inside this warp's shared
+    // area, and the caller's end check rejects it.
     uint32_t wa = sw + 4u * (r >> 5);
     uint32_t a = bswap32(lds32(wa));
     uint32_t b = bswap32(lds32(wa + 4u));
-    wa += 8u;
+    uint32_t c = lds32(wa + 8u);
+    wa += 12u;
     uint32_t p = r & 31u;
     uint32_t lo = 0u, sh = 0u;
     const uint32_t kmul = 1u << (32u - kshift);  // x >> kshift == mulhi(x, 2^(32 - kshift))
     while (left8 > 0) {
         uint32_t x, syms, c8, cb, ey;
-        // straight-line loop in PTX; it exits on an escape (bits byte 255)
-        // or on the lookup that completes the chunk (8 * count >= left8).
-        // Symbols are appended by multiplication (m = 2^sh: lo += syms * m,
-        // spill = mulhi(syms, m)) to keep work off the integer-logic pipe.
+        // straight-line loop in PTX; it exits on the lookup that completes
+        // the chunk (8 * count >= left8) or on an escape, whose count byte
+        // reads as all ones through the sign-replicating byte permute (the
+        // escape flag is the entry's top bit).  The next stream word is
+        // loaded only when the window crosses into c, one lookup ahead of its
+        // use.  Symbols are appended by multiplication (m = 2^sh: lo += syms
+        // * m, spill = mulhi(syms, m)) to keep work off the integer-logic
+        // pipe.
         asm volatile(
             "{\n\t"
-            ".reg .pred pe, pl, pa, pf;\n\t"
+            ".reg .pred pl, pa, pf;\n\t"
             ".reg .b32 t0, t1, sp, ex, nx, ad;\n"
             "LANES_LOOP:\n\t"
-            "shf.l.wrap.b32 %0, %9, %8, %10;\n\t"  // x = stream bits [p, p + 32)
-            "mul.hi.u32 t0, %0, %16;\n\t"          // fast-table key
-            "mad.lo.u32 ad, t0, 8, %15;\n\t"
+            "shf.l.wrap.b32 %0, %7, %6, %9;\n\t"  // x = stream bits [p, p + 32)
+            "mul.hi.u32 t0, %0, %15;\n\t"         // fast-table key
+            "mad.lo.u32 ad, t0, 8, %14;\n\t"
             "ld.shared.v2.u32 {ex, %4}, [ad];\n\t"
-            "ld.shared.u32 nx, [%11];\n\t"  // the word after b
             "and.b32 %3, %4, 255;\n\t"
-            "prmt.b32 %2, %4, 0, 0x4441;\n\t"
-            "setp.eq.u32 pe, %3, 255;\n\t"
-            "setp.ge.s32 pl, %2, %14;\n\t"
-            "or.pred pe, pe, pl;\n\t"
-            "@pe bra LANES_EXIT;\n\t"
-            "mad.lo.u32 %10, %3, 1, %10;\n\t"  // p += bits used
-            "setp.ge.u32 pa, %10, 32;\n\t"
-            "prmt.b32 nx, nx, 0, 0x0123;\n\t"
-            "selp.b32 %8, %9, %8, pa;\n\t"  // a = b
-            "selp.b32 %9, nx, %9, pa;\n\t"  // b = next word
-            "@pa add.u32 %11, %11, 4;\n\t"
-            "and.b32 %10, %10, 31;\n\t"
-            "shl.b32 t1, 1, %13;\n\t"  // m = 2^sh
-            "mad.lo.u32 %12, ex, t1, %12;\n\t"
+            "prmt.b32 %2, %4, 0, 0xBBB1;\n\t"
+            "setp.ge.u32 pl, %2, %13;\n\t"
+            "@pl bra LANES_EXIT;\n\t"
+            "mad.lo.u32 %9, %3, 1, %9;\n\t"  // p += bits used
+            "setp.ge.u32 pa, %9, 32;\n\t"
+            "prmt.b32 nx, %8, 0, 0x0123;\n\t"
+            "selp.b32 %6, %7, %6, pa;\n\t"  // a = b
+            "selp.b32 %7, nx, %7, pa;\n\t"  // b = c
+            "@pa ld.shared.u32 %8, [%10];\n\t"
+            "@pa add.u32 %10, %10, 4;\n\t"
+            "and.b32 %9, %9, 31;\n\t"
+            "shl.b32 t1, 1, %12;\n\t"  // m = 2^sh
+            "mad.lo.u32 %11, ex, t1, %11;\n\t"
             "mul.hi.u32 sp, ex, t1;\n\t"
-            "mad.lo.u32 %13, %2, 1, %13;\n\t"  // sh += 8 * count
-            "st.shared.u32 [%7], %12;\n\t"
-            "setp.ge.u32 pf, %13, 32;\n\t"
-            "@pf add.u32 %7, %7, 128;\n\t"  // next word slot of this lane
-            "selp.b32 %12, sp, %12, pf;\n\t"
-            "and.b32 %13, %13, 31;\n\t"
-            "sub.s32 %14, %14, %2;\n\t"
+            "mad.lo.u32 %12, %2, 1, %12;\n\t"  // sh += 8 * count
+            "st.shared.u32 [%5], %11;\n\t"
+            "setp.ge.u32 pf, %12, 32;\n\t"
+            "@pf add.u32 %5, %5, 128;\n\t"  // next word slot of this lane
+            "selp.b32 %11, sp, %11, pf;\n\t"
+            "and.b32 %12, %12, 31;\n\t"
+            "sub.s32 %13, %13, %2;\n\t"
             "bra LANES_LOOP;\n"
             "LANES_EXIT:\n\t"
             "mov.b32 %1, ex;\n\t"
             "}"
-            : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(err), "+r"(r), "+r"(ep), "+r"(a), "+r"(b),
-              "+r"(p), "+r"(wa), "+r"(lo), "+r"(sh), "+r"(left8)
+            : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(ep), "+r"(a), "+r"(b), "+r"(c), "+r"(p),
+              "+r"(wa), "+r"(lo), "+r"(sh), "+r"(left8)
             : "r"(fast), "r"(kmul)
             : "memory");
         if (cb != 255u) {
@@ -147,7 +152,8 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         p += cb;
         if (p >= 32u) {
             a = b;
-            b = bswap32(lds32(wa));
+            b = bswap32(c);
+            c = lds32(wa);
             wa += 4u;
             p -= 32u;
         }
@@ -163,7 +169,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         left8 -= (int)c8;
     }
     if (sh) sts32(ep, lo);
-    return 8u * (wa - sw) - 64u + p;
+    return 8u * (wa - sw) - 96u + p;
 }
 
 // Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes) | 2 x
