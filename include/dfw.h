@@ -257,7 +257,9 @@ dfw_status dfw_plan_lanes(const uint8_t *stream, const dfw_table *table, uint16_
  * plan, asynchronous on cuda_stream.  Device buffers: d_stream
  * (table->stream_bytes), d_mant (dfw_mant_bytes(n)), d_lut (lut_words),
  * d_chunk_bits (32 * n_groups u16), d_group_start (n_groups + 1 u64), d_out
- * (n bf16).  Errors as dfw_decode; a group whose chunk bits disagree with
+ * (n bf16; 32-byte alignment lets the kernel store whole 32-byte sectors).
+ * n must be below 2^38 (chunk indices are 32-bit; DFW_EINVAL otherwise).
+ * Errors as dfw_decode; a group whose chunk bits disagree with
  * group_start, or whose codewords do not end where chunk_bits says, writes
  * nothing / is flagged through dfw_check.
  */

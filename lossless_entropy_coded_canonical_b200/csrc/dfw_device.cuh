@@ -85,6 +85,12 @@ __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
     return false;
 }
 
+// Waits for a phase of an mbarrier: one inline try (the copy has usually
+// landed by now), the bounded loop only if that fails.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    return mbar_try_wait(bar, parity) || mbar_wait_bounded(bar, parity);
+}
+
 __device__ __forceinline__ uint32_t bswap32(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
 
 // Shared-memory accesses by 32-bit shared-window address.

@@ -46,7 +46,9 @@ struct LanesParams {
     const uint16_t *chunk_bits;
     const uint64_t *group_start;
     uint16_t *out;
-    uint64_t n, n_chunks, n_groups, stream_bytes, mant_bytes;
+    uint64_t stream_bytes, mant_bytes;
+    uint32_t n_chunks, n_groups;  // both below 2^32 (checked on the host)
+    uint32_t last_t;              // codewords in the last chunk (1..64)
     uint32_t fast_bits, n_tables, sbuf_bytes;
     uint32_t out32;  // out is 32-byte aligned: one 256-bit store per 16 weights
 };
@@ -126,7 +128,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             "@pf add.u32 %5, %5, 128;\n\t"  // next word slot of this lane
             "selp.b32 %11, sp, %11, pf;\n\t"
             "and.b32 %12, %12, 31;\n\t"
-            "sub.s32 %13, %13, %2;\n\t"
+            "mad.lo.s32 %13, %2, -1, %13;\n\t"  // left8 -= 8 * count
             "bra LANES_LOOP;\n"
             "LANES_EXIT:\n\t"
             "mov.b32 %1, ex;\n\t"
@@ -221,12 +223,12 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         return;
     }
 
-    const uint64_t gstride = (uint64_t)gridDim.x * NWARP;
-    uint64_t g = (uint64_t)blockIdx.x * NWARP + warp;
+    const uint32_t gstride = gridDim.x * NWARP;
+    uint32_t g = blockIdx.x * NWARP + warp;
     if (g >= prm.n_groups) return;  // no CTA barrier follows
 
     // lane 0: chunk_bits and stream span of group gg into slot s
-    auto issue_stream = [&](uint64_t gg, uint32_t s, uint64_t s0, uint64_t s1) {
+    auto issue_stream = [&](uint32_t gg, uint32_t s, uint64_t s0, uint64_t s1) {
         uint8_t *slot = wslots + s * slot_bytes;
         const uint32_t bar = bar_s0 + 8u * s;
         const uint64_t sb0 = (s0 >> 3) & ~15ull;
@@ -237,12 +239,12 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         }
         fence_proxy_async();
         mbar_expect_tx(bar, 64u + sbytes);
-        bulk_load(smem_u32(slot), prm.chunk_bits + gg * GROUP_CHUNKS, 64u, bar);
+        bulk_load(smem_u32(slot), prm.chunk_bits + (size_t)gg * GROUP_CHUNKS, 64u, bar);
         if (sbytes) bulk_load(smem_u32(slot + 64), prm.stream + sb0, sbytes, bar);
     };
     // lane 0: the group's raw bytes into the warp buffer
-    auto issue_mant = [&](uint64_t gg) {
-        const uint64_t m0 = gg * (uint64_t)GROUP_SYMS;
+    auto issue_mant = [&](uint32_t gg) {
+        const uint64_t m0 = (uint64_t)gg * GROUP_SYMS;
         const uint32_t bytes = (uint32_t)min((uint64_t)GROUP_SYMS, prm.mant_bytes - m0);
         fence_proxy_async();
         mbar_expect_tx(bar_m, bytes);
@@ -250,7 +252,8 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
     };
 
     uint64_t gs0 = __ldg(prm.group_start + g), gs1 = __ldg(prm.group_start + g + 1);
-    uint64_t g1 = g + gstride, ns0 = 0, ns1 = 0;
+    uint32_t g1 = g + gstride;
+    uint64_t ns0 = 0, ns1 = 0;
     if (g1 < prm.n_groups) {
         ns0 = __ldg(prm.group_start + g1);
         ns1 = __ldg(prm.group_start + g1 + 1);
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         const uint32_t s = k & 1u;
         const uint8_t *slot = wslots + s * slot_bytes;
         const bool has_next = g1 < prm.n_groups;
-        const uint64_t g2 = g1 + gstride;
+        const uint32_t g2 = g1 + gstride;
         uint64_t ms0 = 0, ms1 = 0;
         if (g2 < prm.n_groups) {  // starts two groups ahead, for the copy issued next round
             ms0 = __ldg(prm.group_start + g2);
@@ -273,7 +276,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         __syncwarp();  // every lane is done with the other slot
         if (has_next && lane == 0) issue_stream(g1, s ^ 1u, ns0, ns1);
 
-        bool ok = mbar_wait_bounded(bar_s0 + 8u * s, (k >> 1) & 1u);
+        bool ok = mbar_wait(bar_s0 + 8u * s, (k >> 1) & 1u);
         const uint32_t cbits = reinterpret_cast<const uint16_t *>(slot)[lane];
         uint32_t incl = cbits;
 #pragma unroll
@@ -282,8 +285,8 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
             if (lane >= d) incl += y;
         }
         const uint32_t excl = incl - cbits, gbits = __shfl_sync(0xFFFFFFFFu, incl, 31);
-        const uint64_t c = g * GROUP_CHUNKS + lane;
-        const uint32_t t = c < prm.n_chunks ? (uint32_t)min((uint64_t)LANE_SYMS, prm.n - LANE_SYMS * c) : 0u;
+        const uint32_t c = g * GROUP_CHUNKS + lane;
+        const uint32_t t = c + 1u < prm.n_chunks ? LANE_SYMS : (c + 1u == prm.n_chunks ? prm.last_t : 0u);
         const uint64_t sb0 = (gs0 >> 3) & ~15ull;
         const bool valid = __all_sync(0xFFFFFFFFu, gs1 >= gs0 && gs1 - gs0 == gbits && cbits <= 32u * LANE_SYMS &&
                                                        span_bytes(gs0, gs1) <= prm.sbuf_bytes &&
@@ -296,7 +299,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
                                               g_hier, prm.n_tables, exps, err);
             if (end != r + cbits) err |= ST_COUNT;
         }
-        ok = mbar_wait_bounded(bar_m, k & 1u) && ok;
+        ok = mbar_wait(bar_m, k & 1u) && ok;
         if (!__all_sync(0xFFFFFFFFu, ok)) {  // a bulk copy never completed: give up
             if (lane == 0) {
                 atomicOr(&g_status, ST_TIMEOUT);
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
             // join: piece q (16 weights) of this lane's chunk, in the order
             // (j + lane / 2) mod 4 so lanes spread over the banks
             const uint32_t mrow = smem_u32(mbuf) + 64u * lane;
-            uint16_t *dst = prm.out + LANE_SYMS * c;
+            uint16_t *dst = prm.out + (size_t)c * LANE_SYMS;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
@@ -384,7 +387,7 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     const uint64_t n = table->n;
     if (info->chunk_symbols != LANE_SYMS || info->group_chunks != GROUP_CHUNKS ||
         info->n_chunks != (n + LANE_SYMS - 1) / LANE_SYMS ||
-        info->n_groups != (info->n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS)
+        info->n_groups != (info->n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS || info->n_chunks >= (1ull << 32))
         return DFW_EINVAL;
     const uint32_t fb = info->fast_bits;
     if (fb < (uint32_t)FAST_BITS_MIN || fb > (uint32_t)FAST_BITS_MAX || info->lut_tables < 1 ||
@@ -403,9 +406,9 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     prm.chunk_bits = d_chunk_bits;
     prm.group_start = d_group_start;
     prm.out = d_out;
-    prm.n = n;
-    prm.n_chunks = info->n_chunks;
-    prm.n_groups = info->n_groups;
+    prm.n_chunks = (uint32_t)info->n_chunks;
+    prm.n_groups = (uint32_t)info->n_groups;
+    prm.last_t = (uint32_t)(n - LANE_SYMS * (info->n_chunks - 1));
     prm.stream_bytes = table->stream_bytes;
     prm.mant_bytes = (n + 15) & ~15ull;
     prm.fast_bits = fb;
