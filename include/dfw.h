@@ -45,7 +45,10 @@
  *     8..12) keyed by the next K stream bits at a codeword start: it lists up
  *     to four whole codewords inside those K bits (their symbols, how many,
  *     the bits they use and where each ends) or marks an escape when the
- *     first codeword is longer than K bits.  Then a hierarchy of 256-entry
+ *     first codeword is longer than K bits.  Its symbols are stored rotated
+ *     right by one bit, (e >> 1) | (e << 7) mod 256: bits 6..0 are then the
+ *     bf16 pattern's high byte below the sign and bit 7 the top bit of its low
+ *     byte, so the decoder assembles bf16 with byte masks alone.  Then a hierarchy of 256-entry
  *     tables keyed by successive bytes of the code: table 0 resolves every
  *     codeword of at most 8 bits and points to a subtable for longer ones (at
  *     most four levels for 32-bit codes); escapes are resolved through it.

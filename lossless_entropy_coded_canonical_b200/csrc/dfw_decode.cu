@@ -73,7 +73,7 @@ __device__ __forceinline__ uint32_t decode_window(const uint32_t (&wd)[NSEG + 1]
                 if (e.y & FAST_ESC) {
                     const uint32_t f = resolve_escape(x, g_hier, n_tables);
                     if (f & ESC_BAD) err |= ST_LUT;
-                    syms = f & 0xFFu;
+                    syms = rot_sym(f);
                     c8 = 8u;
                     pn = p + (int)((f >> LUT_LEN_SHIFT) & 63u);
                 } else {

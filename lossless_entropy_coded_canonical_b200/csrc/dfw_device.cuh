@@ -147,22 +147,29 @@ __device__ __noinline__ uint32_t resolve_escape(uint32_t x, const uint32_t *__re
     return ESC_BAD | (1u << LUT_LEN_SHIFT);  // length 1 keeps the walk finite
 }
 
-// Four (exponent, raw byte) pairs -> four bf16 patterns in two words.
-__device__ __forceinline__ void join4(uint32_t E, uint32_t M, uint32_t &w0, uint32_t &w1) {
-    const uint32_t hi = (M & 0x80808080u) | ((E >> 1) & 0x7F7F7F7Fu);  // sign | exp[7:1]
-    const uint32_t lo = ((E << 7) & 0x80808080u) | (M & 0x7F7F7F7Fu);  // exp[0] | mant
+// Exponent symbols are kept rotated right by one bit, r = (e >> 1) | (e << 7)
+// (mod 256): bits 6..0 of r are the bf16 pattern's high byte below the sign,
+// bit 7 of r is the top bit of its low byte.  The fast table stores its
+// symbols this way; a symbol from the byte-keyed hierarchy is rotated here.
+// Only the low byte of e is used (a hierarchy leaf carries its length above).
+__device__ __forceinline__ uint32_t rot_sym(uint32_t e) { return ((e & 0xFFu) >> 1) | ((e & 1u) << 7); }
+
+// Four (rotated exponent, raw byte) pairs -> four bf16 patterns in two words.
+__device__ __forceinline__ void join4(uint32_t R, uint32_t M, uint32_t &w0, uint32_t &w1) {
+    const uint32_t hi = (M & 0x80808080u) | (R & 0x7F7F7F7Fu);  // sign | exp[7:1]
+    const uint32_t lo = (R & 0x80808080u) | (M & 0x7F7F7F7Fu);  // exp[0] | mant
     w0 = __byte_perm(lo, hi, 0x5140);
     w1 = __byte_perm(lo, hi, 0x7362);
 }
 
-__device__ __forceinline__ uint16_t join1(uint32_t e, uint32_t m) {
-    return (uint16_t)(((m & 0x80u) << 8) | (e << 7) | (m & 0x7Fu));
+__device__ __forceinline__ uint16_t join1(uint32_t r, uint32_t m) {
+    return (uint16_t)((((m & 0x80u) | (r & 0x7Fu)) << 8) | (r & 0x80u) | (m & 0x7Fu));
 }
 
 // One distinct exponent: every weight is (sym, raw byte).
 __global__ void fill_single(const uint8_t *__restrict__ mant, uint32_t sym, uint64_t n,
                             uint16_t *__restrict__ out) {
-    const uint32_t E = sym * 0x01010101u;
+    const uint32_t E = rot_sym(sym) * 0x01010101u;
     const uint64_t nfull = n >> 3;
     for (uint64_t c = blockIdx.x * (uint64_t)blockDim.x + threadIdx.x; c < nfull;
          c += (uint64_t)gridDim.x * blockDim.x) {
@@ -174,7 +181,7 @@ __global__ void fill_single(const uint8_t *__restrict__ mant, uint32_t sym, uint
     }
     if (blockIdx.x == 0 && threadIdx.x < (n & 7)) {
         const uint64_t j = (nfull << 3) + threadIdx.x;
-        out[j] = join1(sym, mant[j]);
+        out[j] = join1(rot_sym(sym), mant[j]);
     }
 }
 

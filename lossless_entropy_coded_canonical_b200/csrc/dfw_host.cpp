@@ -343,7 +343,9 @@ static bool hier_decode(const std::vector<uint32_t> &lut, uint32_t x, int &sym, 
 }
 
 // Fast table: for every K-bit key, the whole codewords (at most four) that
-// start at the key's first bit and end within its K bits.
+// start at the key's first bit and end within its K bits.  Symbols are stored
+// rotated right by one bit, the order in which the bf16 pattern's two bytes
+// use the exponent's bits, so the device joins them with masks alone.
 dfw_status build_fast(const std::vector<uint32_t> &lut, int fast_bits, std::vector<uint32_t> &fast) {
     if (fast_bits < FAST_BITS_MIN || fast_bits > FAST_BITS_MAX) return DFW_EINVAL;
     const uint32_t entries = 1u << fast_bits;
@@ -356,7 +358,7 @@ dfw_status build_fast(const std::vector<uint32_t> &lut, int fast_bits, std::vect
             int sym = 0, len = 0;
             if (!hier_decode(lut, x << pos, sym, len)) break;
             if (pos + len > fast_bits) break;
-            syms |= (uint32_t)sym << (8 * cnt);
+            syms |= (((uint32_t)sym >> 1) | (((uint32_t)sym & 1u) << 7)) << (8 * cnt);  // rotated right by one
             pos += len;
             ends |= 1u << (pos - 1);
             ++cnt;

@@ -147,7 +147,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         } else {  // first codeword longer than the fast key
             const uint32_t f = resolve_escape(x, g_hier, n_tables);
             if (f & ESC_BAD) err |= ST_LUT;
-            syms = f & 0xFFu;
+            syms = rot_sym(f);
             c8 = 8u;
             cb = (f >> LUT_LEN_SHIFT) & 63u;  // <= 32: at most one word to shift in
         }

@@ -178,6 +178,11 @@ def _split_lut(pl):
     return img[: 2 * nf].reshape(nf, 2), img[2 * nf:]
 
 
+def _unrotate(r):
+    """A fast-table symbol r = (e >> 1) | (e << 7) mod 256 back to e."""
+    return ((r << 1) | (r >> 7)) & 0xFF
+
+
 def _fast_window_walk(fast, hier, K, stream_u8, total_bits, W):
     """Emulates the device's phase 1 on every window: fast lookups of K bits,
     escapes through the byte hierarchy, and the window-end rule (a lookup that
@@ -225,7 +230,8 @@ def _fast_window_walk(fast, hier, K, stream_u8, total_bits, W):
             if p + cb > wend:
                 r = wend - p
                 take = min(c, 1 + bin(ends & ((1 << (r - 1)) - 1)).count("1"))
-            syms += [(e0 >> (8 * i)) & 0xFF for i in range(take)]
+            # fast-table symbols are stored rotated right by one bit
+            syms += [_unrotate((e0 >> (8 * i)) & 0xFF) for i in range(take)]
             p += cb
         out.append(syms)
     return out
