@@ -271,6 +271,54 @@ dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, cons
                             const dfw_table *table, const dfw_lanes_info *info, uint16_t *d_out,
                             void *cuda_stream);
 
+/*
+ * ENCODING ON THE GPU (two calls; same stream bytes as dfw_encode, and the
+ * known-start plan's chunk_bits and group_start made on the way).  Source:
+ * DFloat11 abstract (frequency-based codes for the bf16 exponents); the
+ * LazyWeights write-up (Huffman; lanes with known starts).
+ *
+ * dfw_encode_device_scratch_bytes -- device scratch bytes the first call
+ * needs (a few KB, whatever n).
+ *
+ * dfw_encode_device -- first call: splits the n bf16 patterns into raw bytes
+ * and an exponent histogram on the GPU, builds the code on the host
+ * (package-merge, canonical; exactly as dfw_encode), then counts each
+ * chunk's bits and each group's start on the GPU.  Synchronises cuda_stream
+ * twice (to read the histogram and the totals).
+ *   d_bf16         device, n bf16 patterns (16-byte aligned)
+ *   cap            length cap, 1..32
+ *   d_mant         device, dfw_mant_bytes(n) bytes (output)
+ *   d_chunk_bits   device, 32 * n_groups u16 (output)
+ *   d_group_start  device, n_groups + 1 u64 (output)
+ *   d_scratch      device, scratch_bytes >= dfw_encode_device_scratch_bytes(n)
+ *   table          host, output: as dfw_encode (stream_bytes tells the caller
+ *                  how large a stream to allocate for dfw_pack_device)
+ *   info           host; in: fast_bits (0 = 12); out: as dfw_plan_lanes
+ * n_groups = ceil(ceil(n / 64) / 32).  Errors: DFW_EINVAL, DFW_EALIGN,
+ * DFW_ENOMEM (scratch too small), DFW_ECAP, DFW_ECUDA.
+ *
+ * dfw_pack_device -- second call: zeroes the stream and packs the codewords
+ * at the positions the first call counted.  Asynchronous on cuda_stream.
+ *   d_bf16, table, info, d_group_start   as returned by the first call
+ *   d_stream   device, stream_capacity >= table->stream_bytes (output)
+ * Errors: DFW_EINVAL, DFW_EALIGN, DFW_ENOMEM, DFW_ECUDA.
+ *
+ * dfw_lanes_lut -- the LUT image (host, info->lut_words u32) for a table and
+ * info->fast_bits, without walking a stream.  Errors: DFW_EINVAL.
+ */
+uint64_t dfw_encode_device_scratch_bytes(uint64_t n);
+
+dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
+                             uint16_t *d_chunk_bits, uint64_t *d_group_start, void *d_scratch,
+                             uint64_t scratch_bytes, dfw_table *table, dfw_lanes_info *info,
+                             void *cuda_stream);
+
+dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *table, const dfw_lanes_info *info,
+                           const uint64_t *d_group_start, uint8_t *d_stream, uint64_t stream_capacity,
+                           void *cuda_stream);
+
+dfw_status dfw_lanes_lut(const dfw_table *table, const dfw_lanes_info *info, uint32_t *lut);
+
 /* Static English text for a status code. */
 const char *dfw_strerror(dfw_status status);
 

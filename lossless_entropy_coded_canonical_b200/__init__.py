@@ -26,6 +26,7 @@ from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, 
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
            "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "LanesInfo",
+           "encode_device", "encode_device_scratch_bytes",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
            "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
 
@@ -272,6 +273,47 @@ def decode_lanes(dl: DeviceLanes, out: torch.Tensor | None = None, stream=None) 
                                   _ptr(dl.group_start), ctypes.byref(dl.table), ctypes.byref(dl.info), _ptr(out),
                                   _stream_handle(stream)), "dfw_decode_lanes")
     return out
+
+
+def encode_device(x: torch.Tensor, cap: int = 32, fast_bits: int = 0, stream=None,
+                  scratch: torch.Tensor | None = None) -> DeviceLanes:
+    """Encodes a bf16 tensor that is already on the GPU (``dfw_encode_device``
+    then ``dfw_pack_device``): the same stream bytes as :func:`encode`, the
+    known-start plan made on the way, and the LUT image built on the host and
+    uploaded.  Returns a :class:`DeviceLanes` ready for :func:`decode_lanes`.
+    ``scratch`` (uint8, at least ``encode_device_scratch_bytes()``) may be
+    passed to reuse one buffer across calls."""
+    if not x.is_cuda:
+        raise ValueError("encode_device takes a CUDA tensor")
+    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected bf16 bit patterns, got {x.dtype}")
+    x = x.contiguous().reshape(-1)
+    dev, n = x.device, x.numel()
+    n_groups = -(-(-(-n // 64)) // 32)
+    mant = torch.empty(mant_bytes(n), dtype=torch.uint8, device=dev)
+    chunk_bits = torch.empty(32 * n_groups, dtype=torch.int16, device=dev)
+    group_start = torch.empty(n_groups + 1, dtype=torch.int64, device=dev)
+    need = encode_device_scratch_bytes()
+    if scratch is None:
+        scratch = torch.empty(need, dtype=torch.uint8, device=dev)
+    if scratch.numel() * scratch.element_size() < need:
+        raise ValueError(f"scratch needs {need} bytes")
+    table, info = Table(), LanesInfo()
+    info.fast_bits = fast_bits
+    sh = _stream_handle(stream)
+    _check(lib().dfw_encode_device(_ptr(x), n, cap, _ptr(mant), _ptr(chunk_bits), _ptr(group_start),
+                                   _ptr(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(table),
+                                   ctypes.byref(info), sh), "dfw_encode_device")
+    stream_buf = torch.empty(int(table.stream_bytes), dtype=torch.uint8, device=dev)
+    _check(lib().dfw_pack_device(_ptr(x), ctypes.byref(table), ctypes.byref(info), _ptr(group_start),
+                                 _ptr(stream_buf), stream_buf.numel(), sh), "dfw_pack_device")
+    lut = torch.empty(int(info.lut_words), dtype=torch.int32)
+    _check(lib().dfw_lanes_lut(ctypes.byref(table), ctypes.byref(info), _ptr(lut.numpy())), "dfw_lanes_lut")
+    return DeviceLanes(stream_buf, mant, lut.to(dev), chunk_bits, group_start, table, info, None)
+
+
+def encode_device_scratch_bytes() -> int:
+    return int(lib().dfw_encode_device_scratch_bytes(0))
 
 
 def check(stream=None) -> None:

@@ -15,7 +15,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdfw.so")
-SOURCES = ["dfw_host.cpp", "dfw_decode.cu"]
+SOURCES = ["dfw_host.cpp", "dfw_decode.cu", "dfw_encode.cu"]
 HEADERS = ["dfw_internal.h", "dfw_device.cuh", "dfw_lanes.cuh", os.path.join("..", "..", "include", "dfw.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -1,0 +1,449 @@
+// dfw_encode.cu -- the encoder on the GPU.  Same output as the host encoder
+// (dfw_encode), byte for byte, plus the known-start plan's aux arrays, made
+// in the passes that need them anyway.
+//
+// Source: DFloat11 abstract (frequency-based variable-length codes for the
+// bf16 exponents; bit-exact), the LazyWeights write-up (Huffman; lanes that
+// start at known bits).  The passes:
+//   1  split + histogram   each thread reads 8 bf16 (16 bytes), writes their 8
+//                          raw bytes, and counts their exponents in its
+//                          warp's shared histogram (4 copies, lanes spread
+//                          over them to thin out same-bin atomics)
+//   -  code (host)         package-merge lengths and canonical codes from the
+//                          histogram, exactly as the host encoder does
+//   2  chunk bits          one warp per group of 32 chunks x 64 codewords:
+//                          coalesced loads (lane l holds 8 consecutive
+//                          weights), code lengths from a shared table, a
+//                          3-step shuffle sum per chunk -> chunk_bits[]; the
+//                          group total goes to group_start[g]
+//   3  group starts        one CTA turns the group totals into exclusive
+//                          prefix sums in place (group_start[]), the total
+//                          bit count and the largest group span
+//   4  pack                one warp per group: each lane packs its 8
+//                          codewords at their bit offset (warp prefix sum)
+//                          into the warp's shared word buffer (shared atomic
+//                          OR: neighbours share a word); the warp then writes
+//                          the group's words, big-endian, with plain stores
+//                          inside and atomic ORs on the two words it may
+//                          share with the neighbouring groups (the stream is
+//                          zeroed first)
+// Nothing waits on another CTA; every loop is bounded by n.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "dfw_internal.h"
+
+namespace dfw {
+namespace {
+
+constexpr int SPLIT_NT = 256;     // threads per CTA of pass 1
+constexpr int HIST_COPIES = 4;    // histogram copies per warp
+constexpr int GROUP_NT = 512;     // threads per CTA of passes 2 and 4
+constexpr int SCAN_NT = 1024;     // threads of the pass-3 CTA
+constexpr uint32_t GROUP_W = LANE_SYMS * GROUP_CHUNKS;  // weights per group (2048)
+
+// Layout of the caller's scratch buffer.
+struct EncScratch {
+    unsigned long long hist[256];
+    unsigned long long total_bits;
+    unsigned int max_span;  // largest group span in bytes (as the lanes plan counts it)
+    unsigned int max_group_bits;
+};
+
+struct LenTable {
+    uint8_t len[256];
+};
+struct CodeTable {
+    unsigned long long lc[256];  // (length << 32) | canonical code
+};
+
+__device__ __forceinline__ uint32_t span_bytes_dev(uint64_t start_bit, uint64_t end_bit) {
+    const uint64_t b0 = (start_bit >> 3) & ~15ull;
+    const uint64_t b1 = (((end_bit + 7) >> 3) + 8 + 15) & ~15ull;
+    return (uint32_t)(b1 - b0);
+}
+
+__device__ __forceinline__ uint32_t bswap32_dev(uint32_t x) { return __byte_perm(x, 0, 0x0123); }
+
+// ------------------------------------------------------------ pass 1
+
+// Raw bytes of four bf16 patterns held in two words: (hi byte & 0x80) |
+// (lo byte & 0x7F) per pattern.  Exponents: (hi byte << 1) | (lo byte >> 7).
+__device__ __forceinline__ void split4(uint32_t x0, uint32_t x1, uint32_t &m4, uint32_t &e4) {
+    const uint32_t lo = __byte_perm(x0, x1, 0x6420), hi = __byte_perm(x0, x1, 0x7531);
+    m4 = (hi & 0x80808080u) | (lo & 0x7F7F7F7Fu);
+    e4 = ((hi << 1) & 0xFEFEFEFEu) | ((lo >> 7) & 0x01010101u);
+}
+
+__global__ void __launch_bounds__(SPLIT_NT) enc_split_hist(const uint16_t *__restrict__ in, uint64_t n,
+                                                            uint8_t *__restrict__ mant, uint64_t mant_bytes,
+                                                            unsigned long long *__restrict__ hist) {
+    __shared__ uint32_t h[SPLIT_NT / 32][256 * HIST_COPIES];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < (SPLIT_NT / 32) * 256 * HIST_COPIES; i += SPLIT_NT) (&h[0][0])[i] = 0u;
+    __syncthreads();
+    uint32_t *hw = h[warp] + (lane & (HIST_COPIES - 1));
+    const uint64_t n8 = n >> 3;
+    const uint64_t stride = (uint64_t)gridDim.x * SPLIT_NT;
+    for (uint64_t i = (uint64_t)blockIdx.x * SPLIT_NT + tid; i < n8; i += stride) {
+        const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(in) + i);
+        uint32_t m0, e0, m1, e1;
+        split4(v.x, v.y, m0, e0);
+        split4(v.z, v.w, m1, e1);
+        __stcs(reinterpret_cast<uint2 *>(mant) + i, make_uint2(m0, m1));
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            atomicAdd(hw + HIST_COPIES * ((e0 >> (8 * k)) & 0xFFu), 1u);
+            atomicAdd(hw + HIST_COPIES * ((e1 >> (8 * k)) & 0xFFu), 1u);
+        }
+    }
+    if (blockIdx.x == 0) {  // the < 8 trailing weights and the zero padding of the raw bytes
+        for (uint64_t j = (n8 << 3) + tid; j < mant_bytes; j += SPLIT_NT) {
+            uint8_t m = 0;
+            if (j < n) {
+                const uint32_t u = in[j];
+                m = (uint8_t)(((u >> 8) & 0x80u) | (u & 0x7Fu));
+                atomicAdd(hw + HIST_COPIES * ((u >> 7) & 0xFFu), 1u);
+            }
+            mant[j] = m;
+        }
+    }
+    __syncthreads();
+    for (int b = tid; b < 256; b += SPLIT_NT) {
+        unsigned long long s = 0;
+        for (int w = 0; w < SPLIT_NT / 32; ++w)
+            for (int c = 0; c < HIST_COPIES; ++c) s += h[w][HIST_COPIES * b + c];
+        if (s) atomicAdd(hist + b, s);
+    }
+}
+
+// ------------------------------------------------------------ pass 2
+
+constexpr unsigned FULL = 0xFFFFFFFFu;
+
+// Exponents of the 8 bf16 patterns in v, as two words of 4 bytes.
+__device__ __forceinline__ void exps8(const uint4 v, uint32_t &e0, uint32_t &e1) {
+    uint32_t m;
+    split4(v.x, v.y, m, e0);
+    split4(v.z, v.w, m, e1);
+}
+
+// The 8 weights of lane `lane` in step j of a group: weights 8 (32 j + lane)
+// .. + 7 of the group, i.e. of chunk 4 j + lane / 8.  Fills the exponents
+// (0 past n) and returns how many of the 8 exist.
+__device__ __forceinline__ uint32_t load8(const uint16_t *__restrict__ in, uint64_t n, uint64_t e0, uint32_t &x0,
+                                          uint32_t &x1) {
+    if (e0 + 8 <= n) {
+        exps8(__ldcs(reinterpret_cast<const uint4 *>(in + e0)), x0, x1);
+        return 8u;
+    }
+    x0 = x1 = 0u;
+    uint32_t c = 0;
+    for (uint64_t k = e0; k < n; ++k, ++c) {  // the tensor's last, partial step
+        const uint32_t e = (in[k] >> 7) & 0xFFu;
+        if (c < 4) x0 |= e << (8 * c);
+        else x1 |= e << (8 * (c - 4));
+    }
+    return c;
+}
+
+__global__ void __launch_bounds__(GROUP_NT) enc_chunk_bits(const uint16_t *__restrict__ in, uint64_t n,
+                                                            const LenTable lt, uint16_t *__restrict__ chunk_bits,
+                                                            uint64_t *__restrict__ group_start, uint32_t n_groups) {
+    __shared__ uint32_t s_len[256];
+    for (int i = threadIdx.x; i < 256; i += GROUP_NT) s_len[i] = lt.len[i];
+    __syncthreads();
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t wstride = gridDim.x * (GROUP_NT / 32);
+    for (uint32_t g = blockIdx.x * (GROUP_NT / 32) + (threadIdx.x >> 5); g < n_groups; g += wstride) {
+        const uint64_t base = (uint64_t)g * GROUP_W;
+        uint32_t mine = 0;
+#pragma unroll 2
+        for (uint32_t j = 0; j < 8; ++j) {
+            uint32_t x0, x1;
+            const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+            uint32_t b = 0;
+            for (uint32_t k = 0; k < 4; ++k) b += k < cnt ? s_len[(x0 >> (8 * k)) & 0xFFu] : 0u;
+            for (uint32_t k = 4; k < 8; ++k) b += k < cnt ? s_len[(x1 >> (8 * (k - 4))) & 0xFFu] : 0u;
+            // lanes 8q .. 8q + 7 hold chunk 4 j + q: sum them
+            b += __shfl_xor_sync(FULL, b, 1);
+            b += __shfl_xor_sync(FULL, b, 2);
+            b += __shfl_xor_sync(FULL, b, 4);
+            const uint32_t from = __shfl_sync(FULL, b, 8u * (lane & 3u));
+            if ((lane >> 2) == j) mine = from;  // lane l keeps chunk l
+        }
+        chunk_bits[(uint64_t)g * GROUP_CHUNKS + lane] = (uint16_t)mine;
+        uint32_t tot = mine;
+        for (int d = 16; d > 0; d >>= 1) tot += __shfl_xor_sync(FULL, tot, d);
+        if (lane == 0) group_start[g] = tot;  // the group's total until pass 3
+    }
+}
+
+// ------------------------------------------------------------ pass 3
+
+__global__ void __launch_bounds__(SCAN_NT) enc_group_scan(uint64_t *__restrict__ gs, uint32_t n_groups,
+                                                          EncScratch *__restrict__ res) {
+    __shared__ unsigned long long s_part[SCAN_NT];
+    const uint32_t tid = threadIdx.x;
+    const uint32_t per = (n_groups + SCAN_NT - 1) / SCAN_NT;
+    const uint32_t lo = min(n_groups, tid * per), hi = min(n_groups, lo + per);
+    unsigned long long s = 0;
+    uint32_t mb = 0;
+    for (uint32_t i = lo; i < hi; ++i) {
+        const uint64_t v = gs[i];
+        s += v;
+        mb = max(mb, (uint32_t)v);
+    }
+    s_part[tid] = s;
+    __syncthreads();
+    for (uint32_t d = 1; d < SCAN_NT; d <<= 1) {  // inclusive scan of the thread sums
+        const unsigned long long v = tid >= d ? s_part[tid - d] : 0ull;
+        __syncthreads();
+        s_part[tid] += v;
+        __syncthreads();
+    }
+    unsigned long long run = s_part[tid] - s;
+    uint32_t ms = 16;
+    for (uint32_t i = lo; i < hi; ++i) {
+        const uint64_t v = gs[i];
+        gs[i] = run;
+        ms = max(ms, span_bytes_dev(run, run + v));
+        run += v;
+    }
+    if (tid == SCAN_NT - 1) {
+        gs[n_groups] = run;
+        res->total_bits = run;
+    }
+    atomicMax(&res->max_span, ms);
+    atomicMax(&res->max_group_bits, mb);
+}
+
+// ------------------------------------------------------------ pass 4
+
+__global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict__ in, uint64_t n, const CodeTable ct,
+                                                      const uint64_t *__restrict__ group_start, uint32_t n_groups,
+                                                      uint32_t *__restrict__ stream_words, uint32_t buf_words) {
+    extern __shared__ __align__(16) uint32_t s_dyn[];
+    unsigned long long *s_lc = reinterpret_cast<unsigned long long *>(s_dyn);
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+    uint32_t *buf = s_dyn + 512 + warp * buf_words;
+    for (int i = threadIdx.x; i < 256; i += GROUP_NT) s_lc[i] = ct.lc[i];
+    for (uint32_t i = lane; i < buf_words; i += 32) buf[i] = 0u;
+    __syncthreads();
+    const uint32_t wstride = gridDim.x * (GROUP_NT / 32);
+    for (uint32_t g = blockIdx.x * (GROUP_NT / 32) + warp; g < n_groups; g += wstride) {
+        const uint64_t gs0 = group_start[g], gs1 = group_start[g + 1];
+        if (gs1 <= gs0) continue;  // warp-uniform
+        const uint64_t base = (uint64_t)g * GROUP_W;
+        const uint32_t sh0 = (uint32_t)(gs0 & 31u);
+        uint32_t carry = sh0;
+        for (uint32_t j = 0; j < 8; ++j) {
+            uint32_t x0, x1;
+            const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+            unsigned long long lc[8];
+            uint32_t b = 0;
+#pragma unroll
+            for (uint32_t k = 0; k < 8; ++k) {
+                const uint32_t e = ((k < 4 ? x0 : x1) >> (8 * (k & 3))) & 0xFFu;
+                lc[k] = k < cnt ? s_lc[e] : 0ull;
+                b += (uint32_t)(lc[k] >> 32);
+            }
+            uint32_t incl = b;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(FULL, incl, d);
+                if (lane >= (uint32_t)d) incl += y;
+            }
+            const uint32_t off = carry + incl - b;  // bit offset in the warp's buffer
+            carry += __shfl_sync(FULL, incl, 31);
+            if (b) {
+                unsigned long long acc = 0;
+                uint32_t nacc = off & 31u, wi = off >> 5;
+#pragma unroll
+                for (uint32_t k = 0; k < 8; ++k) {
+                    const uint32_t L = (uint32_t)(lc[k] >> 32);
+                    if (!L) continue;
+                    acc = (acc << L) | (uint32_t)lc[k];
+                    nacc += L;
+                    if (nacc >= 32u) {
+                        atomicOr(buf + wi, (uint32_t)(acc >> (nacc - 32u)));
+                        ++wi;
+                        nacc -= 32u;
+                    }
+                }
+                if (nacc) atomicOr(buf + wi, (uint32_t)(acc << (32u - nacc)));
+            }
+        }
+        __syncwarp();
+        const uint32_t nw = (uint32_t)((sh0 + (gs1 - gs0) + 31u) >> 5);
+        uint32_t *dst = stream_words + (gs0 >> 5);
+        for (uint32_t i = lane; i < nw; i += 32) {
+            const uint32_t v = bswap32_dev(buf[i]);
+            buf[i] = 0u;
+            if (i == 0 || i + 1 == nw) atomicOr(dst + i, v);  // may be shared with a neighbouring group
+            else dst[i] = v;
+        }
+        __syncwarp();
+    }
+}
+
+}  // namespace
+}  // namespace dfw
+
+// ------------------------------------------------------------ host side
+
+namespace {
+
+using namespace dfw;
+
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
+}
+
+bool misaligned(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+}  // namespace
+
+extern "C" uint64_t dfw_encode_device_scratch_bytes(uint64_t n) {
+    (void)n;
+    return (sizeof(EncScratch) + 255) & ~(uint64_t)255;
+}
+
+extern "C" dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
+                                        uint16_t *d_chunk_bits, uint64_t *d_group_start, void *d_scratch,
+                                        uint64_t scratch_bytes, dfw_table *table, dfw_lanes_info *info,
+                                        void *cuda_stream) {
+    if (!table || !info || cap < 1 || cap > DFW_MAX_CAP) return DFW_EINVAL;
+    const uint32_t fb = info->fast_bits;
+    std::memset(table, 0, sizeof(*table));
+    table->version = DFW_FORMAT_VERSION;
+    table->cap = (uint32_t)cap;
+    table->n = n;
+    table->stream_bytes = stream_bytes_for(0);
+    const uint64_t n_chunks = (n + LANE_SYMS - 1) / LANE_SYMS;
+    const uint64_t n_groups = (n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+    if (n_chunks >= (1ull << 32)) return DFW_EINVAL;
+    if (n == 0) {
+        dfw_lanes_info q;
+        std::memset(&q, 0, sizeof(q));
+        q.fast_bits = fb;
+        const dfw_status st = dfw_plan_lanes_query(table, &q);
+        if (st != DFW_OK) return st;
+        q.max_group_bytes = 16;
+        *info = q;
+        if (d_group_start && cudaMemsetAsync(d_group_start, 0, sizeof(uint64_t), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
+            return DFW_ECUDA;
+        return DFW_OK;
+    }
+    if (!d_bf16 || !d_mant || !d_chunk_bits || !d_group_start || !d_scratch) return DFW_EINVAL;
+    if (misaligned(d_bf16) || misaligned(d_mant) || misaligned(d_chunk_bits) || misaligned(d_group_start) ||
+        misaligned(d_scratch))
+        return DFW_EALIGN;
+    if (scratch_bytes < sizeof(EncScratch)) return DFW_ENOMEM;
+    const int sms = device_sms();
+    if (sms <= 0) return DFW_ECUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    EncScratch *sc = static_cast<EncScratch *>(d_scratch);
+
+    // pass 1: raw bytes and the exponent histogram
+    if (cudaMemsetAsync(sc, 0, sizeof(EncScratch), s) != cudaSuccess) return DFW_ECUDA;
+    {
+        const uint64_t want = ((n >> 3) + SPLIT_NT - 1) / SPLIT_NT, cap_blocks = (uint64_t)sms * 8;
+        const unsigned blocks = (unsigned)std::max<uint64_t>(1, std::min(want, cap_blocks));
+        enc_split_hist<<<blocks, SPLIT_NT, 0, s>>>(d_bf16, n, d_mant, dfw_mant_bytes(n), sc->hist);
+        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    }
+    uint64_t hist[256];
+    if (cudaMemcpyAsync(hist, sc->hist, sizeof(hist), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return DFW_ECUDA;
+
+    // the code, on the host, exactly as the host encoder builds it
+    uint64_t sum = 0;
+    int k = 0, only = 0;
+    for (int b = 0; b < 256; ++b) {
+        sum += hist[b];
+        if (hist[b]) {
+            ++k;
+            only = b;
+        }
+    }
+    if (sum != n) return DFW_ECUDA;  // the histogram pass did not complete
+    table->n_symbols = (uint32_t)k;
+    table->single_symbol = k == 1 ? (uint32_t)only : 0u;
+    dfw_status st = code_lengths(hist, cap, table->len);
+    if (st != DFW_OK) return st;
+
+    // passes 2 and 3: chunk bits, group totals -> group starts
+    LenTable lt;
+    std::memcpy(lt.len, table->len, 256);
+    {
+        const uint64_t want = (n_groups + GROUP_NT / 32 - 1) / (GROUP_NT / 32), cap_blocks = (uint64_t)sms * 4;
+        enc_chunk_bits<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, 0, s>>>(d_bf16, n, lt, d_chunk_bits,
+                                                                                 d_group_start, (uint32_t)n_groups);
+        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+        enc_group_scan<<<1, SCAN_NT, 0, s>>>(d_group_start, (uint32_t)n_groups, sc);
+        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    }
+    unsigned long long res[2];  // total_bits, (max_group_bits << 32) | max_span
+    if (cudaMemcpyAsync(res, &sc->total_bits, sizeof(res), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return DFW_ECUDA;
+    uint64_t expect = 0;
+    for (int b = 0; b < 256; ++b) expect += hist[b] * table->len[b];
+    if (res[0] != expect) return DFW_ECUDA;  // the counting passes disagree with the histogram
+    table->total_bits = res[0];
+    table->stream_bytes = stream_bytes_for(res[0]);
+
+    dfw_lanes_info q;
+    std::memset(&q, 0, sizeof(q));
+    q.fast_bits = fb;
+    st = dfw_plan_lanes_query(table, &q);
+    if (st != DFW_OK) return st;
+    q.max_group_bytes = std::max<uint32_t>(16u, (uint32_t)(res[1] & 0xFFFFFFFFull));
+    *info = q;
+    return DFW_OK;
+}
+
+extern "C" dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *table, const dfw_lanes_info *info,
+                                      const uint64_t *d_group_start, uint8_t *d_stream, uint64_t stream_capacity,
+                                      void *cuda_stream) {
+    dfw_status st = validate_table(table);
+    if (st != DFW_OK) return st;
+    if (!info || !d_stream) return DFW_EINVAL;
+    if (stream_capacity < table->stream_bytes) return DFW_ENOMEM;
+    const uint64_t n = table->n;
+    const uint64_t n_chunks = (n + LANE_SYMS - 1) / LANE_SYMS;
+    const uint64_t n_groups = (n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+    if (info->n_groups != n_groups || info->max_group_bytes < 16 || info->max_group_bytes > 64u * 1024u)
+        return DFW_EINVAL;
+    if (misaligned(d_stream) || (n && (misaligned(d_bf16) || misaligned(d_group_start)))) return DFW_EALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (cudaMemsetAsync(d_stream, 0, table->stream_bytes, s) != cudaSuccess) return DFW_ECUDA;
+    if (table->total_bits == 0) return DFW_OK;  // zero or one distinct exponent: no bits
+    if (!d_bf16 || !d_group_start) return DFW_EINVAL;
+    const int sms = device_sms();
+    if (sms <= 0) return DFW_ECUDA;
+    uint32_t code[256];
+    canonical_codes(table->len, code);
+    CodeTable ct;
+    for (int b = 0; b < 256; ++b) ct.lc[b] = ((unsigned long long)table->len[b] << 32) | code[b];
+    const uint32_t buf_words = info->max_group_bytes / 4 + 2;
+    const size_t smem = 2048 + (size_t)(GROUP_NT / 32) * buf_words * 4;
+    if (smem > 227u * 1024u) return DFW_EINVAL;
+    if (cudaFuncSetAttribute(enc_pack, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+        return DFW_ECUDA;
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, enc_pack, GROUP_NT, smem) != cudaSuccess) return DFW_ECUDA;
+    const uint64_t want = (n_groups + GROUP_NT / 32 - 1) / (GROUP_NT / 32);
+    const uint64_t cap_blocks = (uint64_t)sms * (uint64_t)std::max(1, per_sm);
+    enc_pack<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, smem, s>>>(
+        d_bf16, n, ct, d_group_start, (uint32_t)n_groups, reinterpret_cast<uint32_t *>(d_stream), buf_words);
+    return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+}

@@ -662,3 +662,21 @@ extern "C" const char *dfw_strerror(dfw_status s) {
     }
     return "unknown status";
 }
+
+extern "C" dfw_status dfw_lanes_lut(const dfw_table *table, const dfw_lanes_info *info, uint32_t *lut) {
+    if (!info || !lut) return DFW_EINVAL;
+    dfw_lanes_info q;
+    std::memset(&q, 0, sizeof(q));
+    q.fast_bits = info->fast_bits;
+    dfw_status st = dfw_plan_lanes_query(table, &q);
+    if (st != DFW_OK) return st;
+    if (q.lut_words != info->lut_words || q.fast_bits != info->fast_bits) return DFW_EINVAL;
+    std::vector<uint32_t> img, fast;
+    st = build_lut(table, img);
+    if (st != DFW_OK) return st;
+    st = build_fast(img, (int)q.fast_bits, fast);
+    if (st != DFW_OK) return st;
+    std::memcpy(lut, fast.data(), fast.size() * sizeof(uint32_t));
+    std::memcpy(lut + fast.size(), img.data(), img.size() * sizeof(uint32_t));
+    return DFW_OK;
+}
