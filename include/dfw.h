@@ -319,6 +319,32 @@ dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *table, const
 
 dfw_status dfw_lanes_lut(const dfw_table *table, const dfw_lanes_info *info, uint32_t *lut);
 
+/*
+ * dfw_encode_device_noalloc -- dfw_encode_device without a scratch argument,
+ * for callers that cannot allocate device memory when they encode: a serving
+ * runtime that reserves all of the GPU's memory at start-up and allows no
+ * allocation afterwards, or code that must not call cudaMalloc because the
+ * call would synchronise the device or re-enter the caller's own allocator.
+ * The pages describe no such call; it exists for those callers only.
+ *
+ * The scratch is an array of DFW_NOALLOC_SCRATCH_BYTES compiled into the
+ * library: every GPU that loads the library holds one until the process
+ * exits.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture begins.  All calls share the array and clear it before use,
+ * so calls whose GPU work overlaps (two streams, two host threads) race on it:
+ * the caller must not overlap them.  Arguments, outputs, synchronisation and
+ * errors as dfw_encode_device; DFW_ENOMEM if the scratch that n needs
+ * exceeded DFW_NOALLOC_SCRATCH_BYTES (the need is a fixed 2,304 bytes, so no
+ * n reaches it today).  The call makes no cudaMalloc, cudaFree or other
+ * device allocation; the inputs and outputs are the caller's.
+ */
+#define DFW_NOALLOC_SCRATCH_BYTES 4096
+
+dfw_status dfw_encode_device_noalloc(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
+                                     uint16_t *d_chunk_bits, uint64_t *d_group_start, dfw_table *table,
+                                     dfw_lanes_info *info, void *cuda_stream);
+
 /* Static English text for a status code. */
 const char *dfw_strerror(dfw_status status);
 

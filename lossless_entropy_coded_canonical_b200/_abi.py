@@ -60,6 +60,7 @@ SIGNATURES = {
     "dfw_encode_device": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _vp, _u64, _TP, _LP, _vp]),
     "dfw_pack_device": (_i, [_vp, _TP, _LP, _vp, _vp, _u64, _vp]),
     "dfw_lanes_lut": (_i, [_TP, _LP, _vp]),
+    "dfw_encode_device_noalloc": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _TP, _LP, _vp]),
     "dfw_check": (_i, [_vp]),
     "dfw_strerror": (ctypes.c_char_p, [_i]),
 }

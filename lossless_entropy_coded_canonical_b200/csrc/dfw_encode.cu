@@ -32,6 +32,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "dfw_internal.h"
 
@@ -446,4 +447,48 @@ extern "C" dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *t
     enc_pack<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, smem, s>>>(
         d_bf16, n, ct, d_group_start, (uint32_t)n_groups, reinterpret_cast<uint32_t *>(d_stream), buf_words);
     return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+}
+
+// ------------------------------------------------------------ no-allocation variant
+//
+// For callers that cannot allocate device memory where they encode: the
+// scratch of the first call lives in an array compiled into the library
+// instead of a caller buffer.  One array per device that loads the library,
+// held until the process exits; every call shares it (dfw_encode_device
+// clears it first), so calls whose GPU work overlaps race on it.
+
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DFW_NOALLOC_SCRATCH_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {nullptr};
+std::mutex g_noalloc_mu;
+
+// The array's device address on the current device; looked up (and cached)
+// on the first call there.
+dfw_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return DFW_ECUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return DFW_ECUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return DFW_OK;
+}
+
+}  // namespace
+
+extern "C" dfw_status dfw_encode_device_noalloc(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
+                                                uint16_t *d_chunk_bits, uint64_t *d_group_start, dfw_table *table,
+                                                dfw_lanes_info *info, void *cuda_stream) {
+    if (dfw_encode_device_scratch_bytes(n) > DFW_NOALLOC_SCRATCH_BYTES) return DFW_ENOMEM;
+    void *scratch = nullptr;
+    const dfw_status st = noalloc_scratch(&scratch);
+    if (st != DFW_OK) return st;
+    return dfw_encode_device(d_bf16, n, cap, d_mant, d_chunk_bits, d_group_start, scratch,
+                             DFW_NOALLOC_SCRATCH_BYTES, table, info, cuda_stream);
 }
