@@ -335,11 +335,11 @@ dfw_status dfw_lanes_lut(const dfw_table *table, const dfw_lanes_info *info, uin
  * so calls whose GPU work overlaps (two streams, two host threads) race on it:
  * the caller must not overlap them.  Arguments, outputs, synchronisation and
  * errors as dfw_encode_device; DFW_ENOMEM if the scratch that n needs
- * exceeded DFW_NOALLOC_SCRATCH_BYTES (the need is a fixed 2,304 bytes, so no
+ * exceeded DFW_NOALLOC_SCRATCH_BYTES (the need is a fixed 10,496 bytes, so no
  * n reaches it today).  The call makes no cudaMalloc, cudaFree or other
  * device allocation; the inputs and outputs are the caller's.
  */
-#define DFW_NOALLOC_SCRATCH_BYTES 4096
+#define DFW_NOALLOC_SCRATCH_BYTES 16384
 
 dfw_status dfw_encode_device_noalloc(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
                                      uint16_t *d_chunk_bits, uint64_t *d_group_start, dfw_table *table,

@@ -16,9 +16,12 @@
 //                          weights), code lengths from a shared table, a
 //                          3-step shuffle sum per chunk -> chunk_bits[]; the
 //                          group total goes to group_start[g]
-//   3  group starts        one CTA turns the group totals into exclusive
-//                          prefix sums in place (group_start[]), the total
-//                          bit count and the largest group span
+//   3  group starts        CTAs over contiguous ranges of groups: one
+//                          kernel sums each range, a second adds the earlier
+//                          ranges' sums and turns the group totals into
+//                          exclusive prefix sums in place (group_start[]);
+//                          the last range writes the total bit count; all
+//                          record the largest group span
 //   4  pack                one warp per group: each lane packs its 8
 //                          codewords at their bit offset (warp prefix sum)
 //                          into the warp's shared word buffer (shared atomic
@@ -42,15 +45,17 @@ namespace {
 constexpr int SPLIT_NT = 256;     // threads per CTA of pass 1
 constexpr int HIST_COPIES = 4;    // histogram copies per warp
 constexpr int GROUP_NT = 512;     // threads per CTA of passes 2 and 4
-constexpr int SCAN_NT = 1024;     // threads of the pass-3 CTA
+constexpr int SCAN_NT = 256;      // threads per CTA of pass 3
 constexpr uint32_t GROUP_W = LANE_SYMS * GROUP_CHUNKS;  // weights per group (2048)
 
 // Layout of the caller's scratch buffer.
+constexpr uint32_t SCAN_CTAS = 1024;  // most CTAs of the group-start passes
 struct EncScratch {
     unsigned long long hist[256];
     unsigned long long total_bits;
     unsigned int max_span;  // largest group span in bytes (as the lanes plan counts it)
     unsigned int max_group_bits;
+    unsigned long long range_total[SCAN_CTAS];  // pass 3a: bits of each CTA's range of groups
 };
 
 struct LenTable {
@@ -160,11 +165,19 @@ __global__ void __launch_bounds__(GROUP_NT) enc_chunk_bits(const uint16_t *__res
     const uint32_t wstride = gridDim.x * (GROUP_NT / 32);
     for (uint32_t g = blockIdx.x * (GROUP_NT / 32) + (threadIdx.x >> 5); g < n_groups; g += wstride) {
         const uint64_t base = (uint64_t)g * GROUP_W;
+        const bool whole = base + GROUP_W <= n;
+        uint4 raw[8];  // all eight loads in flight before any is used
+        if (whole) {
+#pragma unroll
+            for (uint32_t j = 0; j < 8; ++j)
+                raw[j] = __ldcs(reinterpret_cast<const uint4 *>(in + base + 8u * (32u * j + lane)));
+        }
         uint32_t mine = 0;
-#pragma unroll 2
+#pragma unroll
         for (uint32_t j = 0; j < 8; ++j) {
-            uint32_t x0, x1;
-            const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+            uint32_t x0, x1, cnt = 8u;
+            if (whole) exps8(raw[j], x0, x1);
+            else cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
             uint32_t b = 0;
             for (uint32_t k = 0; k < 4; ++k) b += k < cnt ? s_len[(x0 >> (8 * k)) & 0xFFu] : 0u;
             for (uint32_t k = 4; k < 8; ++k) b += k < cnt ? s_len[(x1 >> (8 * (k - 4))) & 0xFFu] : 0u;
@@ -184,41 +197,79 @@ __global__ void __launch_bounds__(GROUP_NT) enc_chunk_bits(const uint16_t *__res
 
 // ------------------------------------------------------------ pass 3
 
-__global__ void __launch_bounds__(SCAN_NT) enc_group_scan(uint64_t *__restrict__ gs, uint32_t n_groups,
-                                                          EncScratch *__restrict__ res) {
-    __shared__ unsigned long long s_part[SCAN_NT];
-    const uint32_t tid = threadIdx.x;
-    const uint32_t per = (n_groups + SCAN_NT - 1) / SCAN_NT;
-    const uint32_t lo = min(n_groups, tid * per), hi = min(n_groups, lo + per);
+// Block-wide inclusive scan of one value per thread (SCAN_NT threads);
+// returns the inclusive prefix and sets `total` for every thread.
+__device__ __forceinline__ unsigned long long block_scan(unsigned long long x, unsigned long long &total,
+                                                         unsigned long long *s_warp) {
+    const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+    unsigned long long incl = x;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const unsigned long long y = __shfl_up_sync(FULL, incl, d);
+        if (lane >= (uint32_t)d) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    unsigned long long before = 0;
+    total = 0;
+#pragma unroll
+    for (int w = 0; w < SCAN_NT / 32; ++w) {
+        const unsigned long long v = s_warp[w];
+        if (w < (int)warp) before += v;
+        total += v;
+    }
+    __syncthreads();  // s_warp may be reused
+    return before + incl;
+}
+
+// Pass 3a: CTA b sums the group totals of its range [b R, (b + 1) R).
+__global__ void __launch_bounds__(SCAN_NT) enc_range_totals(const uint64_t *__restrict__ gs, uint32_t n_groups,
+                                                            uint32_t range, EncScratch *__restrict__ res) {
+    __shared__ unsigned long long s_warp[SCAN_NT / 32];
+    const uint32_t lo = blockIdx.x * range, hi = min(n_groups, lo + range);
     unsigned long long s = 0;
     uint32_t mb = 0;
-    for (uint32_t i = lo; i < hi; ++i) {
+    for (uint32_t i = lo + threadIdx.x; i < hi; i += SCAN_NT) {
         const uint64_t v = gs[i];
         s += v;
         mb = max(mb, (uint32_t)v);
     }
-    s_part[tid] = s;
-    __syncthreads();
-    for (uint32_t d = 1; d < SCAN_NT; d <<= 1) {  // inclusive scan of the thread sums
-        const unsigned long long v = tid >= d ? s_part[tid - d] : 0ull;
-        __syncthreads();
-        s_part[tid] += v;
-        __syncthreads();
-    }
-    unsigned long long run = s_part[tid] - s;
+    unsigned long long total;
+    block_scan(s, total, s_warp);
+    if (threadIdx.x == 0) res->range_total[blockIdx.x] = total;
+    for (int d = 16; d > 0; d >>= 1) mb = max(mb, __shfl_xor_sync(FULL, mb, d));
+    if ((threadIdx.x & 31u) == 0) atomicMax(&res->max_group_bits, mb);
+}
+
+// Pass 3b: CTA b adds the totals of the ranges before its own, then turns
+// its range's group totals into exclusive prefix sums in place, a tile of
+// SCAN_NT at a time.  The last CTA writes group_start[n_groups] and the total.
+__global__ void __launch_bounds__(SCAN_NT) enc_range_scan(uint64_t *__restrict__ gs, uint32_t n_groups,
+                                                          uint32_t range, EncScratch *__restrict__ res) {
+    __shared__ unsigned long long s_warp[SCAN_NT / 32];
+    unsigned long long part = 0, carry;
+    for (uint32_t b = threadIdx.x; b < blockIdx.x; b += SCAN_NT) part += res->range_total[b];
+    block_scan(part, carry, s_warp);  // carry = bits of every earlier range
+    const uint32_t lo = blockIdx.x * range, hi = min(n_groups, lo + range);
     uint32_t ms = 16;
-    for (uint32_t i = lo; i < hi; ++i) {
-        const uint64_t v = gs[i];
-        gs[i] = run;
-        ms = max(ms, span_bytes_dev(run, run + v));
-        run += v;
+    for (uint32_t base = lo; base < hi; base += SCAN_NT) {
+        const uint32_t i = base + threadIdx.x;
+        const uint64_t v = i < hi ? gs[i] : 0ull;
+        unsigned long long tile;
+        const unsigned long long incl = block_scan(v, tile, s_warp);
+        if (i < hi) {
+            const unsigned long long start = carry + incl - v;
+            gs[i] = start;
+            ms = max(ms, span_bytes_dev(start, start + v));
+        }
+        carry += tile;
     }
-    if (tid == SCAN_NT - 1) {
-        gs[n_groups] = run;
-        res->total_bits = run;
+    if (blockIdx.x + 1 == gridDim.x && threadIdx.x == 0) {
+        gs[n_groups] = carry;
+        res->total_bits = carry;
     }
-    atomicMax(&res->max_span, ms);
-    atomicMax(&res->max_group_bits, mb);
+    for (int d = 16; d > 0; d >>= 1) ms = max(ms, __shfl_xor_sync(FULL, ms, d));
+    if ((threadIdx.x & 31u) == 0) atomicMax(&res->max_span, ms);
 }
 
 // ------------------------------------------------------------ pass 4
@@ -239,10 +290,19 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
         if (gs1 <= gs0) continue;  // warp-uniform
         const uint64_t base = (uint64_t)g * GROUP_W;
         const uint32_t sh0 = (uint32_t)(gs0 & 31u);
+        const bool whole = base + GROUP_W <= n;
+        uint4 raw[8];  // all eight loads in flight before any is used
+        if (whole) {
+#pragma unroll
+            for (uint32_t j = 0; j < 8; ++j)
+                raw[j] = __ldcs(reinterpret_cast<const uint4 *>(in + base + 8u * (32u * j + lane)));
+        }
         uint32_t carry = sh0;
+#pragma unroll
         for (uint32_t j = 0; j < 8; ++j) {
-            uint32_t x0, x1;
-            const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+            uint32_t x0, x1, cnt = 8u;
+            if (whole) exps8(raw[j], x0, x1);
+            else cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
             unsigned long long lc[8];
             uint32_t b = 0;
 #pragma unroll
@@ -259,7 +319,15 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
             }
             const uint32_t off = carry + incl - b;  // bit offset in the warp's buffer
             carry += __shfl_sync(FULL, incl, 31);
-            if (b) {
+            if (b && b <= 32u) {  // the common case: the 8 codewords fit one word, placed with <= 2 ORs
+                unsigned long long v = 0;
+#pragma unroll
+                for (uint32_t k = 0; k < 8; ++k) v = (v << (uint32_t)(lc[k] >> 32)) | (uint32_t)lc[k];
+                const uint32_t sh = off & 31u, wi = off >> 5;
+                const unsigned long long placed = v << (64u - sh - b);
+                atomicOr(buf + wi, (uint32_t)(placed >> 32));
+                if (sh + b > 32u) atomicOr(buf + wi + 1, (uint32_t)placed);
+            } else if (b) {
                 unsigned long long acc = 0;
                 uint32_t nacc = off & 31u, wi = off >> 5;
 #pragma unroll
@@ -389,7 +457,13 @@ extern "C" dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int 
         enc_chunk_bits<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, 0, s>>>(d_bf16, n, lt, d_chunk_bits,
                                                                                  d_group_start, (uint32_t)n_groups);
         if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
-        enc_group_scan<<<1, SCAN_NT, 0, s>>>(d_group_start, (uint32_t)n_groups, sc);
+        // pass 3: ranges of whole tiles, at most SCAN_CTAS of them
+        uint64_t range = (n_groups + SCAN_CTAS - 1) / SCAN_CTAS;
+        range = (range + SCAN_NT - 1) / SCAN_NT * SCAN_NT;
+        const unsigned ctas = (unsigned)((n_groups + range - 1) / range);
+        enc_range_totals<<<ctas, SCAN_NT, 0, s>>>(d_group_start, (uint32_t)n_groups, (uint32_t)range, sc);
+        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+        enc_range_scan<<<ctas, SCAN_NT, 0, s>>>(d_group_start, (uint32_t)n_groups, (uint32_t)range, sc);
         if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
     }
     unsigned long long res[2];  // total_bits, (max_group_bits << 32) | max_span
