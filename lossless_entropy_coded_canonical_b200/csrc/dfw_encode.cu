@@ -274,6 +274,14 @@ __global__ void __launch_bounds__(SCAN_NT) enc_range_scan(uint64_t *__restrict__
 
 // ------------------------------------------------------------ pass 4
 
+// x << s with PTX semantics: shifts of 32 or more give 0 (a 32-bit codeword
+// shifts an empty accumulator by 32).
+__device__ __forceinline__ uint32_t shl_clamp(uint32_t x, uint32_t s) {
+    uint32_t r;
+    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(s));
+    return r;
+}
+
 __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict__ in, uint64_t n, const CodeTable ct,
                                                       const uint64_t *__restrict__ group_start, uint32_t n_groups,
                                                       uint32_t *__restrict__ stream_words, uint32_t buf_words) {
@@ -290,19 +298,10 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
         if (gs1 <= gs0) continue;  // warp-uniform
         const uint64_t base = (uint64_t)g * GROUP_W;
         const uint32_t sh0 = (uint32_t)(gs0 & 31u);
-        const bool whole = base + GROUP_W <= n;
-        uint4 raw[8];  // all eight loads in flight before any is used
-        if (whole) {
-#pragma unroll
-            for (uint32_t j = 0; j < 8; ++j)
-                raw[j] = __ldcs(reinterpret_cast<const uint4 *>(in + base + 8u * (32u * j + lane)));
-        }
         uint32_t carry = sh0;
-#pragma unroll
         for (uint32_t j = 0; j < 8; ++j) {
-            uint32_t x0, x1, cnt = 8u;
-            if (whole) exps8(raw[j], x0, x1);
-            else cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+            uint32_t x0, x1;
+            const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
             unsigned long long lc[8];
             uint32_t b = 0;
 #pragma unroll
@@ -320,11 +319,11 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
             const uint32_t off = carry + incl - b;  // bit offset in the warp's buffer
             carry += __shfl_sync(FULL, incl, 31);
             if (b && b <= 32u) {  // the common case: the 8 codewords fit one word, placed with <= 2 ORs
-                unsigned long long v = 0;
+                uint32_t v = 0;
 #pragma unroll
-                for (uint32_t k = 0; k < 8; ++k) v = (v << (uint32_t)(lc[k] >> 32)) | (uint32_t)lc[k];
+                for (uint32_t k = 0; k < 8; ++k) v = shl_clamp(v, (uint32_t)(lc[k] >> 32)) | (uint32_t)lc[k];
                 const uint32_t sh = off & 31u, wi = off >> 5;
-                const unsigned long long placed = v << (64u - sh - b);
+                const unsigned long long placed = (unsigned long long)v << (64u - sh - b);
                 atomicOr(buf + wi, (uint32_t)(placed >> 32));
                 if (sh + b > 32u) atomicOr(buf + wi + 1, (uint32_t)placed);
             } else if (b) {
