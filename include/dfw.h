@@ -272,6 +272,43 @@ dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, cons
                             void *cuda_stream);
 
 /*
+ * dfw_decode_gemv_lanes -- decode fused with its consumer: y_i = W_i x_i for
+ * each of the k tensors of a scope (a transformer block's seven matrices, or
+ * one), without writing the decoded weights anywhere.  Source: Huff-LLM
+ * abstract (weights stay compressed up to the compute units) and the
+ * LazyWeights write-up (decoding on demand, invisible to the consumer);
+ * DFloat11 abstract point (iii) (per-block decompression).
+ *   d_stream .. info    the scope's known-start plan, as dfw_decode_lanes
+ *   k                   1..DFW_GEMV_MAX_TENSORS tensors
+ *   tensor_offsets      host, k + 1 entries: tensor i is weights
+ *                       [tensor_offsets[i], tensor_offsets[i+1]), first 0,
+ *                       last n (as dfw_encode_multi writes them)
+ *   cols                host, k entries: tensor i is a row-major matrix of
+ *                       (size / cols[i]) rows x cols[i] columns; cols[i] a
+ *                       multiple of 64 (so every 64-weight chunk lies in one
+ *                       row); each tensor below 2^32 weights
+ *   d_x                 host array of k device pointers: bf16 x_i, cols[i]
+ *                       entries, 32-byte aligned
+ *   d_y                 host array of k device pointers: fp32 y_i, one per row
+ *   d_partial           device scratch, partial_elems >= n / 64 fp32 (16-byte
+ *                       aligned): one partial dot product per chunk
+ * Arithmetic: bf16 x bf16 products are exact; they are summed in fp32 with
+ * fused multiply-adds, in an order fixed by the layout, so repeated calls
+ * give identical bits; |y - exact| <= gamma(cols) * sum |w x| with
+ * gamma(m) = m u / (1 - m u), u = 2^-24.  Asynchronous on cuda_stream (two
+ * launches).  Errors: DFW_EINVAL, DFW_EALIGN, DFW_ENOMEM (partial too
+ * small), DFW_ECUDA; corrupt plans through dfw_check (y then undefined).
+ */
+#define DFW_GEMV_MAX_TENSORS 8
+
+dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                                 const uint16_t *d_chunk_bits, const uint64_t *d_group_start,
+                                 const dfw_table *table, const dfw_lanes_info *info, int k,
+                                 const uint64_t *tensor_offsets, const uint32_t *cols,
+                                 const uint16_t *const *d_x, float *const *d_y, float *d_partial,
+                                 uint64_t partial_elems, void *cuda_stream);
+
+/*
  * ENCODING ON THE GPU (two calls; same stream bytes as dfw_encode, and the
  * known-start plan's chunk_bits and group_start made on the way).  Source:
  * DFloat11 abstract (frequency-based codes for the bf16 exponents); the

@@ -26,7 +26,7 @@ from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, 
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
            "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "LanesInfo",
-           "encode_device", "encode_device_scratch_bytes",
+           "encode_device", "encode_device_scratch_bytes", "decode_gemv_lanes",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
            "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
 
@@ -273,6 +273,36 @@ def decode_lanes(dl: DeviceLanes, out: torch.Tensor | None = None, stream=None) 
                                   _ptr(dl.group_start), ctypes.byref(dl.table), ctypes.byref(dl.info), _ptr(out),
                                   _stream_handle(stream)), "dfw_decode_lanes")
     return out
+
+
+def decode_gemv_lanes(dl: DeviceLanes, xs, cols, ys=None, partial: torch.Tensor | None = None,
+                      tensor_offsets=None, stream=None):
+    """y_i = W_i x_i for every tensor of a scope, decoded on the fly
+    (``dfw_decode_gemv_lanes``): the decoded weights are never written.
+    ``xs``: one bf16 CUDA vector per tensor (cols[i] entries); ``cols``:
+    columns per tensor (multiples of 64); returns fp32 ``ys`` (one per row)."""
+    offs = dl.tensor_offsets if tensor_offsets is None else tensor_offsets
+    if offs is None:
+        offs = np.array([0, dl.n], dtype=np.uint64)
+    offs = np.ascontiguousarray(np.asarray(offs, dtype=np.uint64))
+    k = offs.size - 1
+    cols = np.ascontiguousarray(np.asarray(cols, dtype=np.uint32))
+    if len(xs) != k or cols.size != k:
+        raise ValueError("one x and one column count per tensor")
+    dev = dl.mant.device
+    if ys is None:
+        ys = [torch.empty(int(offs[i + 1] - offs[i]) // int(cols[i]), dtype=torch.float32, device=dev)
+              for i in range(k)]
+    if partial is None:
+        partial = torch.empty(max(1, dl.n // 64), dtype=torch.float32, device=dev)
+    xs = [x.contiguous() for x in xs]
+    xp = (ctypes.c_void_p * k)(*[x.data_ptr() for x in xs])
+    yp = (ctypes.c_void_p * k)(*[y.data_ptr() for y in ys])
+    _check(lib().dfw_decode_gemv_lanes(_ptr(dl.stream), _ptr(dl.mant), _ptr(dl.lut), _ptr(dl.chunk_bits),
+                                       _ptr(dl.group_start), ctypes.byref(dl.table), ctypes.byref(dl.info), k,
+                                       _ptr(offs), _ptr(cols), xp, yp, _ptr(partial), partial.numel(),
+                                       _stream_handle(stream)), "dfw_decode_gemv_lanes")
+    return ys
 
 
 def encode_device(x: torch.Tensor, cap: int = 32, fast_bits: int = 0, stream=None,

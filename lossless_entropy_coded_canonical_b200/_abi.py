@@ -56,6 +56,7 @@ SIGNATURES = {
     "dfw_plan_lanes_query": (_i, [_TP, _LP]),
     "dfw_plan_lanes": (_i, [_vp, _TP, _vp, _vp, _vp, _LP]),
     "dfw_decode_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _vp, _vp]),
+    "dfw_decode_gemv_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _i, _vp, _vp, _vp, _vp, _vp, _u64, _vp]),
     "dfw_encode_device_scratch_bytes": (_u64, [_u64]),
     "dfw_encode_device": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _vp, _u64, _TP, _LP, _vp]),
     "dfw_pack_device": (_i, [_vp, _TP, _LP, _vp, _vp, _u64, _vp]),

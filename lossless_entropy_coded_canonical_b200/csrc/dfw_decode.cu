@@ -480,6 +480,23 @@ extern "C" dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d
     return launch_decode_lanes(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, d_out, s, sms);
 }
 
+extern "C" dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                                            const uint16_t *d_chunk_bits, const uint64_t *d_group_start,
+                                            const dfw_table *table, const dfw_lanes_info *info, int k,
+                                            const uint64_t *tensor_offsets, const uint32_t *cols,
+                                            const uint16_t *const *d_x, float *const *d_y, float *d_partial,
+                                            uint64_t partial_elems, void *cuda_stream) {
+    dfw_status st = validate_table(table);
+    if (st != DFW_OK) return st;
+    if (!info || table->n == 0) return DFW_EINVAL;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFW_ECUDA;
+    return launch_gemv_lanes(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, k, tensor_offsets,
+                             cols, d_x, d_y, d_partial, partial_elems, static_cast<cudaStream_t>(cuda_stream), sms);
+}
+
 extern "C" dfw_status dfw_check(void *cuda_stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return DFW_ECUDA;
     unsigned int v = 0, zero = 0;

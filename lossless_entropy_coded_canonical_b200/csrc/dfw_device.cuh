@@ -124,6 +124,26 @@ __device__ __forceinline__ void stg256_cs(void *p, uint4 a, uint4 b) {
                  : "memory");
 }
 
+// 32-byte read-only load (sm_100 256-bit vector load); 32-byte aligned address.
+__device__ __forceinline__ void ldg256_nc(const void *p, uint4 &a, uint4 &b) {
+    asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z), "=r"(b.w)
+                 : "l"(p));
+}
+
+// acc + w.lo * x.lo, then + w.hi * x.hi: two bf16 pairs, fp32 accumulation
+// (the product of two bf16 values is exact in the fused multiply-add).
+__device__ __forceinline__ float fma2_bf16(uint32_t w, uint32_t x, float acc) {
+    asm("{\n\t.reg .b16 wl, wh, xl, xh;\n\t"
+        "mov.b32 {wl, wh}, %1;\n\t"
+        "mov.b32 {xl, xh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, wl, xl, %0;\n\t"
+        "fma.rn.f32.bf16 %0, wh, xh, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w), "r"(x));
+    return acc;
+}
+
 // --------------------------------------------------------------- decoding
 
 // A codeword longer than the fast table's key: walk the byte-keyed hierarchy

@@ -38,6 +38,10 @@ constexpr uint32_t FAST_ESC_WORD = FAST_ESC | 255u;
 constexpr uint32_t LANE_SYMS = 64;
 constexpr uint32_t GROUP_CHUNKS = 32;
 
+// Tensors one fused decode + matrix-vector launch can serve (a transformer
+// block has seven).
+constexpr uint32_t GEMV_MAX_TENSORS = DFW_GEMV_MAX_TENSORS;
+
 // Bits of the device status word.
 constexpr uint32_t ST_COUNT = 1u;   // a tile decoded a different number of codes than out_start says
 constexpr uint32_t ST_LUT = 2u;     // a LUT pointer left the table or a code ran past four levels

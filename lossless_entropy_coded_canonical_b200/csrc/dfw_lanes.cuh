@@ -31,6 +31,8 @@
 // copies are bounded.
 #pragma once
 
+#include <cstring>
+
 #include "dfw_device.cuh"
 
 namespace dfw {
@@ -174,6 +176,97 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
     return 8u * (wa - sw) - 96u + p;
 }
 
+// What a lane does with its decoded chunk (64 rotated exponents in its word
+// slots at exps, exps + 128, ...; its 64 raw bytes at mrow): t weights of
+// chunk c, t < 64 only for the last chunk of the scope.
+
+// Decode: join into bf16 and store (piece q = 16 weights, in the order
+// (j + lane / 2) mod 4 so lanes spread over the banks).
+struct StoreEpi {
+    struct Params {};
+    __device__ static __forceinline__ void apply(const LanesParams &prm, const Params &, uint32_t lane, uint32_t c,
+                                                 uint32_t t, uint32_t mrow, uint32_t exps) {
+        uint16_t *dst = prm.out + (size_t)c * LANE_SYMS;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
+            const uint4 m = lds128(mrow + 16u * q);
+            const uint32_t e0 = lds32(exps + 512u * q), e1 = lds32(exps + 512u * q + 128u),
+                           e2 = lds32(exps + 512u * q + 256u), e3 = lds32(exps + 512u * q + 384u);
+            uint4 r0, r1;
+            join4(e0, m.x, r0.x, r0.y);
+            join4(e1, m.y, r0.z, r0.w);
+            join4(e2, m.z, r1.x, r1.y);
+            join4(e3, m.w, r1.z, r1.w);
+            if (16u * q + 16u <= t) {
+                if (prm.out32) {
+                    stg256_cs(dst + 16u * q, r0, r1);  // a whole sector per lane
+                } else {
+                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q), r0);
+                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q + 8u), r1);
+                }
+            } else {  // the last, partial chunk of the tensor: one weight at a time
+                for (uint32_t i = 16u * q; i < t; ++i) {
+                    const uint32_t e = (lds32(exps + 128u * (i >> 2)) >> (8u * (i & 3u))) & 0xFFu;
+                    const uint32_t mb = (lds32(mrow + (i & ~3u)) >> (8u * (i & 3u))) & 0xFFu;
+                    dst[i] = join1(e, mb);
+                }
+            }
+        }
+    }
+};
+
+// Decode fused with y = W x: the chunk's 64 weights never leave the SM.
+// Every tensor is whole chunks (its columns a multiple of 64), so a chunk is
+// 64 consecutive columns of one row; the lane writes that row segment's dot
+// product with x to partial[c] (fp32, products exact, one rounding per
+// fused multiply-add, four interleaved sums added in a fixed order).
+struct DotEpi {
+    struct Params {
+        uint32_t k;                              // tensors in the scope
+        uint32_t cols[GEMV_MAX_TENSORS];         // columns (a multiple of 64)
+        uint64_t off[GEMV_MAX_TENSORS + 1];      // first weight of each tensor
+        const uint16_t *x[GEMV_MAX_TENSORS];     // bf16 input of each tensor, 32-byte aligned
+        float *partial;                          // one fp32 per chunk
+    };
+    __device__ static __forceinline__ void apply(const LanesParams &, const Params &ep, uint32_t lane, uint32_t c,
+                                                 uint32_t t, uint32_t mrow, uint32_t exps) {
+        if (t == 0) return;
+        const uint64_t w0 = (uint64_t)c * LANE_SYMS;
+        uint32_t ti = 0;
+#pragma unroll
+        for (uint32_t i = 1; i < GEMV_MAX_TENSORS; ++i)
+            if (i < ep.k && w0 >= ep.off[i]) ti = i;
+        const uint32_t col0 = (uint32_t)(w0 - ep.off[ti]) % ep.cols[ti];
+        const uint16_t *xp = ep.x[ti] + col0;
+        float acc[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
+            const uint4 m = lds128(mrow + 16u * q);
+            const uint32_t e0 = lds32(exps + 512u * q), e1 = lds32(exps + 512u * q + 128u),
+                           e2 = lds32(exps + 512u * q + 256u), e3 = lds32(exps + 512u * q + 384u);
+            uint4 r0, r1, x0, x1;
+            ldg256_nc(xp + 16u * q, x0, x1);
+            join4(e0, m.x, r0.x, r0.y);
+            join4(e1, m.y, r0.z, r0.w);
+            join4(e2, m.z, r1.x, r1.y);
+            join4(e3, m.w, r1.z, r1.w);
+            float a = 0.f;
+            a = fma2_bf16(r0.x, x0.x, a);
+            a = fma2_bf16(r0.y, x0.y, a);
+            a = fma2_bf16(r0.z, x0.z, a);
+            a = fma2_bf16(r0.w, x0.w, a);
+            a = fma2_bf16(r1.x, x1.x, a);
+            a = fma2_bf16(r1.y, x1.y, a);
+            a = fma2_bf16(r1.z, x1.z, a);
+            a = fma2_bf16(r1.w, x1.w, a);
+            acc[j] = a;
+        }
+        ep.partial[c] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+};
+
 // Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes) | 2 x
 // (chunk_bits | stream span) | raw bytes (2048) | exponent word slots
 // (EXP_WORDS x 32).
@@ -181,8 +274,8 @@ __host__ __device__ constexpr uint32_t warp_smem_bytes(uint32_t sbuf_bytes) {
     return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + 4u * EXP_WORDS * 32u;
 }
 
-template <int NT>
-__global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
+template <int NT, class Epi>
+__global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const typename Epi::Params ep) {
     constexpr int NWARP = NT / 32;
     extern __shared__ __align__(16) uint8_t smem[];
     const uint32_t n_fast = 1u << prm.fast_bits;
@@ -313,36 +406,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm) {
         } else if (!good) {
             if (err) atomicOr(&g_status, err);
         } else {
-            // join: piece q (16 weights) of this lane's chunk, in the order
-            // (j + lane / 2) mod 4 so lanes spread over the banks
-            const uint32_t mrow = smem_u32(mbuf) + 64u * lane;
-            uint16_t *dst = prm.out + (size_t)c * LANE_SYMS;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
-                const uint4 m = lds128(mrow + 16u * q);
-                const uint32_t e0 = lds32(exps + 512u * q), e1 = lds32(exps + 512u * q + 128u),
-                               e2 = lds32(exps + 512u * q + 256u), e3 = lds32(exps + 512u * q + 384u);
-                uint4 r0, r1;
-                join4(e0, m.x, r0.x, r0.y);
-                join4(e1, m.y, r0.z, r0.w);
-                join4(e2, m.z, r1.x, r1.y);
-                join4(e3, m.w, r1.z, r1.w);
-                if (16u * q + 16u <= t) {
-                    if (prm.out32) {
-                        stg256_cs(dst + 16u * q, r0, r1);  // a whole sector per lane
-                    } else {
-                        __stcs(reinterpret_cast<uint4 *>(dst + 16u * q), r0);
-                        __stcs(reinterpret_cast<uint4 *>(dst + 16u * q + 8u), r1);
-                    }
-                } else {  // the last, partial chunk of the tensor: one weight at a time
-                    for (uint32_t i = 16u * q; i < t; ++i) {
-                        const uint32_t e = (lds32(exps + 128u * (i >> 2)) >> (8u * (i & 3u))) & 0xFFu;
-                        const uint32_t mb = (lds32(mrow + (i & ~3u)) >> (8u * (i & 3u))) & 0xFFu;
-                        dst[i] = join1(e, mb);
-                    }
-                }
-            }
+            Epi::apply(prm, ep, lane, c, t, smem_u32(mbuf) + 64u * lane, exps);
         }
         if (!has_next) break;
         __syncwarp();  // all lanes have read the raw bytes
@@ -361,29 +425,59 @@ uint32_t lanes_smem(uint32_t fast_bits, uint32_t sbuf_bytes) {
     return (8u << fast_bits) + (NT / 32) * warp_smem_bytes(sbuf_bytes);
 }
 
-typedef void (*lanes_fn)(const LanesParams);
-struct LanesVariant {
-    int nt;
-    lanes_fn fn;
-    uint32_t (*smem)(uint32_t, uint32_t);
-    int smem_set[16];  // dynamic shared memory opted in, per device
+// One table of CTA shapes per epilogue, largest CTA first: a larger CTA
+// shares one copy of the fast table among more warps; data with long codes
+// needs bigger stream slots and falls back to a smaller CTA.
+template <class Epi>
+struct LanesVariants {
+    typedef void (*fn_t)(const LanesParams, const typename Epi::Params);
+    struct V {
+        int nt;
+        fn_t fn;
+        uint32_t (*smem)(uint32_t, uint32_t);
+        int smem_set[16];  // dynamic shared memory opted in, per device
+    };
+    static V v[5];
 };
-// Largest CTA first: a larger CTA shares one copy of the fast table among
-// more warps; data with long codes needs bigger stream slots and falls back
-// to a smaller CTA.
-LanesVariant g_lanes[] = {
-    {1024, decode_lanes<1024>, lanes_smem<1024>, {0}},
-    {768, decode_lanes<768>, lanes_smem<768>, {0}},
-    {512, decode_lanes<512>, lanes_smem<512>, {0}},
-    {256, decode_lanes<256>, lanes_smem<256>, {0}},
-    {128, decode_lanes<128>, lanes_smem<128>, {0}},
+template <class Epi>
+typename LanesVariants<Epi>::V LanesVariants<Epi>::v[5] = {
+    {1024, decode_lanes<1024, Epi>, lanes_smem<1024>, {0}},
+    {768, decode_lanes<768, Epi>, lanes_smem<768>, {0}},
+    {512, decode_lanes<512, Epi>, lanes_smem<512>, {0}},
+    {256, decode_lanes<256, Epi>, lanes_smem<256>, {0}},
+    {128, decode_lanes<128, Epi>, lanes_smem<128>, {0}},
 };
 
-}  // namespace
+template <class Epi>
+dfw_status launch_lanes(const LanesParams &prm, const typename Epi::Params &ep, uint64_t n_groups, cudaStream_t s,
+                        int sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
+    for (auto &v : LanesVariants<Epi>::v) {
+        const uint32_t smem = v.smem(prm.fast_bits, prm.sbuf_bytes);
+        if (smem > 227u * 1024u) continue;
+        if (!v.smem_set[dev]) {
+            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+                return DFW_ECUDA;
+            v.smem_set[dev] = 1;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess) return DFW_ECUDA;
+        if (per_sm < 1) continue;
+        const uint64_t wpc = (uint64_t)v.nt / 32;
+        const uint64_t warps = (uint64_t)per_sm * sms * wpc;
+        const uint64_t want = n_groups < warps ? n_groups : warps;
+        v.fn<<<(unsigned)((want + wpc - 1) / wpc), v.nt, smem, s>>>(prm, ep);
+        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+    }
+    return DFW_EINVAL;  // even the smallest CTA does not fit
+}
 
-dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
-                               const uint16_t *d_chunk_bits, const uint64_t *d_group_start, const dfw_table *table,
-                               const dfw_lanes_info *info, uint16_t *d_out, cudaStream_t s, int sms) {
+// Checks a known-start plan against its table and fills the kernel
+// parameters (out left null).
+dfw_status lanes_params(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                        const uint16_t *d_chunk_bits, const uint64_t *d_group_start, const dfw_table *table,
+                        const dfw_lanes_info *info, LanesParams &prm) {
     const uint64_t n = table->n;
     if (info->chunk_symbols != LANE_SYMS || info->group_chunks != GROUP_CHUNKS ||
         info->n_chunks != (n + LANE_SYMS - 1) / LANE_SYMS ||
@@ -399,13 +493,12 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
         return DFW_EALIGN;
     if (info->max_group_bytes < 16 || (info->max_group_bytes & 15u) || info->max_group_bytes > 64u * 1024u)
         return DFW_EINVAL;
-    LanesParams prm;
     prm.stream = d_stream;
     prm.mant = d_mant;
     prm.lut = d_lut;
     prm.chunk_bits = d_chunk_bits;
     prm.group_start = d_group_start;
-    prm.out = d_out;
+    prm.out = nullptr;
     prm.n_chunks = (uint32_t)info->n_chunks;
     prm.n_groups = (uint32_t)info->n_groups;
     prm.last_t = (uint32_t)(n - LANE_SYMS * (info->n_chunks - 1));
@@ -414,27 +507,143 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     prm.fast_bits = fb;
     prm.n_tables = info->lut_tables;
     prm.sbuf_bytes = info->max_group_bytes;
-    prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
-    for (LanesVariant &v : g_lanes) {
-        const uint32_t smem = v.smem(fb, prm.sbuf_bytes);
-        if (smem > 227u * 1024u) continue;
-        if (!v.smem_set[dev]) {
-            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
-                return DFW_ECUDA;
-            v.smem_set[dev] = 1;
-        }
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess) return DFW_ECUDA;
-        if (per_sm < 1) continue;
-        const uint64_t wpc = (uint64_t)v.nt / 32;
-        const uint64_t warps = (uint64_t)per_sm * sms * wpc;
-        const uint64_t want = info->n_groups < warps ? info->n_groups : warps;
-        v.fn<<<(unsigned)((want + wpc - 1) / wpc), v.nt, smem, s>>>(prm);
-        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+    prm.out32 = 0u;
+    return DFW_OK;
+}
+
+// y = W x, one warp per output row: the row's chunk partials summed lane by
+// lane, then a fixed xor tree (the same order on every run).
+struct RowsParams {
+    uint32_t k;
+    uint32_t per_row[GEMV_MAX_TENSORS];     // chunks per row (columns / 64)
+    uint64_t chunk0[GEMV_MAX_TENSORS];      // first chunk of each tensor
+    uint64_t row0[GEMV_MAX_TENSORS + 1];    // rows before each tensor
+    float *y[GEMV_MAX_TENSORS];
+    const float *partial;
+};
+
+__global__ void __launch_bounds__(256) gemv_rows(const RowsParams rp) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint64_t total = rp.row0[rp.k];
+    const uint64_t wstride = (uint64_t)gridDim.x * 8u;
+    for (uint64_t R = (uint64_t)blockIdx.x * 8u + (threadIdx.x >> 5); R < total; R += wstride) {
+        uint32_t ti = 0;
+#pragma unroll
+        for (uint32_t i = 1; i < GEMV_MAX_TENSORS; ++i)
+            if (i < rp.k && R >= rp.row0[i]) ti = i;
+        const uint64_t r = R - rp.row0[ti];
+        const uint32_t per = rp.per_row[ti];
+        const float *p = rp.partial + rp.chunk0[ti] + r * per;
+        float sum = 0.f;
+        for (uint32_t j = lane; j < per; j += 32) sum += p[j];
+#pragma unroll
+        for (int d = 16; d > 0; d >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, d);
+        if (lane == 0) rp.y[ti][r] = sum;
     }
-    return DFW_EINVAL;  // even the smallest CTA does not fit
+}
+
+// Partials for a one-exponent scope (no stream): every weight is (sym, raw byte).
+__global__ void __launch_bounds__(256) gemv_single_partials(const uint8_t *__restrict__ mant, uint32_t sym,
+                                                            uint32_t n_chunks, const DotEpi::Params ep) {
+    const uint32_t R = rot_sym(sym) * 0x01010101u;
+    for (uint32_t c = blockIdx.x * 256u + threadIdx.x; c < n_chunks; c += gridDim.x * 256u) {
+        const uint64_t w0 = (uint64_t)c * LANE_SYMS;
+        uint32_t ti = 0;
+#pragma unroll
+        for (uint32_t i = 1; i < GEMV_MAX_TENSORS; ++i)
+            if (i < ep.k && w0 >= ep.off[i]) ti = i;
+        const uint32_t col0 = (uint32_t)(w0 - ep.off[ti]) % ep.cols[ti];
+        const uint16_t *xp = ep.x[ti] + col0;
+        float acc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 m = __ldg(reinterpret_cast<const uint4 *>(mant + w0) + q);
+            uint4 r0, r1, x0, x1;
+            ldg256_nc(xp + 16u * q, x0, x1);
+            join4(R, m.x, r0.x, r0.y);
+            join4(R, m.y, r0.z, r0.w);
+            join4(R, m.z, r1.x, r1.y);
+            join4(R, m.w, r1.z, r1.w);
+            float a = 0.f;
+            a = fma2_bf16(r0.x, x0.x, a);
+            a = fma2_bf16(r0.y, x0.y, a);
+            a = fma2_bf16(r0.z, x0.z, a);
+            a = fma2_bf16(r0.w, x0.w, a);
+            a = fma2_bf16(r1.x, x1.x, a);
+            a = fma2_bf16(r1.y, x1.y, a);
+            a = fma2_bf16(r1.z, x1.z, a);
+            a = fma2_bf16(r1.w, x1.w, a);
+            acc[q] = a;
+        }
+        ep.partial[c] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+}
+
+}  // namespace
+
+dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                               const uint16_t *d_chunk_bits, const uint64_t *d_group_start, const dfw_table *table,
+                               const dfw_lanes_info *info, uint16_t *d_out, cudaStream_t s, int sms) {
+    LanesParams prm;
+    const dfw_status st = lanes_params(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, prm);
+    if (st != DFW_OK) return st;
+    prm.out = d_out;
+    prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
+    return launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, info->n_groups, s, sms);
+}
+
+dfw_status launch_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
+                             const uint16_t *d_chunk_bits, const uint64_t *d_group_start, const dfw_table *table,
+                             const dfw_lanes_info *info, int k, const uint64_t *tensor_offsets, const uint32_t *cols,
+                             const uint16_t *const *d_x, float *const *d_y, float *d_partial, uint64_t partial_elems,
+                             cudaStream_t s, int sms) {
+    const uint64_t n = table->n;
+    if (k < 1 || k > (int)GEMV_MAX_TENSORS || !tensor_offsets || !cols || !d_x || !d_y || !d_partial)
+        return DFW_EINVAL;
+    if (tensor_offsets[0] != 0 || tensor_offsets[k] != n) return DFW_EINVAL;
+    const uint64_t n_chunks = n / LANE_SYMS;
+    if (partial_elems < n_chunks) return DFW_ENOMEM;
+    DotEpi::Params ep;
+    RowsParams rp;
+    std::memset(&ep, 0, sizeof(ep));
+    std::memset(&rp, 0, sizeof(rp));
+    ep.k = rp.k = (uint32_t)k;
+    ep.partial = d_partial;
+    rp.partial = d_partial;
+    for (int i = 0; i < k; ++i) {
+        const uint64_t size = tensor_offsets[i + 1] - tensor_offsets[i];
+        if (tensor_offsets[i + 1] <= tensor_offsets[i] || cols[i] == 0 || cols[i] % LANE_SYMS || size % cols[i] ||
+            size >= (1ull << 32) || !d_x[i] || !d_y[i])
+            return DFW_EINVAL;
+        if ((reinterpret_cast<uintptr_t>(d_x[i]) & 31u) || (reinterpret_cast<uintptr_t>(d_y[i]) & 3u))
+            return DFW_EALIGN;
+        ep.cols[i] = cols[i];
+        ep.off[i] = tensor_offsets[i];
+        ep.x[i] = d_x[i];
+        rp.per_row[i] = cols[i] / LANE_SYMS;
+        rp.chunk0[i] = tensor_offsets[i] / LANE_SYMS;
+        rp.row0[i + 1] = rp.row0[i] + size / cols[i];
+        rp.y[i] = d_y[i];
+    }
+    ep.off[k] = n;
+    if (!d_mant || (reinterpret_cast<uintptr_t>(d_mant) & 15u) || (reinterpret_cast<uintptr_t>(d_partial) & 15u))
+        return d_mant ? DFW_EALIGN : DFW_EINVAL;
+    if (table->total_bits == 0) {  // one distinct exponent: no stream, no plan needed
+        const uint64_t want = (n_chunks + 255) / 256, cap = (uint64_t)sms * 8;
+        gemv_single_partials<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(d_mant, table->single_symbol,
+                                                                                 (uint32_t)n_chunks, ep);
+        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    } else {
+        LanesParams prm;
+        const dfw_status st = lanes_params(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, prm);
+        if (st != DFW_OK) return st;
+        const dfw_status st2 = launch_lanes<DotEpi>(prm, ep, info->n_groups, s, sms);
+        if (st2 != DFW_OK) return st2;
+    }
+    const uint64_t rows = rp.row0[k];
+    const uint64_t want = (rows + 7) / 8, cap = (uint64_t)sms * 16;
+    gemv_rows<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(rp);
+    return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
 }
 
 }  // namespace dfw

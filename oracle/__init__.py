@@ -233,3 +233,28 @@ def chunk_aux(enc: Encoded, M: int = 64, G: int = 32) -> tuple[np.ndarray, np.nd
     _check(_load().oracle_chunk_aux(_p(stream, ctypes.c_uint8), enc.total_bits, _p(ln, ctypes.c_uint8), enc.n, M, G,
                                     _p(bits, ctypes.c_uint32), _p(starts, ctypes.c_uint64)), "chunk_aux")
     return bits[: n_groups * G], starts
+
+
+# ---------------------------------------------------------------- y = W x
+
+def bf16_values(u) -> np.ndarray:
+    """Exact float64 values of bf16 bit patterns: a bf16 is the upper half of
+    an IEEE binary32 whose lower 16 bits are zero."""
+    u = np.ascontiguousarray(_u16(u))
+    return (u.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def gemv(w, rows: int, cols: int, x) -> np.ndarray:
+    """y = W x in float64 for the row-major bf16 matrix W (rows x cols bit
+    patterns, e.g. the oracle's decode) and the bf16 vector x (cols).  Every
+    product of two bf16 values is exact in float64 (8 + 8 significand bits);
+    the sums use numpy's float64 matrix product as a library step."""
+    W = bf16_values(w).reshape(rows, cols)
+    return W @ bf16_values(x)
+
+
+def gemv_abs(w, rows: int, cols: int, x) -> np.ndarray:
+    """sum_j |W[i, j] x[j]| per row: the scale of the rounding-error bound of
+    any fp32 summation of the products."""
+    W = np.abs(bf16_values(w).reshape(rows, cols))
+    return W @ np.abs(bf16_values(x))

@@ -520,3 +520,69 @@ def test_chunk_aux_against_independent_walk(oracle, M, G, kind):
         assert starts[g] == st[M * G * g]
     assert starts[-1] == enc.total_bits
     assert int(bits.sum()) == enc.total_bits
+
+
+# ---------------------------------------------------------------- y = W x
+
+def _u16_normal(rng, n: int) -> np.ndarray:
+    """bf16 patterns of N(0, 0.02) draws (round to nearest even by hand)."""
+    f = (rng.standard_normal(n) * 0.02).astype(np.float32).view(np.uint32)
+    return ((f + 0x7FFF + ((f >> 16) & 1)) >> 16).astype(np.uint16)
+
+
+def _bf16_of(v: float) -> int:
+    """bf16 pattern of a float32-exact value whose low 16 bits are zero."""
+    u = int(np.array([v], np.float32).view(np.uint32)[0])
+    assert u & 0xFFFF == 0
+    return u >> 16
+
+
+def test_bf16_values_closed_forms(oracle):
+    pats = np.array([0x3F80, 0xC000, 0x0001, 0x8000, 0x7F80, 0x4049, 0x3C23], np.uint16)
+    want = [1.0, -2.0, 2.0 ** -133, -0.0, np.inf, 3.140625, 0.0099487304687500]
+    got = oracle.bf16_values(pats)
+    assert got[:5].tolist() == want[:5] and np.signbit(got[3])
+    # 0x4049 = 2^1 * (1 + 0x49 / 128); 0x3C23 = 2^-7 * (1 + 0x23 / 128)
+    assert got[5] == 2.0 * (1 + 0x49 / 128) == want[5]
+    assert got[6] == 2.0 ** -7 * (1 + 0x23 / 128)
+
+
+def test_gemv_hand_worked(oracle):
+    """tests/golden/gemv_small.txt: a 2 x 64 case summed by hand."""
+    kv = dict(line.split(":", 1) for line in open(os.path.join(GOLDEN, "gemv_small.txt"))
+              if ":" in line and not line.startswith("#"))
+    rows, cols = int(kv["rows"]), int(kv["cols"])
+    want = [float(v) for v in kv["y"].split()]
+    w = np.empty((rows, cols), np.uint16)
+    w[0, :] = 0x3F80
+    w[1, 0::2] = 0x3F00
+    w[1, 1::2] = 0xBE80
+    x = np.array([_bf16_of(j + 1) for j in range(cols)], np.uint16)
+    assert oracle.gemv(w.reshape(-1), rows, cols, x).tolist() == want
+
+
+def test_gemv_basis_vectors_pick_columns(oracle):
+    rng = np.random.default_rng(5)
+    rows, cols = 7, 128
+    w = _u16_normal(rng, rows * cols)
+    for j in (0, 1, 63, 64, 127):
+        x = np.zeros(cols, np.uint16)
+        x[j] = 0x3F80  # 1.0
+        y = oracle.gemv(w, rows, cols, x)
+        assert np.array_equal(y, oracle.bf16_values(w).reshape(rows, cols)[:, j])
+
+
+def test_gemv_against_exact_rationals(oracle):
+    """Exact rational sums (fractions) of the same products: the float64
+    result is within float64 rounding of them."""
+    from fractions import Fraction
+    rng = np.random.default_rng(6)
+    rows, cols = 3, 192
+    w, x = _u16_normal(rng, rows * cols), _u16_normal(rng, cols)
+    y = oracle.gemv(w, rows, cols, x)
+    scale = oracle.gemv_abs(w, rows, cols, x)
+    wv = oracle.bf16_values(w).reshape(rows, cols)
+    xv = oracle.bf16_values(x)
+    for i in range(rows):
+        exact = sum(Fraction(float(wv[i, j])) * Fraction(float(xv[j])) for j in range(cols))
+        assert abs(Fraction(float(y[i])) - exact) <= Fraction(cols * 2.0 ** -53) * Fraction(float(scale[i]))
