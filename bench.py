@@ -428,6 +428,98 @@ def run_encode_mode(args, rank, world, blocks, wdesc, device):
     return 0 if ok else 1
 
 
+# ------------------------------------------------------------------ gemv mode
+
+def run_gemv_mode(args, rank, world, blocks, wdesc, device):
+    """Times decode fused with y = W x (``dfw_decode_gemv_lanes``) over every
+    scope of the workload (each tensor read as a row-major [out, in] matrix,
+    the embedding as a tied 128256 x 4096 output matrix), against decode into
+    the scratch buffer followed by cuBLAS's bf16 matrix-vector product on the
+    same inputs, timed in the same run."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    devs, _ = prepare(blocks, device, args.window, args.tile, args.threads, "lanes")
+    gen = torch.Generator(device=device).manual_seed(77)
+    work = []
+    for b, d in zip(blocks, devs):
+        cols = [workloads.matrix_cols(t) for t in b.tensors]
+        xs = [torch.randn(c, generator=gen, device=device).to(torch.bfloat16) for c in cols]
+        offs = [int(v) for v in d.tensor_offsets]
+        ys = [torch.empty((offs[i + 1] - offs[i]) // cols[i], dtype=torch.float32, device=device)
+              for i in range(len(cols))]
+        work.append((d, cols, xs, ys, offs))
+    nmax = max(d.n for d in devs)
+    partial = torch.empty(nmax // 64 + 1, dtype=torch.float32, device=device)
+    scratch = torch.empty(nmax, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def fused():
+        for d, cols, xs, ys, _ in work:
+            dfw.decode_gemv_lanes(d, xs, cols, ys=ys, partial=partial, stream=stream)
+
+    def unfused():
+        for d, cols, xs, ys, offs in work:
+            dfw.decode_lanes(d, scratch, stream=stream)
+            for i, c in enumerate(cols):
+                w = scratch[offs[i]: offs[i + 1]].view(-1, c)
+                torch.mv(w, xs[i])
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    sampler = ClockSampler(int(device.index or 0))
+    sampler.start()
+    ms_fused = timed(fused)
+    clocks = sampler.stop()
+    ms_unfused = timed(unfused)
+    ok = dfw.check_status(stream) == dfw.OK
+    # every y against fp64 of the decoded weights (decode_lanes is bit-exact
+    # by its own tests) within the fp32 summation bound
+    fused()
+    for d, cols, xs, ys, offs in work:
+        dfw.decode_lanes(d, scratch, stream=stream)
+        for i, c in enumerate(cols):
+            w = scratch[offs[i]: offs[i + 1]].view(-1, c).double()
+            x = xs[i].double()
+            want, scale = w @ x, w.abs() @ x.abs()
+            gamma = c * 2.0 ** -24 / (1 - c * 2.0 ** -24)
+            ok = ok and bool(((ys[i].double() - want).abs() <= gamma * scale + 1e-30).all())
+    n_total = sum(d.n for d in devs)
+    alg = sum(int(d.table.stream_bytes) + d.n + 2 * d.chunk_bits.numel() + 8 * d.group_start.numel()
+              + 4 * d.lut.numel() + 8 * (d.n // 64) + sum(2 * c for c in cols) + 4 * sum(y.numel() for y in ys)
+              for d, cols, _, ys, _ in work)
+    peak, peak_kind = measured_peak_hbm()
+    achieved = alg / (ms_fused * 1e-3) / 1e9
+    line = {
+        "metric": "weights/s through decode fused with y = W x (bf16 x, fp32 y; weights never written)",
+        "value": world * n_total / (ms_fused * 1e-3), "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_fused, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8+bf16->fp32", "data": "synthetic",
+        "config": {"workload": wdesc, "weights": n_total, "code_tables": len(devs), "mode": "gemv",
+                   "l2": "inputs larger than L2 (each step reads every scope's compressed form)",
+                   "parallelism": f"replica{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_kind, "kernel": "decode_lanes<DotEpi> + gemv_rows",
+                     "algorithmic_bytes_per_step": alg},
+        "unfused": {"ms_per_step": ms_unfused, "what": "decode_lanes into scratch, then torch.mv (cuBLAS, bf16)",
+                    "speedup_of_fused": ms_unfused / ms_fused},
+        "clocks": clocks, "gpu_launches": args.steps * 2 * len(devs), "verified_within_fp32_bound": bool(ok),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if ok else 1
+
+
 # ------------------------------------------------------------------ main
 
 def main(argv=None):
@@ -446,8 +538,9 @@ def main(argv=None):
     ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--mode", default="decode", choices=["decode", "encode"],
-                    help="decode: the decode path (default); encode: the GPU encoder")
+    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv"],
+                    help="decode: the decode path (default); encode: the GPU encoder; "
+                         "gemv: decode fused with y = W x")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -471,8 +564,9 @@ def main(argv=None):
     import lossless_entropy_coded_canonical_b200 as dfw
     dfw.lib()
     dfw.check()
-    if args.mode == "encode":
-        rc = run_encode_mode(args, rank, world, blocks, wdesc, device)
+    if args.mode in ("encode", "gemv"):
+        run = run_encode_mode if args.mode == "encode" else run_gemv_mode
+        rc = run(args, rank, world, blocks, wdesc, device)
         if world > 1:
             dist.destroy_process_group()
         return rc

@@ -211,3 +211,15 @@ def scaled(block: BlockSpec, n_total: int) -> BlockSpec:
 
 def generate_block(block: BlockSpec, device="cpu") -> list[torch.Tensor]:
     return [generate(t, device) for t in block.tensors]
+
+
+def matrix_cols(t: TensorSpec) -> int:
+    """Columns (input features) of a tensor read as a row-major [out, in]
+    matrix: transformer matrices take the 4096-wide hidden state except the
+    MLP down projection, which takes the intermediate state; a square test
+    matrix takes its side."""
+    if t.name == "down":
+        return t.numel // 4096
+    if t.name == "w":
+        return int(round(t.numel ** 0.5))
+    return 4096
