@@ -70,10 +70,10 @@ __device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_
 // last codeword decoded.
 //
 // The inner loop is straight-line code: it keeps the word after the current
-// pair in a register, selects it in when the position crosses a word (and
-// only then loads the next one), and it always stores the accumulator's low
-// word and advances by select.  Only an escape or the chunk's last lookup
-// leaves it, for one step of the general path.
+// pair in a register, moves it in (predicated) when the position crosses a
+// word and only then loads the next one; it always stores the accumulator's
+// low word and moves to the next slot when the word is full.  Only an escape
+// or the chunk's last lookup leaves it, for one step of the general path.
 __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int left8, uint32_t fast,
                                                  uint32_t kshift, const uint32_t *__restrict__ g_hier,
                                                  uint32_t n_tables, uint32_t ep, uint32_t &err) {
@@ -88,7 +88,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
     uint32_t c = lds32(wa + 8u);
     wa += 12u;
     uint32_t p = r & 31u;
-    uint32_t lo = 0u, sh = 0u;
+    uint32_t lo = 0u, m = 1u;  // m = 2^(bits of lo in use)
     const uint32_t kmul = 1u << (32u - kshift);  // x >> kshift == mulhi(x, 2^(32 - kshift))
     while (left8 > 0) {
         uint32_t x, syms, c8, cb, ey;
@@ -97,13 +97,13 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         // reads as all ones through the sign-replicating byte permute (the
         // escape flag is the entry's top bit).  The next stream word is
         // loaded only when the window crosses into c, one lookup ahead of its
-        // use.  Symbols are appended by multiplication (m = 2^sh: lo += syms
-        // * m, spill = mulhi(syms, m)) to keep work off the integer-logic
-        // pipe.
+        // use.  Symbols are appended by multiplication with m = 2^sh (lo +=
+        // syms * m, spill = mulhi(syms, m)); m advances by a rotation by
+        // 8 * count, which wraps exactly when the word fills.
         asm volatile(
             "{\n\t"
             ".reg .pred pl, pa, pf;\n\t"
-            ".reg .b32 t0, t1, sp, ex, nx, ad;\n"
+            ".reg .b32 t0, mn, sp, ex, ad;\n"
             "LANES_LOOP:\n\t"
             "shf.l.wrap.b32 %0, %7, %6, %9;\n\t"  // x = stream bits [p, p + 32)
             "mul.hi.u32 t0, %0, %15;\n\t"         // fast-table key
@@ -115,28 +115,26 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             "@pl bra LANES_EXIT;\n\t"
             "mad.lo.u32 %9, %3, 1, %9;\n\t"  // p += bits used
             "setp.ge.u32 pa, %9, 32;\n\t"
-            "prmt.b32 nx, %8, 0, 0x0123;\n\t"
-            "selp.b32 %6, %7, %6, pa;\n\t"  // a = b
-            "selp.b32 %7, nx, %7, pa;\n\t"  // b = c
+            "@pa mov.b32 %6, %7;\n\t"                // a = b
+            "@pa prmt.b32 %7, %8, 0, 0x0123;\n\t"    // b = c, byte-swapped
             "@pa ld.shared.u32 %8, [%10];\n\t"
             "@pa add.u32 %10, %10, 4;\n\t"
             "and.b32 %9, %9, 31;\n\t"
-            "shl.b32 t1, 1, %12;\n\t"  // m = 2^sh
-            "mad.lo.u32 %11, ex, t1, %11;\n\t"
-            "mul.hi.u32 sp, ex, t1;\n\t"
-            "mad.lo.u32 %12, %2, 1, %12;\n\t"  // sh += 8 * count
+            "mad.lo.u32 %11, ex, %12, %11;\n\t"      // lo += syms * m
+            "mul.hi.u32 sp, ex, %12;\n\t"            // the part past the word
             "st.shared.u32 [%5], %11;\n\t"
-            "setp.ge.u32 pf, %12, 32;\n\t"
-            "@pf add.u32 %5, %5, 128;\n\t"  // next word slot of this lane
-            "selp.b32 %11, sp, %11, pf;\n\t"
-            "and.b32 %12, %12, 31;\n\t"
-            "mad.lo.s32 %13, %2, -1, %13;\n\t"  // left8 -= 8 * count
+            "shf.l.wrap.b32 mn, %12, %12, %2;\n\t"   // m rotated by 8 * count
+            "setp.le.u32 pf, mn, %12;\n\t"           // wrapped: the word is full
+            "@pf add.u32 %5, %5, 128;\n\t"           // next word slot of this lane
+            "@pf mov.b32 %11, sp;\n\t"
+            "mov.b32 %12, mn;\n\t"
+            "mad.lo.s32 %13, %2, -1, %13;\n\t"       // left8 -= 8 * count
             "bra LANES_LOOP;\n"
             "LANES_EXIT:\n\t"
             "mov.b32 %1, ex;\n\t"
             "}"
             : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(ep), "+r"(a), "+r"(b), "+r"(c), "+r"(p),
-              "+r"(wa), "+r"(lo), "+r"(sh), "+r"(left8)
+              "+r"(wa), "+r"(lo), "+r"(m), "+r"(left8)
             : "r"(fast), "r"(kmul)
             : "memory");
         if (cb != 255u) {
@@ -161,18 +159,18 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             wa += 4u;
             p -= 32u;
         }
-        const uint32_t hi = __funnelshift_l(syms, 0u, sh);
-        lo |= syms << sh;
-        sh += c8;
-        if (sh >= 32u) {
+        const uint32_t spill = __umulhi(syms, m);
+        lo += syms * m;
+        const uint32_t mn = __funnelshift_l(m, m, c8);
+        if (mn <= m) {
             sts32(ep, lo);
             ep += 128u;
-            lo = hi;
-            sh -= 32u;
+            lo = spill;
         }
+        m = mn;
         left8 -= (int)c8;
     }
-    if (sh) sts32(ep, lo);
+    if (m != 1u) sts32(ep, lo);
     return 8u * (wa - sw) - 96u + p;
 }
 
