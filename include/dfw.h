@@ -382,6 +382,73 @@ dfw_status dfw_encode_device_noalloc(const uint16_t *d_bf16, uint64_t n, int cap
                                      uint16_t *d_chunk_bits, uint64_t *d_group_start, dfw_table *table,
                                      dfw_lanes_info *info, void *cuda_stream);
 
+/*
+ * rANS VARIANT (the ANS coder of the ~1.5:1 page's abstract; the LazyWeights
+ * write-up compares Huffman with rANS).  The pages fix no format; this one:
+ *   - the same split: exponent symbols coded, raw bytes stored as they are;
+ *   - frequencies quantised to M = 2^DFW_RANS_SCALE_BITS: floor(count M / n),
+ *     at least 1 for a present exponent; a positive remainder goes to the
+ *     most frequent exponent, a negative one is taken one unit at a time from
+ *     the exponent with the largest frequency above 1 (smallest exponent on
+ *     ties, both ways);
+ *   - states x in [2^16, 2^32); exponent s (frequency f, cumulative start c)
+ *     encodes as x' = floor(x / f) M + (x mod f) + c after emitting the low
+ *     16 bits of x while x >= f (2^16 / M) 2^16; decoding inverts it and
+ *     reloads 16 bits while x < 2^16;
+ *   - blocks of DFW_RANS_BLOCK exponents, coded independently; in a block,
+ *     exponent i belongs to state i mod DFW_RANS_LANES; the encoder runs
+ *     backwards so a decoder takes steps k = 0, 1, ... (exponents 32k ..
+ *     32k + 31, one per state) and then reloads the states that need it in
+ *     increasing state order, each taking the next word;
+ *   - a block is its 32 final encoder states (u32), its words in decoding
+ *     order (u16), zero padding to 16 bytes; block_start[b] is its byte
+ *     offset, block_start[n_blocks] the stream length.  Every state starts
+ *     at 2^16, so a correct decode ends with every state at 2^16.
+ */
+#define DFW_RANS_SCALE_BITS 12
+#define DFW_RANS_LANES 32
+#define DFW_RANS_BLOCK 16384
+
+typedef struct dfw_rans_table {
+    uint32_t version;          /* DFW_FORMAT_VERSION */
+    uint32_t scale_bits;       /* DFW_RANS_SCALE_BITS */
+    uint32_t lanes;            /* DFW_RANS_LANES */
+    uint32_t block_syms;       /* DFW_RANS_BLOCK */
+    uint64_t n;                /* weights */
+    uint64_t n_blocks;         /* ceil(n / block_syms) */
+    uint64_t stream_bytes;     /* block_start[n_blocks] */
+    uint32_t max_block_bytes;  /* largest block */
+    uint32_t reserved;         /* zero */
+    uint16_t freq[256];        /* quantised frequency per exponent (sum 2^scale_bits) */
+} dfw_rans_table;
+
+/* Worst-case rANS stream bytes for n weights. */
+uint64_t dfw_rans_stream_bound(uint64_t n);
+
+/*
+ * dfw_rans_encode -- host: the k tensors' concatenation (one table), coded
+ * as above; blocks are coded by n_threads threads (0 = all), the bytes are
+ * the same for any thread count.
+ *   stream       host, stream_capacity bytes (dfw_rans_stream_bound(n) suffices)
+ *   mant         host, dfw_mant_bytes(n) raw bytes (output)
+ *   block_start  host, n_blocks + 1 u64 (output)
+ * Errors: DFW_EINVAL, DFW_ENOMEM (table->stream_bytes then holds the need).
+ */
+dfw_status dfw_rans_encode(const uint16_t *const *tensors, const uint64_t *sizes, int k,
+                           uint8_t *stream, uint64_t stream_capacity, uint8_t *mant,
+                           uint64_t mant_capacity, uint64_t *block_start, dfw_rans_table *table,
+                           int n_threads);
+
+/*
+ * dfw_rans_decode -- GPU: one warp per block, 32 states decoded per step,
+ * reloads ranked by warp ballot.  Device buffers d_stream (stream_bytes,
+ * 16-byte aligned), d_mant (dfw_mant_bytes(n)), d_block_start (n_blocks + 1),
+ * d_out (n bf16).  A block that does not end with every state at 2^16 and
+ * every word used is flagged through dfw_check.  Errors as dfw_decode.
+ */
+dfw_status dfw_rans_decode(const uint8_t *d_stream, const uint8_t *d_mant, const uint64_t *d_block_start,
+                           const dfw_rans_table *table, uint16_t *d_out, void *cuda_stream);
+
 /* Static English text for a status code. */
 const char *dfw_strerror(dfw_status status);
 

@@ -21,12 +21,13 @@ from dataclasses import dataclass
 import numpy as np
 import torch
 
-from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, LanesInfo, PlanInfo, Table,
-                   check as _check, lib)
+from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, LanesInfo, PlanInfo, RansTable,
+                   Table, check as _check, lib)
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
            "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "LanesInfo",
            "encode_device", "encode_device_scratch_bytes", "decode_gemv_lanes",
+           "rans_encode", "RansEncoded", "DeviceRans", "rans_decode", "RansTable",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
            "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
 
@@ -344,6 +345,85 @@ def encode_device(x: torch.Tensor, cap: int = 32, fast_bits: int = 0, stream=Non
 
 def encode_device_scratch_bytes() -> int:
     return int(lib().dfw_encode_device_scratch_bytes(0))
+
+
+# ---------------------------------------------------------------- rANS variant
+
+@dataclass
+class RansEncoded:
+    """Host result of dfw_rans_encode."""
+    stream: torch.Tensor       # uint8[table.stream_bytes]
+    mant: torch.Tensor         # uint8[mant_bytes(n)]
+    block_start: torch.Tensor  # int64 view of uint64[n_blocks + 1]
+    table: RansTable
+    tensor_offsets: np.ndarray | None = None
+
+    @property
+    def n(self) -> int:
+        return int(self.table.n)
+
+
+def rans_encode(tensors, n_threads: int = 0, pin: bool = False) -> RansEncoded:
+    """Encodes one host bf16 tensor, or several with one table, with the rANS
+    variant of the exponent coder (``dfw_rans_encode``)."""
+    if isinstance(tensors, (torch.Tensor, np.ndarray)):
+        tensors = [tensors]
+    us = [_as_u16_host(t) for t in tensors]
+    k = len(us)
+    n = int(sum(u.numel() for u in us))
+    ptrs = (ctypes.c_void_p * max(k, 1))(*[_ptr(u) for u in us])
+    sizes = (ctypes.c_uint64 * max(k, 1))(*[u.numel() for u in us])
+    table = RansTable()
+    cap = int(lib().dfw_rans_stream_bound(n))
+    stream = torch.empty(max(cap, 16), dtype=torch.uint8, pin_memory=pin)
+    mant = torch.empty(mant_bytes(n), dtype=torch.uint8, pin_memory=pin)
+    nb = (n + 16383) // 16384
+    starts = torch.empty(nb + 1, dtype=torch.int64, pin_memory=pin)
+    _check(lib().dfw_rans_encode(ptrs, sizes, k, _ptr(stream), stream.numel(), _ptr(mant), mant.numel(),
+                                 _ptr(starts), ctypes.byref(table), n_threads), "dfw_rans_encode")
+    used = int(table.stream_bytes)
+    stream = torch.empty(max(used, 16), dtype=torch.uint8, pin_memory=pin).copy_(
+        torch.cat([stream[:used], torch.zeros(max(0, 16 - used), dtype=torch.uint8)]))
+    offs = np.concatenate([[0], np.cumsum([u.numel() for u in us])]).astype(np.uint64)
+    return RansEncoded(stream, mant, starts, table, offs)
+
+
+@dataclass
+class DeviceRans:
+    """An rANS-coded tensor or block resident in device memory."""
+    stream: torch.Tensor
+    mant: torch.Tensor
+    block_start: torch.Tensor
+    table: RansTable
+    tensor_offsets: np.ndarray | None = None
+
+    @staticmethod
+    def upload(enc: RansEncoded, device="cuda") -> "DeviceRans":
+        return DeviceRans(enc.stream.to(device), enc.mant.to(device), enc.block_start.to(device), enc.table,
+                          enc.tensor_offsets)
+
+    @property
+    def n(self) -> int:
+        return int(self.table.n)
+
+    def compressed_bytes(self, with_aux: bool = True) -> int:
+        b = int(self.table.stream_bytes) + self.n + 512
+        return b + (8 * self.block_start.numel() if with_aux else 0)
+
+    def algorithmic_bytes(self) -> int:
+        """Stream + block offsets read, one raw byte read and one bf16
+        written per weight."""
+        return int(self.table.stream_bytes) + 8 * self.block_start.numel() + 3 * self.n
+
+
+def rans_decode(dr: DeviceRans, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    if out is None:
+        out = torch.empty(dr.n, dtype=torch.bfloat16, device=dr.mant.device)
+    if out.numel() < dr.n or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor of at least n elements")
+    _check(lib().dfw_rans_decode(_ptr(dr.stream), _ptr(dr.mant), _ptr(dr.block_start), ctypes.byref(dr.table),
+                                 _ptr(out), _stream_handle(stream)), "dfw_rans_decode")
+    return out
 
 
 def check(stream=None) -> None:

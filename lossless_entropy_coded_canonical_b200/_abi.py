@@ -39,11 +39,19 @@ class LanesInfo(ctypes.Structure):
                 ("lut_tables", ctypes.c_uint32), ("fast_bits", ctypes.c_uint32)]
 
 
+class RansTable(ctypes.Structure):
+    _fields_ = [("version", ctypes.c_uint32), ("scale_bits", ctypes.c_uint32), ("lanes", ctypes.c_uint32),
+                ("block_syms", ctypes.c_uint32), ("n", ctypes.c_uint64), ("n_blocks", ctypes.c_uint64),
+                ("stream_bytes", ctypes.c_uint64), ("max_block_bytes", ctypes.c_uint32),
+                ("reserved", ctypes.c_uint32), ("freq", ctypes.c_uint16 * 256)]
+
+
 _lib = None
 
 # name -> (restype, argtypes); the symbols include/dfw.h declares
 _vp, _u64, _i = ctypes.c_void_p, ctypes.c_uint64, ctypes.c_int
 _TP, _IP, _LP = ctypes.POINTER(Table), ctypes.POINTER(PlanInfo), ctypes.POINTER(LanesInfo)
+_RP = ctypes.POINTER(RansTable)
 SIGNATURES = {
     "dfw_stream_bound": (_u64, [_u64]),
     "dfw_mant_bytes": (_u64, [_u64]),
@@ -62,6 +70,9 @@ SIGNATURES = {
     "dfw_pack_device": (_i, [_vp, _TP, _LP, _vp, _vp, _u64, _vp]),
     "dfw_lanes_lut": (_i, [_TP, _LP, _vp]),
     "dfw_encode_device_noalloc": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _TP, _LP, _vp]),
+    "dfw_rans_stream_bound": (_u64, [_u64]),
+    "dfw_rans_encode": (_i, [_vp, _vp, _i, _vp, _u64, _vp, _u64, _vp, _RP, _i]),
+    "dfw_rans_decode": (_i, [_vp, _vp, _vp, _RP, _vp, _vp]),
     "dfw_check": (_i, [_vp]),
     "dfw_strerror": (ctypes.c_char_p, [_i]),
 }

@@ -15,8 +15,8 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libdfw.so")
-SOURCES = ["dfw_host.cpp", "dfw_decode.cu", "dfw_encode.cu"]
-HEADERS = ["dfw_internal.h", "dfw_device.cuh", "dfw_lanes.cuh", os.path.join("..", "..", "include", "dfw.h")]
+SOURCES = ["dfw_host.cpp", "dfw_decode.cu", "dfw_encode.cu", "dfw_rans.cpp"]
+HEADERS = ["dfw_internal.h", "dfw_device.cuh", "dfw_lanes.cuh", "dfw_rans.cuh", os.path.join("..", "..", "include", "dfw.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

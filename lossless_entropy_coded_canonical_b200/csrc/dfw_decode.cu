@@ -44,6 +44,7 @@ __device__ unsigned int g_status;  // device status word (sticky error bits)
 
 #include "dfw_device.cuh"
 #include "dfw_lanes.cuh"
+#include "dfw_rans.cuh"
 
 namespace dfw {
 namespace {
@@ -495,6 +496,23 @@ extern "C" dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8
         return DFW_ECUDA;
     return launch_gemv_lanes(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, k, tensor_offsets,
                              cols, d_x, d_y, d_partial, partial_elems, static_cast<cudaStream_t>(cuda_stream), sms);
+}
+
+extern "C" dfw_status dfw_rans_decode(const uint8_t *d_stream, const uint8_t *d_mant, const uint64_t *d_block_start,
+                                      const dfw_rans_table *table, uint16_t *d_out, void *cuda_stream) {
+    if (!table || table->version != DFW_FORMAT_VERSION || table->scale_bits != DFW_RANS_SCALE_BITS ||
+        table->lanes != DFW_RANS_LANES || table->block_syms != DFW_RANS_BLOCK ||
+        table->n_blocks != (table->n + DFW_RANS_BLOCK - 1) / DFW_RANS_BLOCK)
+        return DFW_EINVAL;
+    if (table->n == 0) return DFW_OK;
+    if (!d_stream || !d_mant || !d_block_start || !d_out) return DFW_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(d_stream) | reinterpret_cast<uintptr_t>(d_block_start)) & 15u) return DFW_EALIGN;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFW_ECUDA;
+    return launch_rans_decode(d_stream, d_mant, d_block_start, table, d_out, static_cast<cudaStream_t>(cuda_stream),
+                              sms);
 }
 
 extern "C" dfw_status dfw_check(void *cuda_stream) {

@@ -1,0 +1,202 @@
+// dfw_rans.cuh -- GPU decoder of the rANS variant (included by dfw_decode.cu).
+//
+// Persistent warps, one rANS block (16384 exponents, 32 interleaved states)
+// at a time.  Per CTA the decode table for the 2^12 slots is built once in
+// shared memory: entry = exponent | (f - 1) << 8 | (slot - c) << 20, so a
+// step costs one shared load and one multiply-add per state.  Per warp, lane
+// 0 stages blocks into two shared slots with 1-D TMA bulk copies (mbarrier
+// completion, started one block ahead).  A step: each lane decodes the
+// exponent of its state, the warp ballots which states fell below 2^16, each
+// of those takes the word at (next word + its rank among them), and the
+// lane joins its exponent with the raw byte into bf16 (one 2-byte store per
+// lane: 64 contiguous bytes per warp).  A block must end with every state at
+// 2^16 and every word used; otherwise the status word records it.
+#pragma once
+
+#include "dfw_device.cuh"
+
+namespace dfw {
+namespace {
+
+constexpr uint32_t RANS_SLOTS = 1u << DFW_RANS_SCALE_BITS;
+constexpr uint32_t RANS_HEAD = 4u * DFW_RANS_LANES;  // state bytes at the start of a block
+constexpr uint32_t RANS_TABLE_BYTES = 4u * RANS_SLOTS + 1040u;  // decode table + 257 cumulative starts, 16-aligned
+
+struct RansParams {
+    const uint8_t *stream;
+    const uint8_t *mant;
+    const uint64_t *block_start;
+    uint16_t *out;
+    uint64_t n, stream_bytes;
+    uint32_t n_blocks, slot_bytes;
+    uint16_t freq[256];
+};
+
+template <int NT>
+__global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
+    constexpr int NWARP = NT / 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint32_t *s_tab = reinterpret_cast<uint32_t *>(smem);
+    uint32_t *s_cum = s_tab + RANS_SLOTS;  // 257 cumulative starts
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // decode table: exponent s owns slots [c_s, c_s + f_s)
+    if (tid == 0) {
+        uint32_t c = 0;
+        for (int s = 0; s < 256; ++s) {
+            s_cum[s] = c;
+            c += prm.freq[s];
+        }
+        s_cum[256] = c;
+    }
+    __syncthreads();
+    bool bad = s_cum[256] != RANS_SLOTS;
+    for (int s = tid; s < 256 && !bad; s += NT) {
+        const uint32_t f = prm.freq[s], c = s_cum[s];
+        for (uint32_t k = 0; k < f; ++k) s_tab[c + k] = (uint32_t)s | ((f - 1u) << 8) | (k << 20);
+    }
+    if (__syncthreads_or(bad)) {
+        if (tid == 0) atomicOr(&g_status, ST_LUT);
+        return;
+    }
+
+    uint8_t *wbase = smem + RANS_TABLE_BYTES + warp * (16u + 2u * prm.slot_bytes);
+    const uint32_t bar0 = smem_u32(wbase);
+    uint8_t *slots = wbase + 16;
+    const uint32_t gstride = gridDim.x * NWARP;
+    uint32_t b = blockIdx.x * NWARP + warp;
+    if (b >= prm.n_blocks) return;
+    if (lane == 0) {
+        mbar_init(bar0, 1);
+        mbar_init(bar0 + 8u, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+
+    // lane 0: block bb into slot s (its bytes, capped to the slot)
+    auto issue = [&](uint32_t bb, uint32_t s) {
+        const uint64_t b0 = __ldg(prm.block_start + bb), b1 = __ldg(prm.block_start + bb + 1);
+        uint32_t bytes = 0;
+        if (b1 > b0 && b1 <= prm.stream_bytes && !(b0 & 15u)) bytes = (uint32_t)min(b1 - b0, (uint64_t)prm.slot_bytes);
+        bytes &= ~15u;
+        fence_proxy_async();
+        mbar_expect_tx(bar0 + 8u * s, bytes);
+        if (bytes) bulk_load(smem_u32(slots + s * prm.slot_bytes), prm.stream + b0, bytes, bar0 + 8u * s);
+    };
+    if (lane == 0) issue(b, 0);
+
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    for (uint32_t it = 0;; ++it) {
+        const uint32_t s = it & 1u;
+        const uint32_t bn = b + gstride;
+        __syncwarp();  // every lane is done with the other slot
+        if (bn < prm.n_blocks && lane == 0) issue(bn, s ^ 1u);
+        bool ok = mbar_wait(bar0 + 8u * s, (it >> 1) & 1u);
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+            if (lane == 0) {
+                atomicOr(&g_status, ST_TIMEOUT);
+                if (bn < prm.n_blocks) mbar_wait_bounded(bar0 + 8u * (s ^ 1u), ((it + 1) >> 1) & 1u);
+            }
+            return;
+        }
+        const uint64_t b0 = __ldg(prm.block_start + b), b1 = __ldg(prm.block_start + b + 1);
+        const uint64_t i0 = (uint64_t)b * DFW_RANS_BLOCK;
+        const uint32_t cnt = (uint32_t)min((uint64_t)DFW_RANS_BLOCK, prm.n - i0);
+        const bool fits = b1 > b0 && b1 - b0 >= RANS_HEAD && b1 - b0 <= prm.slot_bytes && b1 <= prm.stream_bytes &&
+                          !(b0 & 15u) && !((b1 - b0) & 15u);
+        if (!fits) {
+            if (lane == 0) atomicOr(&g_status, ST_RANGE);
+        } else {
+            const uint32_t sl = smem_u32(slots + s * prm.slot_bytes);
+            const uint32_t words = (uint32_t)(b1 - b0 - RANS_HEAD) / 2u;  // includes the zero padding
+            uint32_t x = lds32(sl + 4u * lane);
+            uint32_t ptr = 0;
+            bool err = false;
+            const uint8_t *mrow = prm.mant + i0;
+            uint16_t *orow = prm.out + i0;
+            const uint32_t steps = (cnt + 31u) / 32u;
+            for (uint32_t k = 0; k < steps; ++k) {
+                const uint32_t i = 32u * k + lane;
+                const bool live = i < cnt;
+                uint32_t e = 0;
+                if (live) {
+                    e = lds32(smem_u32(s_tab) + 4u * (x & (RANS_SLOTS - 1u)));
+                    x = (((e >> 8) & 0xFFFu) + 1u) * (x >> DFW_RANS_SCALE_BITS) + (e >> 20);
+                }
+                const bool need = live && x < 65536u;
+                const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
+                if (need) {
+                    const uint32_t w = ptr + __popc(mask & lt_mask);
+                    uint32_t v = 0;
+                    if (w < words) v = lds16(sl + RANS_HEAD + 2u * w);
+                    else err = true;
+                    x = (x << 16) | v;
+                }
+                ptr += __popc(mask);
+                if (live) orow[i] = join1(rot_sym(e), __ldg(mrow + i));
+            }
+            // integrity: every state back at 2^16, every word used
+            const bool good = __all_sync(0xFFFFFFFFu, !err && x == 65536u) &&
+                              ((RANS_HEAD + 2ull * ptr + 15ull) & ~15ull) == b1 - b0;
+            if (!good && lane == 0) atomicOr(&g_status, ST_COUNT);
+        }
+        if (bn >= prm.n_blocks) break;
+        b = bn;
+    }
+}
+
+struct RansVariant {
+    int nt;
+    void (*fn)(const RansParams);
+    int smem_set[16];
+};
+RansVariant g_rans[] = {
+    {512, rans_decode_kernel<512>, {0}},
+    {256, rans_decode_kernel<256>, {0}},
+    {128, rans_decode_kernel<128>, {0}},
+    {64, rans_decode_kernel<64>, {0}},
+};
+
+}  // namespace
+
+dfw_status launch_rans_decode(const uint8_t *d_stream, const uint8_t *d_mant, const uint64_t *d_block_start,
+                              const dfw_rans_table *t, uint16_t *d_out, cudaStream_t s, int sms) {
+    if (t->max_block_bytes < RANS_HEAD || t->max_block_bytes > 2u * DFW_RANS_BLOCK + RANS_HEAD + 16u ||
+        (t->max_block_bytes & 15u) || t->n_blocks >= (1ull << 32))
+        return DFW_EINVAL;
+    RansParams prm;
+    prm.stream = d_stream;
+    prm.mant = d_mant;
+    prm.block_start = d_block_start;
+    prm.out = d_out;
+    prm.n = t->n;
+    prm.stream_bytes = t->stream_bytes;
+    prm.n_blocks = (uint32_t)t->n_blocks;
+    prm.slot_bytes = t->max_block_bytes;
+    std::memcpy(prm.freq, t->freq, sizeof(prm.freq));
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
+    // the largest CTA whose warps' double-buffered block slots fit (blocks of
+    // incompressible data need 16.5 KB slots)
+    for (RansVariant &v : g_rans) {
+        const uint32_t smem = RANS_TABLE_BYTES + (uint32_t)(v.nt / 32) * (16u + 2u * prm.slot_bytes);
+        if (smem > 227u * 1024u) continue;
+        if (!v.smem_set[dev]) {
+            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+                return DFW_ECUDA;
+            v.smem_set[dev] = 1;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess) return DFW_ECUDA;
+        if (per_sm < 1) continue;
+        const uint64_t wpc = (uint64_t)v.nt / 32;
+        const uint64_t warps = (uint64_t)per_sm * sms * wpc;
+        const uint64_t want = t->n_blocks < warps ? t->n_blocks : warps;
+        v.fn<<<(unsigned)((want + wpc - 1) / wpc), v.nt, smem, s>>>(prm);
+        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+    }
+    return DFW_EINVAL;
+}
+
+
+}  // namespace dfw

@@ -74,6 +74,13 @@ def _load():
         lib.oracle_aux.restype = ctypes.c_int
         lib.oracle_chunk_aux.argtypes = [u8p, u64, u8p, u64, u64, u64, u32p, u64p]
         lib.oracle_chunk_aux.restype = ctypes.c_int
+        lib.oracle_rans_freqs.argtypes = [u64p, ctypes.c_int, u32p]
+        lib.oracle_rans_freqs.restype = ctypes.c_int
+        lib.oracle_rans_encode.argtypes = [u8p, u64, u32p, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint32, u8p, u64,
+                                           u64p, u64p]
+        lib.oracle_rans_encode.restype = ctypes.c_int
+        lib.oracle_rans_decode.argtypes = [u8p, u64p, u64, u32p, ctypes.c_int, ctypes.c_uint32, ctypes.c_uint32, u8p]
+        lib.oracle_rans_decode.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -258,3 +265,69 @@ def gemv_abs(w, rows: int, cols: int, x) -> np.ndarray:
     any fp32 summation of the products."""
     W = np.abs(bf16_values(w).reshape(rows, cols))
     return W @ np.abs(bf16_values(x))
+
+
+# ---------------------------------------------------------------- rANS variant
+
+RANS_SCALE_BITS = 12
+RANS_LANES = 32
+RANS_BLOCK = 8192
+
+
+def rans_freqs(hist, scale_bits: int = RANS_SCALE_BITS) -> np.ndarray:
+    """Quantised frequencies summing to 2^scale_bits (reading R9 of oracle.c)."""
+    h = np.ascontiguousarray(hist, dtype=np.uint64)
+    f = np.zeros(256, np.uint32)
+    _check(_load().oracle_rans_freqs(_p(h, ctypes.c_uint64), scale_bits, _p(f, ctypes.c_uint32)), "rans_freqs")
+    return f
+
+
+class RansEncoded:
+    """The oracle's rANS encoding: stream bytes, block byte offsets, the
+    quantised frequencies, the raw bytes and the coding parameters."""
+
+    def __init__(self, stream, block_start, freq, mant, n, scale_bits, lanes, block_syms):
+        self.stream, self.block_start, self.freq, self.mant = stream, block_start, freq, mant
+        self.n, self.scale_bits, self.lanes, self.block_syms = n, scale_bits, lanes, block_syms
+
+
+def rans_encode_symbols(e, freq, scale_bits=RANS_SCALE_BITS, lanes=RANS_LANES, block_syms=RANS_BLOCK):
+    e = np.ascontiguousarray(e, dtype=np.uint8)
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    n = e.size
+    n_blocks = (n + block_syms - 1) // block_syms
+    cap = 2 * n + n_blocks * (4 * lanes + 16) + 16
+    out = np.zeros(cap, np.uint8)
+    starts = np.zeros(n_blocks + 1, np.uint64)
+    nb = np.zeros(1, np.uint64)
+    _check(_load().oracle_rans_encode(_p(e if n else np.zeros(1, np.uint8), ctypes.c_uint8), n,
+                                      _p(freq, ctypes.c_uint32), scale_bits, lanes, block_syms,
+                                      _p(out, ctypes.c_uint8), cap, _p(starts, ctypes.c_uint64),
+                                      _p(nb, ctypes.c_uint64)), "rans_encode")
+    return out[: int(nb[0])].copy(), starts
+
+
+def rans_decode_symbols(stream, block_start, n, freq, scale_bits=RANS_SCALE_BITS, lanes=RANS_LANES,
+                        block_syms=RANS_BLOCK):
+    e = np.zeros(max(n, 1), np.uint8)
+    stream = np.ascontiguousarray(stream if len(stream) else np.zeros(1, np.uint8), dtype=np.uint8)
+    starts = np.ascontiguousarray(block_start, dtype=np.uint64)
+    freq = np.ascontiguousarray(freq, dtype=np.uint32)
+    rc = _load().oracle_rans_decode(_p(stream, ctypes.c_uint8), _p(starts, ctypes.c_uint64), n,
+                                    _p(freq, ctypes.c_uint32), scale_bits, lanes, block_syms, _p(e, ctypes.c_uint8))
+    return int(rc), e[:n]
+
+
+def rans_encode(u, scale_bits=RANS_SCALE_BITS, lanes=RANS_LANES, block_syms=RANS_BLOCK) -> RansEncoded:
+    e, m = split(u)
+    freq = rans_freqs(histogram(e), scale_bits)
+    stream, starts = rans_encode_symbols(e, freq, scale_bits, lanes, block_syms)
+    return RansEncoded(stream, starts, freq, m, e.size, scale_bits, lanes, block_syms)
+
+
+def rans_decode(enc: RansEncoded) -> np.ndarray:
+    rc, e = rans_decode_symbols(enc.stream, enc.block_start, enc.n, enc.freq, enc.scale_bits, enc.lanes,
+                                enc.block_syms)
+    _check(rc, "rans_decode")
+    return (((enc.mant.astype(np.uint16) & 0x80) << 8) | (e.astype(np.uint16) << 7)
+            | (enc.mant.astype(np.uint16) & 0x7F)).astype(np.uint16)

@@ -404,3 +404,210 @@ int oracle_chunk_aux(const uint8_t *stream, uint64_t total_bits, const uint8_t l
     group_start[n_groups] = total_bits;
     return OR_OK;
 }
+
+/* ======================================================================
+ * rANS variant of the exponent coder (the ANS "bridge" of the ~1.5:1 page's
+ * abstract; the LazyWeights write-up compares Huffman with rANS).  The pages
+ * give no format; the readings taken here:
+ *   R8  range ANS (Duda, "Asymmetric numeral systems", 2013) with a state x
+ *       in [L, L * 2^16), L = 2^16, renormalised 16 bits at a time;
+ *       symbol s with quantised frequency f_s and cumulative start c_s
+ *       (sum of f over smaller symbols; the f_s sum to M = 2^scale_bits)
+ *       encodes as x' = floor(x / f_s) * M + (x mod f_s) + c_s, after
+ *       emitting the low 16 bits of x while x >= f_s * (L / M) * 2^16;
+ *       decoding inverts it: slot = x mod M, s is the symbol whose
+ *       [c_s, c_s + f_s) holds slot, x = f_s * floor(x / M) + slot - c_s,
+ *       then while x < L: x = x * 2^16 + next word.
+ *   R9  frequencies: f_s = max(1, floor(count_s * M / n)) for every present
+ *       symbol, 0 for absent ones; the remainder M - sum f goes to the most
+ *       frequent symbol (smallest symbol on ties) if positive; if negative,
+ *       1 is taken repeatedly from the symbol with the largest f_s > 1
+ *       (smallest symbol on ties).
+ *   R10 interleaving: the symbols are cut into blocks of block_syms; in a
+ *       block, symbol i belongs to state i mod I (I states, "lanes").  The
+ *       encoder walks the block backwards (i = last .. 0), so that a decoder
+ *       taking steps k = 0, 1, ... decodes symbols I k .. I k + I - 1 (one
+ *       per state) and then renormalises the states in increasing state
+ *       order, each taking the next word of the block.  A block is: I final
+ *       encoder states (u32, little-endian), its words in decode order (u16,
+ *       little-endian), zero padding to a multiple of 16 bytes.  Every state
+ *       starts at L, so a decoder must end with every state at L and every
+ *       word consumed.
+ * ====================================================================== */
+
+#define RANS_L 65536u
+
+int oracle_rans_freqs(const uint64_t hist[256], int scale_bits, uint32_t freq[256])
+{
+    if (scale_bits < 8 || scale_bits > 16)
+        return OR_EINVAL;
+    const uint64_t M = 1ull << scale_bits;
+    uint64_t n = 0;
+    for (int s = 0; s < 256; s++)
+        n += hist[s];
+    for (int s = 0; s < 256; s++)
+        freq[s] = 0;
+    if (n == 0)
+        return OR_OK;
+    int64_t sum = 0;
+    for (int s = 0; s < 256; s++) {
+        if (!hist[s])
+            continue;
+        /* floor(count * M / n) without overflow: count <= n < 2^64, M <= 2^16 */
+        const unsigned __int128 q = ((unsigned __int128)hist[s] * M) / n;
+        freq[s] = q ? (uint32_t)q : 1u;
+        sum += freq[s];
+    }
+    int64_t d = (int64_t)M - sum;
+    if (d > 0) {
+        int best = -1;
+        for (int s = 0; s < 256; s++)
+            if (hist[s] && (best < 0 || hist[s] > hist[best]))
+                best = s;
+        freq[best] += (uint32_t)d;
+    }
+    while (d < 0) {
+        int best = -1;
+        for (int s = 0; s < 256; s++)
+            if (freq[s] > 1 && (best < 0 || freq[s] > freq[best]))
+                best = s;
+        if (best < 0)
+            return OR_EINVAL; /* more symbols than M slots */
+        freq[best]--;
+        d++;
+    }
+    return OR_OK;
+}
+
+static void rans_cum(const uint32_t freq[256], uint32_t cum[257])
+{
+    cum[0] = 0;
+    for (int s = 0; s < 256; s++)
+        cum[s + 1] = cum[s] + freq[s];
+}
+
+/* Bytes of one block's encoding for `lanes` states and `words` words. */
+static uint64_t rans_block_bytes(uint32_t lanes, uint64_t words)
+{
+    return (4ull * lanes + 2ull * words + 15) & ~15ull;
+}
+
+/* Encodes exponent symbols e[0..n) (every symbol must have freq > 0).
+ * block_start receives n_blocks + 1 byte offsets. */
+int oracle_rans_encode(const uint8_t *e, uint64_t n, const uint32_t freq[256], int scale_bits,
+                       uint32_t lanes, uint32_t block_syms, uint8_t *out, uint64_t out_cap,
+                       uint64_t *block_start, uint64_t *out_bytes)
+{
+    if (lanes < 1 || lanes > 64 || block_syms < lanes || block_syms % lanes || scale_bits < 8 ||
+        scale_bits > 16)
+        return OR_EINVAL;
+    uint32_t cum[257];
+    rans_cum(freq, cum);
+    if (n && cum[256] != (1u << scale_bits))
+        return OR_EINVAL;
+    const uint64_t n_blocks = (n + block_syms - 1) / block_syms;
+    uint16_t *stack = (uint16_t *)malloc(sizeof(uint16_t) * (block_syms + 1));
+    if (!stack)
+        return OR_ENOMEM;
+    uint64_t pos = 0;
+    for (uint64_t b = 0; b < n_blocks; b++) {
+        block_start[b] = pos;
+        const uint64_t i0 = b * block_syms;
+        const uint64_t cnt = n - i0 < block_syms ? n - i0 : block_syms;
+        uint32_t x[64];
+        for (uint32_t j = 0; j < lanes; j++)
+            x[j] = RANS_L;
+        uint64_t words = 0;
+        for (uint64_t ii = cnt; ii-- > 0;) {
+            const uint32_t j = (uint32_t)(ii % lanes);
+            const uint8_t s = e[i0 + ii];
+            const uint32_t f = freq[s];
+            if (f == 0) {
+                free(stack);
+                return OR_EINVAL;
+            }
+            const uint64_t x_max = ((uint64_t)(RANS_L >> scale_bits) << 16) * f;
+            if (x[j] >= x_max) {
+                stack[words++] = (uint16_t)(x[j] & 0xFFFFu);
+                x[j] >>= 16;
+            }
+            x[j] = ((x[j] / f) << scale_bits) + (x[j] % f) + cum[s];
+        }
+        const uint64_t bytes = rans_block_bytes(lanes, words);
+        if (pos + bytes > out_cap) {
+            free(stack);
+            return OR_ENOMEM;
+        }
+        uint8_t *p = out + pos;
+        memset(p, 0, bytes);
+        for (uint32_t j = 0; j < lanes; j++)
+            for (int k = 0; k < 4; k++)
+                p[4 * j + k] = (uint8_t)(x[j] >> (8 * k));
+        for (uint64_t w = 0; w < words; w++) { /* decode order = reverse of emission */
+            const uint16_t v = stack[words - 1 - w];
+            p[4 * lanes + 2 * w] = (uint8_t)(v & 0xFF);
+            p[4 * lanes + 2 * w + 1] = (uint8_t)(v >> 8);
+        }
+        pos += bytes;
+    }
+    block_start[n_blocks] = pos;
+    *out_bytes = pos;
+    free(stack);
+    return OR_OK;
+}
+
+/* Decodes n symbols; OR_ECORRUPT if a block does not end with every state at
+ * L and every word consumed, or reads past its end. */
+int oracle_rans_decode(const uint8_t *stream, const uint64_t *block_start, uint64_t n,
+                       const uint32_t freq[256], int scale_bits, uint32_t lanes, uint32_t block_syms,
+                       uint8_t *e)
+{
+    if (lanes < 1 || lanes > 64 || block_syms < lanes || block_syms % lanes || scale_bits < 8 ||
+        scale_bits > 16)
+        return OR_EINVAL;
+    uint32_t cum[257];
+    rans_cum(freq, cum);
+    const uint32_t M = 1u << scale_bits;
+    if (n && cum[256] != M)
+        return OR_EINVAL;
+    const uint64_t n_blocks = (n + block_syms - 1) / block_syms;
+    for (uint64_t b = 0; b < n_blocks; b++) {
+        const uint8_t *p = stream + block_start[b];
+        const uint64_t bytes = block_start[b + 1] - block_start[b];
+        if (bytes < 4ull * lanes)
+            return OR_ECORRUPT;
+        const uint64_t max_words = (bytes - 4ull * lanes) / 2;
+        const uint64_t i0 = b * block_syms;
+        const uint64_t cnt = n - i0 < block_syms ? n - i0 : block_syms;
+        uint32_t x[64];
+        for (uint32_t j = 0; j < lanes; j++)
+            x[j] = (uint32_t)p[4 * j] | ((uint32_t)p[4 * j + 1] << 8) | ((uint32_t)p[4 * j + 2] << 16) |
+                   ((uint32_t)p[4 * j + 3] << 24);
+        uint64_t w = 0;
+        for (uint64_t k = 0; k * lanes < cnt; k++) {
+            for (uint32_t j = 0; j < lanes && k * lanes + j < cnt; j++) {
+                const uint32_t slot = x[j] & (M - 1);
+                int s = 0;
+                while (!(cum[s] <= slot && slot < cum[s + 1]))
+                    s++;
+                e[i0 + k * lanes + j] = (uint8_t)s;
+                x[j] = freq[s] * (x[j] >> scale_bits) + slot - cum[s];
+            }
+            for (uint32_t j = 0; j < lanes && k * lanes + j < cnt; j++) {
+                if (x[j] < RANS_L) {
+                    if (w >= max_words)
+                        return OR_ECORRUPT;
+                    const uint32_t v = (uint32_t)p[4 * lanes + 2 * w] | ((uint32_t)p[4 * lanes + 2 * w + 1] << 8);
+                    x[j] = (x[j] << 16) | v;
+                    w++;
+                }
+            }
+        }
+        for (uint32_t j = 0; j < lanes; j++)
+            if (x[j] != RANS_L)
+                return OR_ECORRUPT;
+        if (rans_block_bytes(lanes, w) != bytes)
+            return OR_ECORRUPT;
+    }
+    return OR_OK;
+}

@@ -365,3 +365,38 @@ def test_plan_lanes_detects_corrupt_stream():
     with pytest.raises(dfw.DfwError) as ei:
         dfw.plan_lanes(bad)
     assert ei.value.status in (dfw.ECORRUPT, dfw.EINVAL)
+
+
+# ---------------------------------------------------------------- rANS variant
+
+def _rans_u16(name):
+    if name == "edge":
+        return np.random.default_rng(3).integers(0, 65536, size=70_001, dtype=np.uint64).astype(np.uint16)
+    if name == "one":
+        return np.full(33_333, 0x3F80, np.uint16)
+    block = {"c1": workloads.c1(), "c2": workloads.c2(), "c3": workloads.c3(), "c4a": workloads.c4("a"),
+             "c4b": workloads.c4("b"), "c4c": workloads.c4("c")}[name]
+    return np.concatenate([workloads.as_u16_numpy(t)
+                           for t in workloads.generate_block(workloads.scaled(block, 300_007))])
+
+
+@pytest.mark.parametrize("name", ["c1", "c2", "c3", "c4a", "c4b", "c4c", "edge", "one"])
+def test_rans_encoder_bytes_equal_oracle(oracle, name):
+    u = _rans_u16(name)
+    oenc = oracle.rans_encode(u, 12, 32, 16384)
+    for nt in (1, 3):
+        enc = dfw.rans_encode(torch.from_numpy(u.view(np.int16)), n_threads=nt)
+        used = int(enc.table.stream_bytes)
+        assert np.array_equal(enc.stream.numpy()[:used], oenc.stream)
+        assert np.array_equal(enc.block_start.numpy().view(np.uint64), oenc.block_start)
+        assert np.array_equal(np.frombuffer(bytes(enc.table.freq), np.uint16).astype(np.uint32), oenc.freq)
+        assert np.array_equal(enc.mant.numpy()[: u.size], oenc.mant)
+        assert enc.table.max_block_bytes == int(np.diff(oenc.block_start.astype(np.int64)).max())
+
+
+def test_rans_encode_multi_equals_concatenation(oracle):
+    a, b = _rans_u16("c1")[:40_000], _rans_u16("c2")[:30_001]
+    enc = dfw.rans_encode([torch.from_numpy(a.view(np.int16)), torch.from_numpy(b.view(np.int16))])
+    oenc = oracle.rans_encode(np.concatenate([a, b]), 12, 32, 16384)
+    assert np.array_equal(enc.stream.numpy()[: int(enc.table.stream_bytes)], oenc.stream)
+    assert enc.tensor_offsets.tolist() == [0, 40_000, 70_001]

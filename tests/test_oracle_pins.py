@@ -586,3 +586,99 @@ def test_gemv_against_exact_rationals(oracle):
     for i in range(rows):
         exact = sum(Fraction(float(wv[i, j])) * Fraction(float(xv[j])) for j in range(cols))
         assert abs(Fraction(float(y[i])) - exact) <= Fraction(cols * 2.0 ** -53) * Fraction(float(scale[i]))
+
+
+# ---------------------------------------------------------------- rANS variant
+
+def test_rans_hand_worked(oracle):
+    kv = dict(line.split(":", 1) for line in open(os.path.join(GOLDEN, "rans_tiny.txt"))
+              if ":" in line and not line.startswith("#"))
+    freq = np.zeros(256, np.uint32)
+    freq[0], freq[1] = int(kv["freq0"]), int(kv["freq1"])
+    e = np.array([int(v) for v in kv["symbols"].split()], np.uint8)
+    stream, starts = oracle.rans_encode_symbols(e, freq, int(kv["scale_bits"]), int(kv["lanes"]), 16)
+    want = np.array([int(b, 16) for b in kv["stream"].split()], np.uint8)
+    assert np.array_equal(stream, want) and starts.tolist() == [0, 16]
+    assert int(stream[:4].view(np.uint32)[0]) == int(kv["final_state"])
+    rc, back = oracle.rans_decode_symbols(stream, starts, 2, freq, 8, 1, 16)
+    assert rc == 0 and back.tolist() == [0, 1]
+
+
+def test_rans_freqs_rules(oracle):
+    h = np.zeros(256, np.uint64)
+    h[[3, 9]] = [3000, 1000]  # proportional: exactly 3/4 and 1/4 of 4096
+    f = oracle.rans_freqs(h, 12)
+    assert f[3] == 3072 and f[9] == 1024 and f.sum() == 4096 and np.count_nonzero(f) == 2
+    h = np.zeros(256, np.uint64)
+    h[[0, 1, 2]] = [1, 1, 1]  # floors 1365 each, remainder 1 to the smallest of the tied most frequent
+    f = oracle.rans_freqs(h, 12)
+    assert f[:3].tolist() == [1366, 1365, 1365]
+    h = np.zeros(256, np.uint64)
+    h[0], h[1:201] = 10 ** 9, 1  # 200 rare symbols bumped to 1: the excess comes off the largest
+    f = oracle.rans_freqs(h, 8)
+    assert f.sum() == 256 and (f[1:201] == 1).all() and f[0] == 56 and not f[201:].any()
+    h = np.zeros(256, np.uint64)
+    h[77] = 5
+    assert oracle.rans_freqs(h, 12)[77] == 4096
+
+
+def test_rans_single_symbol_closed_form(oracle):
+    e = np.full(5000, 77, np.uint8)
+    freq = np.zeros(256, np.uint32)
+    freq[77] = 4096
+    stream, starts = oracle.rans_encode_symbols(e, freq, 12, 32, 4096)
+    # every state stays at 65536 and no word is written: 2 blocks of 128 bytes
+    assert starts.tolist() == [0, 128, 256]
+    assert (stream.view(np.uint32) == 65536).all()
+
+
+def test_rans_lanes_are_independent_coders(oracle):
+    """With 32 interleaved states, the final state of lane j equals that of
+    a one-state encoding of every 32nd exponent starting at j."""
+    rng = np.random.default_rng(12)
+    e = rng.choice(np.arange(6, dtype=np.uint8), size=4096, p=[0.4, 0.3, 0.15, 0.1, 0.04, 0.01])
+    freq = oracle.rans_freqs(oracle.histogram(e), 12)
+    stream, starts = oracle.rans_encode_symbols(e, freq, 12, 32, 4096)
+    states = stream[:128].view(np.uint32)
+    for j in (0, 1, 17, 31):
+        s1, _ = oracle.rans_encode_symbols(e[j::32], freq, 12, 1, 128)
+        assert int(s1[:4].view(np.uint32)[0]) == int(states[j])
+
+
+def test_rans_rate_within_information_bounds(oracle):
+    """Per lane, 16 (words) + log2(final state) - 16 is the information
+    sum_i log2(M / f_i) of its exponents up to a rounding term of at most
+    log2(1 / (1 - 2^-4)) < 0.1 bits per exponent (x >= 2^16 while f <= M)."""
+    rng = np.random.default_rng(13)
+    e = rng.choice(np.arange(5, dtype=np.uint8), size=32 * 2000, p=[0.5, 0.25, 0.15, 0.07, 0.03])
+    freq = oracle.rans_freqs(oracle.histogram(e), 12)
+    stream, starts = oracle.rans_encode_symbols(e, freq, 12, 32, e.size)
+    info = np.log2(4096.0 / freq[e].astype(np.float64))
+    words = (stream.size - 128) // 2  # padding < 16 bytes: at most 7 words of zeros
+    total = 16 * words + np.log2(stream[:128].view(np.uint32).astype(np.float64)).sum() - 16 * 32
+    assert info.sum() - 1.0 <= total <= info.sum() + 0.1 * e.size + 16 * 8
+
+
+def _rans_case(name: str) -> np.ndarray:
+    if name == "tiny":
+        return np.array([0x3F80, 0x3F80, 0xBF00, 0x0001, 0x7F80, 0x3F80, 0xC000], np.uint16)
+    block = {"c1": workloads.c1(), "c4a": workloads.c4("a"), "c4b": workloads.c4("b"),
+             "c4c": workloads.c4("c")}[name]
+    return np.concatenate([workloads.as_u16_numpy(t) for t in workloads.generate_block(workloads.scaled(block, 60_003))])
+
+
+@pytest.mark.parametrize("name", ["c1", "c4a", "c4b", "c4c", "tiny"])
+@pytest.mark.parametrize("lanes,block", [(32, 16384), (32, 8192), (1, 64), (8, 4096)])
+def test_rans_roundtrip(oracle, name, lanes, block):
+    u = _rans_case(name)
+    enc = oracle.rans_encode(u, 12, lanes, block)
+    assert np.array_equal(oracle.rans_decode(enc), u)
+
+
+def test_rans_corrupt_state_detected(oracle):
+    u = _rans_case("c1")[:50_000]
+    enc = oracle.rans_encode(u)
+    bad = enc.stream.copy()
+    bad[4 * 5] ^= 0x40  # a bit of state 5 of block 0
+    rc, _ = oracle.rans_decode_symbols(bad, enc.block_start, enc.n, enc.freq)
+    assert rc == oracle.ECORRUPT
