@@ -520,6 +520,75 @@ def run_gemv_mode(args, rank, world, blocks, wdesc, device):
     return 0 if ok else 1
 
 
+# ------------------------------------------------------------------ rans mode
+
+def run_rans_mode(args, rank, world, blocks, wdesc, device):
+    """The rANS variant against the Huffman known-start plan on the same
+    weights, in the same run: compressed size (with and without aux) and
+    decode time of every scope into the scratch buffer."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    devs_h, _ = prepare(blocks, device, args.window, args.tile, args.threads, "lanes")
+    devs_r = []
+    for b in blocks:
+        ts = [t.cpu() for t in workloads.generate_block(b, device)]
+        devs_r.append(dfw.DeviceRans.upload(dfw.rans_encode(ts), device))
+    torch.cuda.synchronize(device)
+    torch.cuda.empty_cache()
+    nmax = max(d.n for d in devs_h)
+    scratch = torch.empty(nmax, dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def timed(step):
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1) / args.steps)
+
+    sampler = ClockSampler(int(device.index or 0))
+    sampler.start()
+    ms_r = timed(lambda: [dfw.rans_decode(d, scratch, stream=stream) for d in devs_r])
+    clocks = sampler.stop()
+    ms_h = timed(lambda: [dfw.decode_lanes(d, scratch, stream=stream) for d in devs_h])
+    ok = dfw.check_status(stream) == dfw.OK
+    for b, d in zip(blocks, devs_r):  # every scope decodes back to its input
+        dfw.rans_decode(d, scratch, stream=stream)
+        ref = torch.cat([t.reshape(-1) for t in workloads.generate_block(b, device)])
+        ok = ok and dfw.check_status(stream) == dfw.OK and torch.equal(scratch[: d.n].view(torch.int16),
+                                                                      ref.view(torch.int16))
+    n_total = sum(d.n for d in devs_r)
+    bits = lambda devs, aux: 8 * sum(d.compressed_bytes(with_aux=aux) for d in devs) / n_total  # noqa: E731
+    alg = sum(d.algorithmic_bytes() for d in devs_r)
+    peak, peak_kind = measured_peak_hbm()
+    achieved = alg / (ms_r * 1e-3) / 1e9
+    line = {
+        "metric": "decoded bf16 weights/sec with the rANS variant (beside the Huffman plan on the same weights)",
+        "value": world * n_total / (ms_r * 1e-3), "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_r, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+        "config": {"workload": wdesc, "weights": n_total, "code_tables": len(devs_r), "mode": "rans",
+                   "rans": "2^12 frequencies, 32 interleaved 32-bit states, blocks of 16384",
+                   "l2": "inputs larger than L2", "parallelism": f"replica{world}" if world > 1 else "single GPU"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "peak_source": peak_kind, "kernel": "rans_decode_kernel",
+                     "algorithmic_bytes_per_step": alg},
+        "rate_bits_per_weight": {"rans": bits(devs_r, True), "rans_no_aux": bits(devs_r, False),
+                                 "huffman_lanes": bits(devs_h, True), "huffman_no_aux": bits(devs_h, False)},
+        "huffman_lanes_ms_per_step": ms_h,
+        "clocks": clocks, "gpu_launches": args.steps * len(devs_r), "verified_bit_exact": bool(ok),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0 if ok else 1
+
+
 # ------------------------------------------------------------------ main
 
 def main(argv=None):
@@ -538,9 +607,9 @@ def main(argv=None):
     ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv"],
+    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv", "rans"],
                     help="decode: the decode path (default); encode: the GPU encoder; "
-                         "gemv: decode fused with y = W x")
+                         "gemv: decode fused with y = W x; rans: the rANS variant beside Huffman")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -564,8 +633,8 @@ def main(argv=None):
     import lossless_entropy_coded_canonical_b200 as dfw
     dfw.lib()
     dfw.check()
-    if args.mode in ("encode", "gemv"):
-        run = run_encode_mode if args.mode == "encode" else run_gemv_mode
+    if args.mode in ("encode", "gemv", "rans"):
+        run = {"encode": run_encode_mode, "gemv": run_gemv_mode, "rans": run_rans_mode}[args.mode]
         rc = run(args, rank, world, blocks, wdesc, device)
         if world > 1:
             dist.destroy_process_group()

@@ -104,6 +104,20 @@ __device__ __forceinline__ uint32_t lds16(uint32_t a) {
     asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
     return v;
 }
+// A 16-bit shared load only where p holds (0 elsewhere), without a branch.
+__device__ __forceinline__ uint32_t lds16_if(bool p, uint32_t a) {
+    uint32_t v = 0;
+    asm volatile(
+        "{\n\t.reg .pred q;\n\t.reg .b16 h;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "mov.b16 h, 0;\n\t"
+        "@q ld.shared.u16 h, [%2];\n\t"
+        "cvt.u32.u16 %0, h;\n\t}"
+        : "+r"(v)
+        : "r"((uint32_t)p), "r"(a)
+        : "memory");
+    return v;
+}
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");

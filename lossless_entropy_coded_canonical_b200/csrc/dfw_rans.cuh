@@ -9,7 +9,9 @@
 // exponent of its state, the warp ballots which states fell below 2^16, each
 // of those takes the word at (next word + its rank among them), and the
 // lane joins its exponent with the raw byte into bf16 (one 2-byte store per
-// lane: 64 contiguous bytes per warp).  A block must end with every state at
+// lane: 64 contiguous bytes per warp).  Raw bytes arrive 4 per lane in
+// coalesced 128-byte rows, three rows (12 steps) ahead of use, and reach
+// the lane that needs them by shuffle.  A block must end with every state at
 // 2^16 and every word used; otherwise the status word records it.
 #pragma once
 
@@ -27,7 +29,7 @@ struct RansParams {
     const uint8_t *mant;
     const uint64_t *block_start;
     uint16_t *out;
-    uint64_t n, stream_bytes;
+    uint64_t n, stream_bytes, mant_bytes;
     uint32_t n_blocks, slot_bytes;
     uint16_t freq[256];
 };
@@ -112,28 +114,49 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
             uint32_t x = lds32(sl + 4u * lane);
             uint32_t ptr = 0;
             bool err = false;
+            // raw bytes: lane l loads the 4 bytes at 128 q + 4 l of the block
+            // (coalesced), three quads ahead; step 4 q + t takes its byte from
+            // lane 8 t + l / 4 by shuffle
             const uint8_t *mrow = prm.mant + i0;
-            uint16_t *orow = prm.out + i0;
-            const uint32_t steps = (cnt + 31u) / 32u;
-            for (uint32_t k = 0; k < steps; ++k) {
-                const uint32_t i = 32u * k + lane;
-                const bool live = i < cnt;
-                uint32_t e = 0;
-                if (live) {
-                    e = lds32(smem_u32(s_tab) + 4u * (x & (RANS_SLOTS - 1u)));
-                    x = (((e >> 8) & 0xFFFu) + 1u) * (x >> DFW_RANS_SCALE_BITS) + (e >> 20);
-                }
-                const bool need = live && x < 65536u;
-                const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
-                if (need) {
+            const uint32_t mlim = (uint32_t)min((uint64_t)DFW_RANS_BLOCK, prm.mant_bytes - i0);
+            auto mload = [&](uint32_t q) -> uint32_t {
+                const uint32_t o = 128u * q + 4u * lane;
+                return o + 4u <= mlim ? __ldg(reinterpret_cast<const uint32_t *>(mrow + o)) : 0u;
+            };
+            uint32_t m1 = mload(0), m2 = mload(1), m3 = mload(2);
+            uint16_t *op = prm.out + i0 + lane;
+            const uint32_t quads = (cnt + 127u) / 128u;
+            const uint32_t tab = smem_u32(s_tab), wbase = sl + RANS_HEAD;
+            const bool whole = cnt == DFW_RANS_BLOCK;  // every block but possibly the scope's last
+            for (uint32_t q = 0; q < quads; ++q) {
+                const uint32_t mc = m1;
+                m1 = m2;
+                m2 = m3;
+                m3 = mload(q + 3u);
+#pragma unroll
+                for (uint32_t t = 0; t < 4; ++t) {
+                    const uint32_t i = 128u * q + 32u * t + lane;
+                    const bool live = whole || i < cnt;
+                    const uint32_t e = lds32(tab + 4u * (x & (RANS_SLOTS - 1u)));
+                    const uint32_t xd = (((e >> 8) & 0xFFFu) + 1u) * (x >> DFW_RANS_SCALE_BITS) + (e >> 20);
+                    x = live ? xd : x;
+                    const bool need = live && x < 65536u;
+                    const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
                     const uint32_t w = ptr + __popc(mask & lt_mask);
-                    uint32_t v = 0;
-                    if (w < words) v = lds16(sl + RANS_HEAD + 2u * w);
-                    else err = true;
-                    x = (x << 16) | v;
+                    const bool rd = need && w < words;
+                    err |= need && !rd;
+                    const uint32_t v = lds16_if(rd, wbase + 2u * w);  // branch-free reload
+                    x = need ? (x << 16) | v : x;
+                    ptr += __popc(mask);
+                    const uint32_t mb = __byte_perm(__shfl_sync(0xFFFFFFFFu, mc, 8u * t + (lane >> 2)), 0u,
+                                                    0x4440u | (lane & 3u));
+                    // bf16 = sign << 15 | exponent << 7 | mantissa: the raw
+                    // byte doubled into both halves keeps its sign at bit 15
+                    // and its mantissa at bits 6..0; the table entry's low
+                    // byte is the exponent
+                    if (live) op[32u * t] = (uint16_t)(((mb * 0x101u) & 0x807Fu) | ((e << 7) & 0x7F80u));
                 }
-                ptr += __popc(mask);
-                if (live) orow[i] = join1(rot_sym(e), __ldg(mrow + i));
+                op += 128;
             }
             // integrity: every state back at 2^16, every word used
             const bool good = __all_sync(0xFFFFFFFFu, !err && x == 65536u) &&
@@ -171,6 +194,7 @@ dfw_status launch_rans_decode(const uint8_t *d_stream, const uint8_t *d_mant, co
     prm.out = d_out;
     prm.n = t->n;
     prm.stream_bytes = t->stream_bytes;
+    prm.mant_bytes = (t->n + 15) & ~15ull;
     prm.n_blocks = (uint32_t)t->n_blocks;
     prm.slot_bytes = t->max_block_bytes;
     std::memcpy(prm.freq, t->freq, sizeof(prm.freq));
