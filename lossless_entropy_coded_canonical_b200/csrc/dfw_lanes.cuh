@@ -12,14 +12,14 @@
 //     warp's raw-byte buffer (started as soon as the previous group's join
 //     has read that buffer);
 //   - each lane finds its chunk's first bit with a warp prefix sum of
-//     chunk_bits and decodes exactly its 64 codewords with the fast table
-//     (up to four codewords per lookup) into its own word slots, interleaved
-//     by lane so stores never conflict;
-//   - each lane joins exponents and raw bytes into bf16, 16 at a time in a
-//     lane-rotated order (which spreads the 128-bit shared reads over the
-//     banks), and stores its chunk's 128 output bytes straight from
-//     registers, one whole 32-byte sector per 256-bit store (two 128-bit
-//     stores when the output is only 16-byte aligned); no staging buffer is
+//     chunk_bits and decodes its 64 codewords with the fast table (up to
+//     four codewords per lookup) into its own word slots, one row per word
+//     index, the 32 lanes side by side;
+//   - the warp then joins exponents and raw bytes into bf16 with the lanes
+//     reassigned: in store j lane l joins piece l & 3 (16 weights) of chunk
+//     8 j + l / 4 and writes it with one 256-bit store, so each store
+//     instruction covers 1 KB of contiguous output (two 128-bit stores per
+//     lane when the output is only 16-byte aligned); no staging buffer is
 //     needed, which leaves shared memory for up to 32 warps per SM.
 // No count phase, no block scan, no CTA barrier after the table load, and no
 // realignment: every chunk's output is 64-weight aligned.
@@ -39,6 +39,16 @@ namespace dfw {
 namespace {
 
 constexpr uint32_t EXP_WORDS = 17;        // a chunk's 64 exponent bytes + up to 3 more from the last lookup
+// Word k of the exponent slots of chunk c (0..31 within its group) lives at
+// EXP_STRIDE * k + 4 c: one row per word index, 34 words wide, so the word is
+// in bank (2 k + c) mod 32.  A lane appending to its own chunk moves down
+// one row per word; the join reads words 4 i .. 4 i + 3 of eight chunks in
+// four pieces i at once, which the two-bank step per row spreads over all 32
+// banks.
+constexpr uint32_t EXP_STRIDE = 136;
+// The slots' area, rounded up to 16 bytes so every warp's area (and the bulk
+// copies and 128-bit loads into it) stays 16-byte aligned.
+constexpr uint32_t EXP_BYTES = (EXP_WORDS * EXP_STRIDE + 15u) & ~15u;
 constexpr uint32_t GROUP_SYMS = LANE_SYMS * GROUP_CHUNKS;  // 2048 weights per warp group
 
 struct LanesParams {
@@ -61,19 +71,31 @@ __device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_
     return (uint32_t)(b1 - b0);
 }
 
+// In shared memory the lanes kernel keeps a fast entry's second word as in
+// the LUT image (byte 0 bits used, byte 1 eight times the count, bits 16..27
+// the end mask) except for escapes, which become LANES_ESC_WORD: no bits, no
+// symbols, and the top bit, which the loop's byte permute spreads over bytes
+// 1 and 2 so an escape subtracts LANES_ESC_DEC from the count and leaves the
+// loop through its ordinary end test.
+constexpr uint32_t LANES_ESC_WORD = 0x80000000u;
+constexpr int LANES_ESC_DEC = 0x00FFFF00;
+
 // Decodes `left8 / 8` codewords starting at bit r of the stream words held in
-// shared memory at sw (32-bit shared address) and appends
-// their symbols to this lane's word slots ep, ep + 128, ... (slots of the 32
-// lanes interleave; a last lookup may append up to three more symbols, which
-// are never read).  fast is the shared address of the
-// fast table.  Returns the stream bit position (relative to sw) after the
-// last codeword decoded.
+// shared memory at sw (32-bit shared address) and appends their symbols to
+// this lane's word slots ep, ep + EXP_STRIDE, ... (slots of the 32 lanes
+// interleave).  fast is the shared address of the fast table.  Returns the
+// stream bit position (relative to sw) after codeword left8 / 8.
 //
-// The inner loop is straight-line code: it keeps the word after the current
-// pair in a register, moves it in (predicated) when the position crosses a
-// word and only then loads the next one; it always stores the accumulator's
-// low word and moves to the next slot when the word is full.  Only an escape
-// or the chunk's last lookup leaves it, for one step of the general path.
+// The inner loop is straight-line code that runs until the chunk's count is
+// reached: the last lookup may decode up to three codewords of the next
+// chunk, whose symbols land in slack slots that are never read, and the exact
+// end is worked out once afterwards from that lookup's end mask.  So a lane
+// that finishes early has nothing left to do but wait for the others.  The
+// loop keeps the word after the current pair in a register, moves it in
+// (predicated) when the position crosses a word and only then loads the next
+// one; it always stores the accumulator's low word and moves to the next slot
+// when the word is full.  Only an escape (a codeword longer than the fast
+// key) leaves it early.
 __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int left8, uint32_t fast,
                                                  uint32_t kshift, const uint32_t *__restrict__ g_hier,
                                                  uint32_t n_tables, uint32_t ep, uint32_t &err) {
@@ -90,68 +112,86 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
     uint32_t p = r & 31u;
     uint32_t lo = 0u, m = 1u;  // m = 2^(bits of lo in use)
     const uint32_t kmul = 1u << (32u - kshift);  // x >> kshift == mulhi(x, 2^(32 - kshift))
-    while (left8 > 0) {
-        uint32_t x, syms, c8, cb, ey;
-        // straight-line loop in PTX; it exits on the lookup that completes
-        // the chunk (8 * count >= left8) or on an escape, whose count byte
-        // reads as all ones through the sign-replicating byte permute (the
-        // escape flag is the entry's top bit).  The next stream word is
-        // loaded only when the window crosses into c, one lookup ahead of its
-        // use.  Symbols are appended by multiplication with m = 2^sh (lo +=
-        // syms * m, spill = mulhi(syms, m)); m advances by a rotation by
-        // 8 * count, which wraps exactly when the word fills.
+    uint32_t x, ey;
+    for (;;) {
+        // Symbols are appended by multiplication with m = 2^sh (lo += syms *
+        // m, spill = mulhi(syms, m)); m advances by a rotation by 8 * count,
+        // which wraps exactly when the word fills.  An escape entry appends
+        // nothing and leaves bits and m alone, but its rotation by zero reads
+        // as a full word, so the slot pointer moves on once: undone below.
         asm volatile(
             "{\n\t"
-            ".reg .pred pl, pa, pf;\n\t"
-            ".reg .b32 t0, mn, sp, ex, ad;\n"
+            ".reg .pred pa, pf, pc;\n\t"
+            ".reg .b32 t0, mn, sp, ex, ad, cb, c8;\n"
+            // two lookups per pass, m and mn trading roles, so the rotated
+            // multiplier needs no copy
             "LANES_LOOP:\n\t"
-            "shf.l.wrap.b32 %0, %7, %6, %9;\n\t"  // x = stream bits [p, p + 32)
-            "mul.hi.u32 t0, %0, %15;\n\t"         // fast-table key
-            "mad.lo.u32 ad, t0, 8, %14;\n\t"
-            "ld.shared.v2.u32 {ex, %4}, [ad];\n\t"
-            "and.b32 %3, %4, 255;\n\t"
-            "prmt.b32 %2, %4, 0, 0xBBB1;\n\t"
-            "setp.ge.u32 pl, %2, %13;\n\t"
-            "@pl bra LANES_EXIT;\n\t"
-            "mad.lo.u32 %9, %3, 1, %9;\n\t"  // p += bits used
-            "setp.ge.u32 pa, %9, 32;\n\t"
-            "@pa mov.b32 %6, %7;\n\t"                // a = b
-            "@pa prmt.b32 %7, %8, 0, 0x0123;\n\t"    // b = c, byte-swapped
-            "@pa ld.shared.u32 %8, [%10];\n\t"
-            "@pa add.u32 %10, %10, 4;\n\t"
-            "and.b32 %9, %9, 31;\n\t"
-            "mad.lo.u32 %11, ex, %12, %11;\n\t"      // lo += syms * m
-            "mul.hi.u32 sp, ex, %12;\n\t"            // the part past the word
-            "st.shared.u32 [%5], %11;\n\t"
-            "shf.l.wrap.b32 mn, %12, %12, %2;\n\t"   // m rotated by 8 * count
-            "setp.le.u32 pf, mn, %12;\n\t"           // wrapped: the word is full
-            "@pf add.u32 %5, %5, 128;\n\t"           // next word slot of this lane
-            "@pf mov.b32 %11, sp;\n\t"
-            "mov.b32 %12, mn;\n\t"
-            "mad.lo.s32 %13, %2, -1, %13;\n\t"       // left8 -= 8 * count
-            "bra LANES_LOOP;\n"
-            "LANES_EXIT:\n\t"
-            "mov.b32 %1, ex;\n\t"
+            // lookup (m -> mn)
+            "shf.l.wrap.b32 %0, %4, %3, %6;\n\t"  // x = stream bits [p, p + 32)
+            "mul.hi.u32 t0, %0, %12;\n\t"         // fast-table key
+            "mad.lo.u32 ad, t0, 8, %11;\n\t"
+            "ld.shared.v2.u32 {ex, %1}, [ad];\n\t"
+            "and.b32 cb, %1, 255;\n\t"
+            "prmt.b32 c8, %1, 0, 0x4BB1;\n\t"     // 8 * count, or LANES_ESC_DEC
+            "mad.lo.u32 %6, cb, 1, %6;\n\t"       // p += bits used (multiply-add pipe)
+            "setp.ge.u32 pa, %6, 32;\n\t"
+            "@pa mov.b32 %3, %4;\n\t"                // a = b
+            "@pa prmt.b32 %4, %5, 0, 0x0123;\n\t"    // b = c, byte-swapped
+            "@pa ld.shared.u32 %5, [%7];\n\t"
+            "@pa add.u32 %7, %7, 4;\n\t"
+            "and.b32 %6, %6, 31;\n\t"
+            "mad.lo.u32 %8, ex, %9, %8;\n\t"        // lo += syms * m
+            "mul.hi.u32 sp, ex, %9;\n\t"            // the part past the word
+            "st.shared.u32 [%2], %8;\n\t"
+            "shf.l.wrap.b32 mn, %9, %9, c8;\n\t"   // m rotated by 8 * count
+            "setp.le.u32 pf, mn, %9;\n\t"          // wrapped: the word is full
+            "@pf add.u32 %2, %2, 136;\n\t"           // next word slot of this lane (EXP_STRIDE)
+            "@pf mov.b32 %8, sp;\n\t"
+            "mad.lo.s32 %10, c8, -1, %10;\n\t"       // left8 -= 8 * count (multiply-add pipe)
+            "setp.gt.s32 pc, %10, 0;\n\t"
+            "@!pc bra LANES_EXIT_A;\n\t"
+            // lookup (mn -> m)
+            "shf.l.wrap.b32 %0, %4, %3, %6;\n\t"  // x = stream bits [p, p + 32)
+            "mul.hi.u32 t0, %0, %12;\n\t"         // fast-table key
+            "mad.lo.u32 ad, t0, 8, %11;\n\t"
+            "ld.shared.v2.u32 {ex, %1}, [ad];\n\t"
+            "and.b32 cb, %1, 255;\n\t"
+            "prmt.b32 c8, %1, 0, 0x4BB1;\n\t"     // 8 * count, or LANES_ESC_DEC
+            "mad.lo.u32 %6, cb, 1, %6;\n\t"       // p += bits used (multiply-add pipe)
+            "setp.ge.u32 pa, %6, 32;\n\t"
+            "@pa mov.b32 %3, %4;\n\t"                // a = b
+            "@pa prmt.b32 %4, %5, 0, 0x0123;\n\t"    // b = c, byte-swapped
+            "@pa ld.shared.u32 %5, [%7];\n\t"
+            "@pa add.u32 %7, %7, 4;\n\t"
+            "and.b32 %6, %6, 31;\n\t"
+            "mad.lo.u32 %8, ex, mn, %8;\n\t"        // lo += syms * m
+            "mul.hi.u32 sp, ex, mn;\n\t"            // the part past the word
+            "st.shared.u32 [%2], %8;\n\t"
+            "shf.l.wrap.b32 %9, mn, mn, c8;\n\t"   // m rotated by 8 * count
+            "setp.le.u32 pf, %9, mn;\n\t"          // wrapped: the word is full
+            "@pf add.u32 %2, %2, 136;\n\t"           // next word slot of this lane (EXP_STRIDE)
+            "@pf mov.b32 %8, sp;\n\t"
+            "mad.lo.s32 %10, c8, -1, %10;\n\t"       // left8 -= 8 * count (multiply-add pipe)
+            "setp.gt.s32 pc, %10, 0;\n\t"
+            "@pc bra LANES_LOOP;\n\t"
+            "bra LANES_DONE;\n"
+            "LANES_EXIT_A:\n\t"
+            "mov.b32 %9, mn;\n"
+            "LANES_DONE:\n\t"
             "}"
-            : "=r"(x), "=r"(syms), "=r"(c8), "=r"(cb), "=r"(ey), "+r"(ep), "+r"(a), "+r"(b), "+r"(c), "+r"(p),
-              "+r"(wa), "+r"(lo), "+r"(m), "+r"(left8)
+            : "=r"(x), "=r"(ey), "+r"(ep), "+r"(a), "+r"(b), "+r"(c), "+r"(p), "+r"(wa), "+r"(lo), "+r"(m),
+              "+r"(left8)
             : "r"(fast), "r"(kmul)
             : "memory");
-        if (cb != 255u) {
-            // the chunk's last lookup: later codewords belong to the next
-            // chunk, so advance only to the end of codeword left8/8 - 1
-            uint32_t ends = (ey >> FAST_ENDS_SHIFT) & 0xFFFu;
-            for (int i = 8; i < left8; i += 8) ends &= ends - 1u;
-            cb = (uint32_t)__ffs(ends);
-            c8 = (uint32_t)left8;
-        } else {  // first codeword longer than the fast key
-            const uint32_t f = resolve_escape(x, g_hier, n_tables);
-            if (f & ESC_BAD) err |= ST_LUT;
-            syms = rot_sym(f);
-            c8 = 8u;
-            cb = (f >> LUT_LEN_SHIFT) & 63u;  // <= 32: at most one word to shift in
-        }
-        p += cb;
+        if (left8 > -LANES_ESC_DEC / 2) break;  // the chunk's count is reached
+        // an escape: take back the slot step and resolve the codeword in the
+        // byte-keyed hierarchy
+        left8 += LANES_ESC_DEC;
+        ep -= EXP_STRIDE;
+        lo = lds32(ep);
+        const uint32_t f = resolve_escape(x, g_hier, n_tables);
+        if (f & ESC_BAD) err |= ST_LUT;
+        p += (f >> LUT_LEN_SHIFT) & 63u;  // <= 32: at most one word to shift in
         if (p >= 32u) {
             a = b;
             b = bswap32(c);
@@ -159,55 +199,99 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             wa += 4u;
             p -= 32u;
         }
+        const uint32_t syms = rot_sym(f);
         const uint32_t spill = __umulhi(syms, m);
         lo += syms * m;
-        const uint32_t mn = __funnelshift_l(m, m, c8);
+        const uint32_t mn = __funnelshift_l(m, m, 8u);
         if (mn <= m) {
             sts32(ep, lo);
-            ep += 128u;
+            ep += EXP_STRIDE;
             lo = spill;
         }
         m = mn;
-        left8 -= (int)c8;
+        left8 -= 8;
+        ey = 0u;
+        if (left8 <= 0) break;
     }
     if (m != 1u) sts32(ep, lo);
-    return 8u * (wa - sw) - 96u + p;
+    uint32_t end = 8u * (wa - sw) - 96u + p;
+    if (left8 < 0) {
+        // the last lookup (a fast entry) ran -left8 / 8 codewords past the
+        // chunk: its end is that of codeword number keep of the lookup
+        uint32_t ends = (ey >> FAST_ENDS_SHIFT) & 0xFFFu;
+        const uint32_t c8 = (ey >> FAST_C8_SHIFT) & 255u;
+        const uint32_t keep = (c8 - (uint32_t)(-left8)) >> 3;  // >= 1
+        for (uint32_t i = 1; i < keep; ++i) ends &= ends - 1u;
+        end = end - (ey & 255u) + (uint32_t)__ffs(ends);
+    }
+    return end;
 }
 
-// What a lane does with its decoded chunk (64 rotated exponents in its word
-// slots at exps, exps + 128, ...; its 64 raw bytes at mrow): t weights of
-// chunk c, t < 64 only for the last chunk of the scope.
+// What a warp does with its decoded group: the 32 chunks' rotated exponents
+// sit in the word slots at exps0 (word k of chunk c at exps0 + EXP_STRIDE * k
+// + 4 c), their 2048 raw bytes at mbuf (chunk c at mbuf + 64 c); g is the
+// group.  A chunk holds 64 weights except the scope's last one (last_t).
 
-// Decode: join into bf16 and store (piece q = 16 weights, in the order
-// (j + lane / 2) mod 4 so lanes spread over the banks).
+// Weights of chunk c of the scope (64 except the last chunk; 0 past it).
+__device__ __forceinline__ uint32_t chunk_weights(const LanesParams &prm, uint32_t c) {
+    return c + 1u < prm.n_chunks ? LANE_SYMS : (c + 1u == prm.n_chunks ? prm.last_t : 0u);
+}
+
+// Sixteen weights: raw bytes at m (16 bytes), rotated exponents in four
+// words at e, e + EXP_STRIDE, ... -> sixteen bf16 patterns.
+__device__ __forceinline__ void join16(uint32_t m_addr, uint32_t e_addr, uint4 &r0, uint4 &r1) {
+    const uint4 m = lds128(m_addr);
+    const uint32_t e0 = lds32(e_addr), e1 = lds32(e_addr + EXP_STRIDE), e2 = lds32(e_addr + 2u * EXP_STRIDE),
+                   e3 = lds32(e_addr + 3u * EXP_STRIDE);
+    join4(e0, m.x, r0.x, r0.y);
+    join4(e1, m.y, r0.z, r0.w);
+    join4(e2, m.z, r1.x, r1.y);
+    join4(e3, m.w, r1.z, r1.w);
+}
+
+// Decode: join into bf16 and store.  Store j of the warp writes bytes
+// [1024 j, 1024 j + 1024) of the group's output, lane l the 32 bytes of piece
+// l & 3 (16 weights) of chunk 8 j + l / 4, so each store instruction writes
+// eight whole 128-byte lines; the raw bytes it reads are one contiguous 512
+// bytes and its exponent words fall in 32 different banks.
 struct StoreEpi {
     struct Params {};
-    __device__ static __forceinline__ void apply(const LanesParams &prm, const Params &, uint32_t lane, uint32_t c,
-                                                 uint32_t t, uint32_t mrow, uint32_t exps) {
-        uint16_t *dst = prm.out + (size_t)c * LANE_SYMS;
+    __device__ static __forceinline__ void apply(const LanesParams &prm, const Params &, uint32_t lane, uint32_t g,
+                                                 uint32_t mbuf, uint32_t exps0) {
+        const uint32_t i = lane & 3u, cl = lane >> 2;
+        const uint32_t mrow = mbuf + 16u * lane;                             // + 512 j
+        const uint32_t erow = exps0 + 4u * cl + 4u * EXP_STRIDE * i;         // + 32 j, + EXP_STRIDE per word
+        uint16_t *dst = prm.out + (size_t)g * GROUP_SYMS + 16u * lane;     // + 512 j
+        const uint32_t c0 = g * GROUP_CHUNKS;
+        const bool whole = c0 + GROUP_CHUNKS < prm.n_chunks ||
+                           (c0 + GROUP_CHUNKS == prm.n_chunks && prm.last_t == LANE_SYMS);
+        if (whole && prm.out32) {  // every group but the scope's last: no checks
 #pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint4 r0, r1;
+                join16(mrow + 512u * j, erow + 32u * j, r0, r1);
+                stg256_cs(dst + 512u * j, r0, r1);  // a whole sector per lane, 1 KB per warp
+            }
+            return;
+        }
+#pragma unroll 1
         for (int j = 0; j < 4; ++j) {
-            const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
-            const uint4 m = lds128(mrow + 16u * q);
-            const uint32_t e0 = lds32(exps + 512u * q), e1 = lds32(exps + 512u * q + 128u),
-                           e2 = lds32(exps + 512u * q + 256u), e3 = lds32(exps + 512u * q + 384u);
             uint4 r0, r1;
-            join4(e0, m.x, r0.x, r0.y);
-            join4(e1, m.y, r0.z, r0.w);
-            join4(e2, m.z, r1.x, r1.y);
-            join4(e3, m.w, r1.z, r1.w);
-            if (16u * q + 16u <= t) {
+            join16(mrow + 512u * j, erow + 32u * j, r0, r1);
+            const uint32_t t = whole ? LANE_SYMS : chunk_weights(prm, c0 + 8u * j + cl);
+            if (16u * i + 16u <= t) {
                 if (prm.out32) {
-                    stg256_cs(dst + 16u * q, r0, r1);  // a whole sector per lane
+                    stg256_cs(dst + 512u * j, r0, r1);
                 } else {
-                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q), r0);
-                    __stcs(reinterpret_cast<uint4 *>(dst + 16u * q + 8u), r1);
+                    __stcs(reinterpret_cast<uint4 *>(dst + 512u * j), r0);
+                    __stcs(reinterpret_cast<uint4 *>(dst + 512u * j + 8u), r1);
                 }
-            } else {  // the last, partial chunk of the tensor: one weight at a time
-                for (uint32_t i = 16u * q; i < t; ++i) {
-                    const uint32_t e = (lds32(exps + 128u * (i >> 2)) >> (8u * (i & 3u))) & 0xFFu;
-                    const uint32_t mb = (lds32(mrow + (i & ~3u)) >> (8u * (i & 3u))) & 0xFFu;
-                    dst[i] = join1(e, mb);
+            } else {  // the last, partial chunk of the scope: one weight at a time
+                const uint32_t cw = 8u * j + cl;
+                for (uint32_t w = 16u * i; w < t; ++w) {
+                    const uint32_t e = (lds32(exps0 + EXP_STRIDE * (w >> 2) + 4u * cw) >> (8u * (w & 3u))) & 0xFFu;
+                    const uint32_t mb = (lds32(mbuf + 64u * cw + (w & ~3u)) >> (8u * (w & 3u))) & 0xFFu;
+                    prm.out[(size_t)(c0 + cw) * LANE_SYMS + w] = join1(e, mb);
                 }
             }
         }
@@ -216,9 +300,10 @@ struct StoreEpi {
 
 // Decode fused with y = W x: the chunk's 64 weights never leave the SM.
 // Every tensor is whole chunks (its columns a multiple of 64), so a chunk is
-// 64 consecutive columns of one row; the lane writes that row segment's dot
-// product with x to partial[c] (fp32, products exact, one rounding per
-// fused multiply-add, four interleaved sums added in a fixed order).
+// 64 consecutive columns of one row; lane l takes chunk l of the group and
+// writes that row segment's dot product with x to partial[c] (fp32, products
+// exact, one rounding per fused multiply-add, four interleaved sums added in
+// a fixed order).
 struct DotEpi {
     struct Params {
         uint32_t k;                              // tensors in the scope
@@ -227,9 +312,11 @@ struct DotEpi {
         const uint16_t *x[GEMV_MAX_TENSORS];     // bf16 input of each tensor, 32-byte aligned
         float *partial;                          // one fp32 per chunk
     };
-    __device__ static __forceinline__ void apply(const LanesParams &, const Params &ep, uint32_t lane, uint32_t c,
-                                                 uint32_t t, uint32_t mrow, uint32_t exps) {
-        if (t == 0) return;
+    __device__ static __forceinline__ void apply(const LanesParams &prm, const Params &ep, uint32_t lane, uint32_t g,
+                                                 uint32_t mbuf, uint32_t exps0) {
+        const uint32_t c = g * GROUP_CHUNKS + lane;
+        if (chunk_weights(prm, c) == 0u) return;
+        const uint32_t mrow = mbuf + 64u * lane, exps = exps0 + 4u * lane;
         const uint64_t w0 = (uint64_t)c * LANE_SYMS;
         uint32_t ti = 0;
 #pragma unroll
@@ -240,16 +327,12 @@ struct DotEpi {
         float acc[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
+            // piece q of the row segment, in the order (j + lane / 2) mod 4,
+            // which spreads the lanes' 16-byte raw-byte reads over the banks
             const uint32_t q = (uint32_t)(j + (lane >> 1)) & 3u;
-            const uint4 m = lds128(mrow + 16u * q);
-            const uint32_t e0 = lds32(exps + 512u * q), e1 = lds32(exps + 512u * q + 128u),
-                           e2 = lds32(exps + 512u * q + 256u), e3 = lds32(exps + 512u * q + 384u);
             uint4 r0, r1, x0, x1;
             ldg256_nc(xp + 16u * q, x0, x1);
-            join4(e0, m.x, r0.x, r0.y);
-            join4(e1, m.y, r0.z, r0.w);
-            join4(e2, m.z, r1.x, r1.y);
-            join4(e3, m.w, r1.z, r1.w);
+            join16(mrow + 16u * q, exps + 4u * EXP_STRIDE * q, r0, r1);
             float a = 0.f;
             a = fma2_bf16(r0.x, x0.x, a);
             a = fma2_bf16(r0.y, x0.y, a);
@@ -267,10 +350,11 @@ struct DotEpi {
 
 // Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes) | 2 x
 // (chunk_bits | stream span) | raw bytes (2048) | exponent word slots
-// (EXP_WORDS x 32).
+// (EXP_WORDS rows of EXP_STRIDE bytes).
 __host__ __device__ constexpr uint32_t warp_smem_bytes(uint32_t sbuf_bytes) {
-    return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + 4u * EXP_WORDS * 32u;
+    return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + EXP_BYTES;
 }
+static_assert(warp_smem_bytes(16u) % 16u == 0u, "per-warp shared areas must stay 16-byte aligned");
 
 template <int NT, class Epi>
 __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const typename Epi::Params ep) {
@@ -285,7 +369,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
     uint8_t *wslots = wbase + 32;
     const uint32_t slot_bytes = 64u + prm.sbuf_bytes;
     uint8_t *mbuf = wslots + 2u * slot_bytes;
-    const uint32_t exps = smem_u32(mbuf + GROUP_SYMS) + 4u * lane;  // word k at exps + 128 k
+    const uint32_t exps0 = smem_u32(mbuf + GROUP_SYMS), exps = exps0 + 4u * lane;  // word k at exps + EXP_STRIDE k
     const uint32_t *g_hier = prm.lut + 2u * n_fast;
     const uint32_t kshift = 32u - prm.fast_bits;
 
@@ -297,9 +381,10 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
     }
     bool bad = false;
     for (uint32_t i = tid; i < n_fast; i += NT) {
-        const uint2 e = __ldg(reinterpret_cast<const uint2 *>(prm.lut) + i);
+        uint2 e = __ldg(reinterpret_cast<const uint2 *>(prm.lut) + i);
         if (e.y & FAST_ESC) {
             bad |= e.y != FAST_ESC_WORD || e.x != 0u;
+            e.y = LANES_ESC_WORD;
         } else {
             const uint32_t cb = e.y & 255u, c8 = (e.y >> FAST_C8_SHIFT) & 255u,
                            ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
@@ -404,7 +489,8 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         } else if (!good) {
             if (err) atomicOr(&g_status, err);
         } else {
-            Epi::apply(prm, ep, lane, c, t, smem_u32(mbuf) + 64u * lane, exps);
+            __syncwarp();  // the epilogue reads other lanes' exponent slots
+            Epi::apply(prm, ep, lane, g, smem_u32(mbuf), exps0);
         }
         if (!has_next) break;
         __syncwarp();  // all lanes have read the raw bytes
