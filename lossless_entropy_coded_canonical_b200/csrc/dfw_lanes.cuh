@@ -444,11 +444,6 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         const uint8_t *slot = wslots + s * slot_bytes;
         const bool has_next = g1 < prm.n_groups;
         const uint32_t g2 = g1 + gstride;
-        uint64_t ms0 = 0, ms1 = 0;
-        if (g2 < prm.n_groups) {  // starts two groups ahead, for the copy issued next round
-            ms0 = __ldg(prm.group_start + g2);
-            ms1 = __ldg(prm.group_start + g2 + 1);
-        }
         __syncwarp();  // every lane is done with the other slot
         if (has_next && lane == 0) issue_stream(g1, s ^ 1u, ns0, ns1);
 
@@ -474,6 +469,14 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
             const uint32_t end = decode_chunk(smem_u32(slot + 64), r, (int)(8u * t), smem_u32(s_fast), kshift,
                                               g_hier, prm.n_tables, exps, err);
             if (end != r + cbits) err |= ST_COUNT;
+        }
+        // starts two groups ahead, for the copy issued next round: loaded
+        // after the decode loop, so they hold no registers during it, and
+        // before the join, which hides their latency
+        uint64_t ms0 = 0, ms1 = 0;
+        if (g2 < prm.n_groups) {
+            ms0 = __ldg(prm.group_start + g2);
+            ms1 = __ldg(prm.group_start + g2 + 1);
         }
         ok = mbar_wait(bar_m, k & 1u) && ok;
         if (!__all_sync(0xFFFFFFFFu, ok)) {  // a bulk copy never completed: give up
