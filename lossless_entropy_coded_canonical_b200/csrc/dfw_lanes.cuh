@@ -99,17 +99,18 @@ constexpr int LANES_ESC_DEC = 0x00FFFF00;
 __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int left8, uint32_t fast,
                                                  uint32_t kshift, const uint32_t *__restrict__ g_hier,
                                                  uint32_t n_tables, uint32_t ep, uint32_t &err) {
-    // a and b hold the two stream words the window [p, p + 32) lies in, c
-    // the word after them (not yet byte-swapped), wa the address of the word
-    // after c: the bit position is 8 * (wa - sw) - 96 + p.  Reads past the
-    // slot (only a corrupt stream causes them) stay inside this warp's shared
-    // area, and the caller's end check rejects it.
+    // p is the bit position (from sw); a and b hold the two stream words the
+    // window [p, p + 32) lies in (the funnel shift takes p mod 32), c the
+    // word after them (not yet byte-swapped), wa the address of the word
+    // after c and qn the position where the window's first word ends.  Reads
+    // past the slot (only a corrupt stream causes them) stay inside this
+    // warp's shared area, and the caller's end check rejects it.
     uint32_t wa = sw + 4u * (r >> 5);
     uint32_t a = bswap32(lds32(wa));
     uint32_t b = bswap32(lds32(wa + 4u));
     uint32_t c = lds32(wa + 8u);
     wa += 12u;
-    uint32_t p = r & 31u;
+    uint32_t p = r, qn = (r & ~31u) + 32u;
     uint32_t lo = 0u, m = 1u;  // m = 2^(bits of lo in use)
     const uint32_t kmul = 1u << (32u - kshift);  // x >> kshift == mulhi(x, 2^(32 - kshift))
     uint32_t x, ey;
@@ -128,18 +129,18 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             "LANES_LOOP:\n\t"
             // lookup (m -> mn)
             "shf.l.wrap.b32 %0, %4, %3, %6;\n\t"  // x = stream bits [p, p + 32)
-            "mul.hi.u32 t0, %0, %12;\n\t"         // fast-table key
-            "mad.lo.u32 ad, t0, 8, %11;\n\t"
+            "mul.hi.u32 t0, %0, %13;\n\t"         // fast-table key
+            "mad.lo.u32 ad, t0, 8, %12;\n\t"
             "ld.shared.v2.u32 {ex, %1}, [ad];\n\t"
             "and.b32 cb, %1, 255;\n\t"
             "prmt.b32 c8, %1, 0, 0x4BB1;\n\t"     // 8 * count, or LANES_ESC_DEC
             "mad.lo.u32 %6, cb, 1, %6;\n\t"       // p += bits used (multiply-add pipe)
-            "setp.ge.u32 pa, %6, 32;\n\t"
+            "setp.ge.u32 pa, %6, %11;\n\t"          // crossed into b
             "@pa mov.b32 %3, %4;\n\t"                // a = b
             "@pa prmt.b32 %4, %5, 0, 0x0123;\n\t"    // b = c, byte-swapped
             "@pa ld.shared.u32 %5, [%7];\n\t"
             "@pa add.u32 %7, %7, 4;\n\t"
-            "and.b32 %6, %6, 31;\n\t"
+            "@pa add.u32 %11, %11, 32;\n\t"         // next word boundary
             "mad.lo.u32 %8, ex, %9, %8;\n\t"        // lo += syms * m
             "mul.hi.u32 sp, ex, %9;\n\t"            // the part past the word
             "st.shared.u32 [%2], %8;\n\t"
@@ -152,18 +153,18 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             "@!pc bra LANES_EXIT_A;\n\t"
             // lookup (mn -> m)
             "shf.l.wrap.b32 %0, %4, %3, %6;\n\t"  // x = stream bits [p, p + 32)
-            "mul.hi.u32 t0, %0, %12;\n\t"         // fast-table key
-            "mad.lo.u32 ad, t0, 8, %11;\n\t"
+            "mul.hi.u32 t0, %0, %13;\n\t"         // fast-table key
+            "mad.lo.u32 ad, t0, 8, %12;\n\t"
             "ld.shared.v2.u32 {ex, %1}, [ad];\n\t"
             "and.b32 cb, %1, 255;\n\t"
             "prmt.b32 c8, %1, 0, 0x4BB1;\n\t"     // 8 * count, or LANES_ESC_DEC
             "mad.lo.u32 %6, cb, 1, %6;\n\t"       // p += bits used (multiply-add pipe)
-            "setp.ge.u32 pa, %6, 32;\n\t"
+            "setp.ge.u32 pa, %6, %11;\n\t"          // crossed into b
             "@pa mov.b32 %3, %4;\n\t"                // a = b
             "@pa prmt.b32 %4, %5, 0, 0x0123;\n\t"    // b = c, byte-swapped
             "@pa ld.shared.u32 %5, [%7];\n\t"
             "@pa add.u32 %7, %7, 4;\n\t"
-            "and.b32 %6, %6, 31;\n\t"
+            "@pa add.u32 %11, %11, 32;\n\t"         // next word boundary
             "mad.lo.u32 %8, ex, mn, %8;\n\t"        // lo += syms * m
             "mul.hi.u32 sp, ex, mn;\n\t"            // the part past the word
             "st.shared.u32 [%2], %8;\n\t"
@@ -180,7 +181,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
             "LANES_DONE:\n\t"
             "}"
             : "=r"(x), "=r"(ey), "+r"(ep), "+r"(a), "+r"(b), "+r"(c), "+r"(p), "+r"(wa), "+r"(lo), "+r"(m),
-              "+r"(left8)
+              "+r"(left8), "+r"(qn)
             : "r"(fast), "r"(kmul)
             : "memory");
         if (left8 > -LANES_ESC_DEC / 2) break;  // the chunk's count is reached
@@ -192,12 +193,12 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         const uint32_t f = resolve_escape(x, g_hier, n_tables);
         if (f & ESC_BAD) err |= ST_LUT;
         p += (f >> LUT_LEN_SHIFT) & 63u;  // <= 32: at most one word to shift in
-        if (p >= 32u) {
+        if (p >= qn) {
             a = b;
             b = bswap32(c);
             c = lds32(wa);
             wa += 4u;
-            p -= 32u;
+            qn += 32u;
         }
         const uint32_t syms = rot_sym(f);
         const uint32_t spill = __umulhi(syms, m);
@@ -214,7 +215,7 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         if (left8 <= 0) break;
     }
     if (m != 1u) sts32(ep, lo);
-    uint32_t end = 8u * (wa - sw) - 96u + p;
+    uint32_t end = p;
     if (left8 < 0) {
         // the last lookup (a fast entry) ran -left8 / 8 codewords past the
         // chunk: its end is that of codeword number keep of the lookup
