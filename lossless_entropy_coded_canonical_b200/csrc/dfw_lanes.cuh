@@ -65,10 +65,12 @@ struct LanesParams {
     uint32_t out32;  // out is 32-byte aligned: one 256-bit store per 16 weights
 };
 
-__device__ __forceinline__ uint32_t span_bytes(uint64_t start_bit, uint64_t end_bit) {
-    const uint64_t b0 = (start_bit >> 3) & ~15ull;
-    const uint64_t b1 = (((end_bit + 7) >> 3) + 8 + 15) & ~15ull;
-    return (uint32_t)(b1 - b0);
+// Bytes a group's stream copy takes: from the 16-byte boundary at or below
+// its first bit s0 to 8 guard bytes past its last byte, rounded up to 16.
+// r0 = s0 mod 128 (the first bit's offset from that boundary) and d = the
+// group's bits (below 2^17), so 32-bit arithmetic suffices.
+__device__ __forceinline__ uint32_t span_bytes(uint32_t r0, uint32_t d) {
+    return (((r0 + d + 7u) >> 3) + 8u + 15u) & ~15u;
 }
 
 // In shared memory the lanes kernel keeps a fast entry's second word as in
@@ -410,8 +412,11 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         const uint32_t bar = bar_s0 + 8u * s;
         const uint64_t sb0 = (s0 >> 3) & ~15ull;
         uint32_t sbytes = 0;
-        if (s1 >= s0 && sb0 < prm.stream_bytes) {
-            sbytes = min(span_bytes(s0, s1), prm.sbuf_bytes);
+        if (sb0 < prm.stream_bytes) {
+            // a start past its end (a corrupt plan) copies a full slot; the
+            // group is rejected before it is decoded
+            const uint64_t d = s1 - s0;
+            sbytes = min(span_bytes((uint32_t)s0 & 127u, d < (1u << 17) ? (uint32_t)d : (1u << 17)), prm.sbuf_bytes);
             sbytes = (uint32_t)min((uint64_t)sbytes, prm.stream_bytes - sb0);
         }
         fence_proxy_async();
@@ -459,14 +464,15 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         const uint32_t excl = incl - cbits, gbits = __shfl_sync(0xFFFFFFFFu, incl, 31);
         const uint32_t c = g * GROUP_CHUNKS + lane;
         const uint32_t t = c + 1u < prm.n_chunks ? LANE_SYMS : (c + 1u == prm.n_chunks ? prm.last_t : 0u);
-        const uint64_t sb0 = (gs0 >> 3) & ~15ull;
-        const bool valid = __all_sync(0xFFFFFFFFu, gs1 >= gs0 && gs1 - gs0 == gbits && cbits <= 32u * LANE_SYMS &&
-                                                       span_bytes(gs0, gs1) <= prm.sbuf_bytes &&
-                                                       sb0 + span_bytes(gs0, gs1) <= prm.stream_bytes &&
+        const uint32_t r0 = (uint32_t)gs0 & 127u;  // first bit, from the copy's 16-byte boundary
+        const uint32_t span = span_bytes(r0, gbits);  // gbits < 2^21; a valid group has <= 32 * 2048
+        const bool valid = __all_sync(0xFFFFFFFFu, gs1 - gs0 == gbits && cbits <= 32u * LANE_SYMS &&
+                                                       span <= prm.sbuf_bytes &&
+                                                       ((gs0 >> 3) & ~15ull) + span <= prm.stream_bytes &&
                                                        (t != 0u || cbits == 0u));
         uint32_t err = 0;
         if (ok && valid && t) {
-            const uint32_t r = (uint32_t)(gs0 - 8ull * sb0) + excl;
+            const uint32_t r = r0 + excl;
             const uint32_t end = decode_chunk(smem_u32(slot + 64), r, (int)(8u * t), smem_u32(s_fast), kshift,
                                               g_hier, prm.n_tables, exps, err);
             if (end != r + cbits) err |= ST_COUNT;
