@@ -402,8 +402,13 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         return;
     }
 
+    // Warp slots are numbered warp-major across the CTAs, so when the groups
+    // do not divide evenly the extra ones spread over all SMs rather than
+    // piling onto the first CTAs.  (The first copies go out only after the
+    // fast table is in: issued earlier, they slow the table load, which every
+    // warp waits for.)
     const uint32_t gstride = gridDim.x * NWARP;
-    uint32_t g = blockIdx.x * NWARP + warp;
+    uint32_t g = (uint32_t)warp * gridDim.x + blockIdx.x;
     if (g >= prm.n_groups) return;  // no CTA barrier follows
 
     // lane 0: chunk_bits and stream span of group gg into slot s
