@@ -351,9 +351,10 @@ struct DotEpi {
     }
 };
 
-// Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes) | 2 x
-// (chunk_bits | stream span) | raw bytes (2048) | exponent word slots
-// (EXP_WORDS rows of EXP_STRIDE bytes).
+// Per-warp shared memory: 3 mbarriers (stream slot 0, 1, raw bytes; warp 0
+// keeps the fast table's in the fourth word) | 2 x (chunk_bits | stream span)
+// | raw bytes (2048) | exponent word slots (EXP_WORDS rows of EXP_STRIDE
+// bytes).
 __host__ __device__ constexpr uint32_t warp_smem_bytes(uint32_t sbuf_bytes) {
     return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + EXP_BYTES;
 }
@@ -376,18 +377,55 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
     const uint32_t *g_hier = prm.lut + 2u * n_fast;
     const uint32_t kshift = 32u - prm.fast_bits;
 
+    // Warp slots are numbered warp-major across the CTAs, so when the groups
+    // do not divide evenly the extra ones spread over all SMs rather than
+    // piling onto the first CTAs.
+    const uint32_t gstride = gridDim.x * NWARP;
+    uint32_t g = (uint32_t)warp * gridDim.x + blockIdx.x;
+    const bool active = g < prm.n_groups;
+    uint32_t g1 = g + gstride;
+    // this warp's first two group starts: their latency overlaps the table load
+    uint64_t gs0 = 0, gs1 = 0, ns0 = 0, ns1 = 0;
+    if (active) {
+        gs0 = __ldg(prm.group_start + g);
+        gs1 = __ldg(prm.group_start + g + 1);
+        if (g1 < prm.n_groups) {
+            ns0 = __ldg(prm.group_start + g1);
+            ns1 = __ldg(prm.group_start + g1 + 1);
+        }
+    }
+
+    // The fast table arrives in one bulk copy (tracked by the spare mbarrier
+    // word of warp 0's area); the group copies go out only after it is in,
+    // since issued earlier they slow it down and every warp waits for it.
+    const uint32_t bar_t = smem_u32(smem + (8u << prm.fast_bits)) + 24u;
     if (lane == 0) {
         mbar_init(bar_s0, 1);
         mbar_init(bar_s0 + 8u, 1);
         mbar_init(bar_m, 1);
+        if (tid == 0) mbar_init(bar_t, 1);
         fence_mbar_init();
+        if (tid == 0) {
+            mbar_expect_tx(bar_t, 8u << prm.fast_bits);
+            bulk_load(smem_u32(s_fast), prm.lut, 8u << prm.fast_bits, bar_t);
+        }
     }
+    __syncthreads();  // the barriers are initialised
+    bool tok = mbar_wait(bar_t, 0u);
+    if (!__syncthreads_and(tok)) {  // the table copy never completed: give up
+        if (tid == 0) {
+            atomicOr(&g_status, ST_TIMEOUT);
+            mbar_wait_bounded(bar_t, 0u);
+        }
+        return;
+    }
+    // check every entry; escapes get the loop's escape word
     bool bad = false;
     for (uint32_t i = tid; i < n_fast; i += NT) {
-        uint2 e = __ldg(reinterpret_cast<const uint2 *>(prm.lut) + i);
+        uint2 e = s_fast[i];
         if (e.y & FAST_ESC) {
             bad |= e.y != FAST_ESC_WORD || e.x != 0u;
-            e.y = LANES_ESC_WORD;
+            s_fast[i].y = LANES_ESC_WORD;
         } else {
             const uint32_t cb = e.y & 255u, c8 = (e.y >> FAST_C8_SHIFT) & 255u,
                            ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
@@ -395,21 +433,12 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
                    8u * cb < c8 || (uint32_t)__popc(ends) * 8u != c8 || (ends >> (cb - 1u)) != 1u ||
                    (e.y & 0x70000000u) || (c8 < 32u && (e.x >> c8) != 0u);
         }
-        s_fast[i] = e;
     }
     if (__syncthreads_or(bad)) {
         if (tid == 0) atomicOr(&g_status, ST_LUT);
         return;
     }
-
-    // Warp slots are numbered warp-major across the CTAs, so when the groups
-    // do not divide evenly the extra ones spread over all SMs rather than
-    // piling onto the first CTAs.  (The first copies go out only after the
-    // fast table is in: issued earlier, they slow the table load, which every
-    // warp waits for.)
-    const uint32_t gstride = gridDim.x * NWARP;
-    uint32_t g = (uint32_t)warp * gridDim.x + blockIdx.x;
-    if (g >= prm.n_groups) return;  // no CTA barrier follows
+    if (!active) return;  // no CTA barrier follows
 
     // lane 0: chunk_bits and stream span of group gg into slot s
     auto issue_stream = [&](uint32_t gg, uint32_t s, uint64_t s0, uint64_t s1) {
@@ -438,13 +467,6 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         bulk_load(smem_u32(mbuf), prm.mant + m0, bytes, bar_m);
     };
 
-    uint64_t gs0 = __ldg(prm.group_start + g), gs1 = __ldg(prm.group_start + g + 1);
-    uint32_t g1 = g + gstride;
-    uint64_t ns0 = 0, ns1 = 0;
-    if (g1 < prm.n_groups) {
-        ns0 = __ldg(prm.group_start + g1);
-        ns1 = __ldg(prm.group_start + g1 + 1);
-    }
     if (lane == 0) {
         issue_stream(g, 0, gs0, gs1);
         issue_mant(g);
