@@ -241,6 +241,27 @@ def run_device(devs, scratch, steps, warmup, stream):
     return total_ms, per_launch, status
 
 
+def run_device_seq(devs, scratch, steps, warmup, stream):
+    """The step as one dfw_decode_lanes_seq call over every scope: the same
+    launches in the same order into the same scratch buffer, each one a
+    programmatic dependent of the one before (it may start while the previous
+    drains and stores only after it completes)."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    for _ in range(warmup):
+        dfw.decode_lanes_seq(devs, scratch, stream=stream)
+    dfw.check(stream)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(steps):
+        dfw.decode_lanes_seq(devs, scratch, stream=stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    return t0.elapsed_time(t1), dfw.check_status(stream)
+
+
 def run_e2e(results, devs, device, steps, stream):
     """Same metric through the public API from pinned host buffers: per block
     H2D of its compressed form, decode, D2H of the decoded weights; copies run
@@ -417,7 +438,9 @@ def run_encode_mode(args, rank, world, blocks, wdesc, device):
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
         "config": {"workload": wdesc, "weights": n_total, "code_tables": len(scopes), "mode": "encode",
                    "l2": "inputs larger than L2 (every step reads every scope's bf16)",
-                   "parallelism": f"replica{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replica{world}" if world > 1 else "single GPU",
+                   "launch": ("one dfw_decode_lanes_seq per step: one launch per scope, each a programmatic "
+                              "dependent of the previous" if lanes else "one dfw_decode_block per scope")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": None, "peak_source": peak_kind, "kernel": "encoder (4 passes + 2 host syncs)",
                      "algorithmic_bytes_per_step": alg, "mean_scope_ms": float(per_scope.mean())},
@@ -648,11 +671,20 @@ def main(argv=None):
     comp_noaux = sum(d.compressed_bytes(with_aux=False) for d in devs)
     alg_bytes = sum(d.algorithmic_bytes() for d in devs)
 
+    lanes = args.variant == "lanes"
     sampler = ClockSampler(local)
     sampler.start()
-    total_ms, per_launch, status = run_device(devs, scratch, args.steps, args.warmup, stream)
+    if lanes:  # the step: one sequence of launches over every scope
+        total_ms, status = run_device_seq(devs, scratch, args.steps, args.warmup, stream)
+    else:
+        total_ms, per_launch, status = run_device(devs, scratch, args.steps, args.warmup, stream)
     clocks = sampler.stop()
     ms_step = max_over_ranks(total_ms / args.steps)
+    per_launch_step_ms = None
+    if lanes:  # the kernel's roofline: the same launches one by one, each bracketed by CUDA events
+        pl_ms, per_launch, st_pl = run_device(devs, scratch, args.steps, 3, stream)
+        per_launch_step_ms = max_over_ranks(pl_ms / args.steps)
+        status = status if status != dfw.OK else st_pl
     ok = status == dfw.OK and verify(blocks, devs, scratch, device)
 
     # roofline of the decode kernel: algorithmic bytes / mean launch duration
@@ -698,7 +730,9 @@ def main(argv=None):
                      "traffic": traffic, "peak_source": peak_kind,
                      "kernel": kernel,
                      "algorithmic_bytes_per_step": alg_bytes,
-                     "mean_launch_ms": float(mean_launch_ms.mean())},
+                     "mean_launch_ms": float(mean_launch_ms.mean()),
+                     "timing": "per-launch CUDA events around each scope's launch, launched one by one",
+                     "one_by_one_ms_per_step": per_launch_step_ms},
         "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": args.steps * len(devs),
         "verified_bit_exact": bool(ok),
     }

@@ -272,6 +272,42 @@ dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, cons
                             void *cuda_stream);
 
 /*
+ * dfw_lanes_scope -- one code-table scope of a sequence: the arguments of a
+ * dfw_decode_lanes call other than the output and the stream (device
+ * buffers as there; table and info in host memory).
+ */
+typedef struct dfw_lanes_scope {
+    const uint8_t *d_stream;
+    const uint8_t *d_mant;
+    const uint32_t *d_lut;
+    const uint16_t *d_chunk_bits;
+    const uint64_t *d_group_start;
+    const dfw_table *table;
+    const dfw_lanes_info *info;
+} dfw_lanes_scope;
+
+/*
+ * dfw_decode_lanes_seq -- k scopes decoded one after another into the same
+ * output buffer: transformer-block-level decompression of a model, block by
+ * block, into one scratch buffer (DFloat11 abstract, point (iii)).  The
+ * result is exactly that of k dfw_decode_lanes calls in order on cuda_stream:
+ * scope i writes d_out[0, n_i) only after scope i - 1 has finished writing.
+ * What differs is scheduling: from the second scope on, each launch is a
+ * programmatic dependent of the one before, so it may start on SMs the
+ * previous launch has left (loading its table, fetching and decoding its
+ * first groups) and it holds its stores until that launch has completed.
+ * Hence every scope's inputs must be complete when the call is made (all
+ * earlier work on cuda_stream counts) and no input may overlap d_out.
+ *   scopes   host array of k scopes (k = 0 does nothing)
+ *   d_out    max over scopes of n bf16, 16-byte aligned (32-byte alignment
+ *            lets the kernel store whole 32-byte sectors)
+ * Every scope is checked before the first launch; errors as
+ * dfw_decode_lanes (nothing is launched on a host-side error); corrupt
+ * streams or plans are flagged through dfw_check.  Asynchronous.
+ */
+dfw_status dfw_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, void *cuda_stream);
+
+/*
  * dfw_decode_gemv_lanes -- decode fused with its consumer: y_i = W_i x_i for
  * each of the k tensors of a scope (a transformer block's seven matrices, or
  * one), without writing the decoded weights anywhere.  Source: Huff-LLM

@@ -21,11 +21,11 @@ from dataclasses import dataclass
 import numpy as np
 import torch
 
-from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, LanesInfo, PlanInfo, RansTable,
-                   Table, check as _check, lib)
+from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, LanesInfo, LanesScope, PlanInfo,
+                   RansTable, Table, check as _check, lib)
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
-           "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "LanesInfo",
+           "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "decode_lanes_seq", "LanesInfo",
            "encode_device", "encode_device_scratch_bytes", "decode_gemv_lanes",
            "rans_encode", "RansEncoded", "DeviceRans", "rans_decode", "RansTable",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
@@ -273,6 +273,24 @@ def decode_lanes(dl: DeviceLanes, out: torch.Tensor | None = None, stream=None) 
     _check(lib().dfw_decode_lanes(_ptr(dl.stream), _ptr(dl.mant), _ptr(dl.lut), _ptr(dl.chunk_bits),
                                   _ptr(dl.group_start), ctypes.byref(dl.table), ctypes.byref(dl.info), _ptr(out),
                                   _stream_handle(stream)), "dfw_decode_lanes")
+    return out
+
+
+def decode_lanes_seq(dls, out: torch.Tensor, stream=None) -> torch.Tensor:
+    """Decodes the scopes ``dls`` one after another into ``out``
+    (``dfw_decode_lanes_seq``): the same result as ``decode_lanes`` on each
+    in order, with each launch allowed to start while the previous drains.
+    ``out`` must hold the largest scope; returns it."""
+    dls = list(dls)
+    if not dls:
+        return out
+    if out.numel() < max(d.n for d in dls) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous tensor holding the largest scope")
+    arr = (LanesScope * len(dls))()
+    for i, d in enumerate(dls):
+        arr[i] = LanesScope(_ptr(d.stream), _ptr(d.mant), _ptr(d.lut), _ptr(d.chunk_bits), _ptr(d.group_start),
+                            ctypes.pointer(d.table), ctypes.pointer(d.info))
+    _check(lib().dfw_decode_lanes_seq(len(dls), arr, _ptr(out), _stream_handle(stream)), "dfw_decode_lanes_seq")
     return out
 
 

@@ -39,6 +39,13 @@ class LanesInfo(ctypes.Structure):
                 ("lut_tables", ctypes.c_uint32), ("fast_bits", ctypes.c_uint32)]
 
 
+class LanesScope(ctypes.Structure):
+    """dfw_lanes_scope: one scope of dfw_decode_lanes_seq."""
+    _fields_ = [("d_stream", ctypes.c_void_p), ("d_mant", ctypes.c_void_p), ("d_lut", ctypes.c_void_p),
+                ("d_chunk_bits", ctypes.c_void_p), ("d_group_start", ctypes.c_void_p),
+                ("table", ctypes.POINTER(Table)), ("info", ctypes.POINTER(LanesInfo))]
+
+
 class RansTable(ctypes.Structure):
     _fields_ = [("version", ctypes.c_uint32), ("scale_bits", ctypes.c_uint32), ("lanes", ctypes.c_uint32),
                 ("block_syms", ctypes.c_uint32), ("n", ctypes.c_uint64), ("n_blocks", ctypes.c_uint64),
@@ -64,6 +71,7 @@ SIGNATURES = {
     "dfw_plan_lanes_query": (_i, [_TP, _LP]),
     "dfw_plan_lanes": (_i, [_vp, _TP, _vp, _vp, _vp, _LP]),
     "dfw_decode_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _vp, _vp]),
+    "dfw_decode_lanes_seq": (_i, [_i, _vp, _vp, _vp]),
     "dfw_decode_gemv_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _i, _vp, _vp, _vp, _vp, _vp, _u64, _vp]),
     "dfw_encode_device_scratch_bytes": (_u64, [_u64]),
     "dfw_encode_device": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _vp, _u64, _TP, _LP, _vp]),

@@ -481,6 +481,17 @@ extern "C" dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d
     return launch_decode_lanes(d_stream, d_mant, d_lut, d_chunk_bits, d_group_start, table, info, d_out, s, sms);
 }
 
+extern "C" dfw_status dfw_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, void *cuda_stream) {
+    if (k < 0 || (k > 0 && (!scopes || !d_out))) return DFW_EINVAL;
+    if (k == 0) return DFW_OK;
+    if (reinterpret_cast<uintptr_t>(d_out) & 15u) return DFW_EALIGN;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return DFW_ECUDA;
+    return launch_decode_lanes_seq(k, scopes, d_out, static_cast<cudaStream_t>(cuda_stream), sms);
+}
+
 extern "C" dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
                                             const uint16_t *d_chunk_bits, const uint64_t *d_group_start,
                                             const dfw_table *table, const dfw_lanes_info *info, int k,

@@ -63,7 +63,19 @@ struct LanesParams {
     uint32_t last_t;              // codewords in the last chunk (1..64)
     uint32_t fast_bits, n_tables, sbuf_bytes;
     uint32_t out32;  // out is 32-byte aligned: one 256-bit store per 16 weights
+    // Launched as a programmatic dependent of the previous decode into the
+    // same output: may start while that launch drains, but waits for it to
+    // complete before its first store.
+    uint32_t wait_prior;
 };
+
+// Programmatic dependent launch: let the next launch on the stream start as
+// SMs free up / wait until the launch before this one has completed and its
+// writes are visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Bytes a group's stream copy takes: from the 16-byte boundary at or below
 // its first bit s0 to 8 guard bytes past its last byte, rounded up to 16.
@@ -376,6 +388,8 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
     const uint32_t exps0 = smem_u32(mbuf + GROUP_SYMS), exps = exps0 + 4u * lane;  // word k at exps + EXP_STRIDE k
     const uint32_t *g_hier = prm.lut + 2u * n_fast;
     const uint32_t kshift = 32u - prm.fast_bits;
+    // the next decode in a sequence may take SMs as this one's CTAs finish
+    griddep_launch_dependents();
 
     // Warp slots are numbered warp-major across the CTAs, so when the groups
     // do not divide evenly the extra ones spread over all SMs rather than
@@ -521,6 +535,9 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
             return;
         }
         const bool good = valid && !__any_sync(0xFFFFFFFFu, err != 0u);
+        // the previous decode of a sequence owns the output until it ends:
+        // wait once, before this warp's first store
+        if (k == 0 && prm.wait_prior) griddep_wait();
         if (!valid) {
             if (lane == 0) atomicOr(&g_status, ST_RANGE);
         } else if (!good) {
@@ -569,9 +586,11 @@ typename LanesVariants<Epi>::V LanesVariants<Epi>::v[5] = {
     {128, decode_lanes<128, Epi>, lanes_smem<128>, {0}},
 };
 
+// pdl: launch as a programmatic dependent of the previous kernel on the
+// stream (prm.wait_prior must then be set).
 template <class Epi>
 dfw_status launch_lanes(const LanesParams &prm, const typename Epi::Params &ep, uint64_t n_groups, cudaStream_t s,
-                        int sms) {
+                        int sms, bool pdl = false) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
     for (auto &v : LanesVariants<Epi>::v) {
@@ -588,8 +607,22 @@ dfw_status launch_lanes(const LanesParams &prm, const typename Epi::Params &ep, 
         const uint64_t wpc = (uint64_t)v.nt / 32;
         const uint64_t warps = (uint64_t)per_sm * sms * wpc;
         const uint64_t want = n_groups < warps ? n_groups : warps;
-        v.fn<<<(unsigned)((want + wpc - 1) / wpc), v.nt, smem, s>>>(prm, ep);
-        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+        const unsigned grid = (unsigned)((want + wpc - 1) / wpc);
+        if (!pdl) {
+            v.fn<<<grid, v.nt, smem, s>>>(prm, ep);
+            return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+        }
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(grid);
+        cfg.blockDim = dim3((unsigned)v.nt);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, v.fn, prm, ep) == cudaSuccess ? DFW_OK : DFW_ECUDA;
     }
     return DFW_EINVAL;  // even the smallest CTA does not fit
 }
@@ -629,6 +662,7 @@ dfw_status lanes_params(const uint8_t *d_stream, const uint8_t *d_mant, const ui
     prm.n_tables = info->lut_tables;
     prm.sbuf_bytes = info->max_group_bytes;
     prm.out32 = 0u;
+    prm.wait_prior = 0u;
     return DFW_OK;
 }
 
@@ -711,6 +745,42 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     prm.out = d_out;
     prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
     return launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, info->n_groups, s, sms);
+}
+
+dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, cudaStream_t s, int sms) {
+    // every scope is checked before the first launch
+    for (int i = 0; i < k; ++i) {
+        const dfw_lanes_scope &sc = scopes[i];
+        dfw_status st = validate_table(sc.table);
+        if (st != DFW_OK) return st;
+        if (!sc.info || !sc.d_mant) return DFW_EINVAL;
+        if (reinterpret_cast<uintptr_t>(sc.d_mant) & 15u) return DFW_EALIGN;
+        if (sc.table->n == 0 || sc.table->total_bits == 0) continue;
+        LanesParams prm;
+        st = lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);
+        if (st != DFW_OK) return st;
+    }
+    bool prior = false;  // a decode into d_out is already on the stream from this call
+    for (int i = 0; i < k; ++i) {
+        const dfw_lanes_scope &sc = scopes[i];
+        const uint64_t n = sc.table->n;
+        if (n == 0) continue;
+        if (sc.table->total_bits == 0) {  // one exponent: an ordinary launch, after the previous one
+            const uint64_t want = ((n >> 3) + 256) / 256, cap = (uint64_t)sms * 8;
+            fill_single<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(sc.d_mant, sc.table->single_symbol, n, d_out);
+            if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+        } else {
+            LanesParams prm;
+            lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);
+            prm.out = d_out;
+            prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
+            prm.wait_prior = prior ? 1u : 0u;
+            const dfw_status st = launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, sc.info->n_groups, s, sms, prior);
+            if (st != DFW_OK) return st;
+        }
+        prior = true;
+    }
+    return DFW_OK;
 }
 
 dfw_status launch_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,

@@ -1,0 +1,135 @@
+"""dfw_decode_lanes_seq: several scopes decoded one after another into one
+output buffer, each launch a programmatic dependent of the previous one.
+
+The result must be exactly that of dfw_decode_lanes called on each scope in
+order (same bytes everywhere in the buffer, including what earlier, larger
+scopes leave beyond a later scope's end), and the last scope's weights must
+be the oracle's decode of that scope.  Repeated runs over a buffer refilled
+with garbage would show a store that overtook the previous scope.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import lossless_entropy_coded_canonical_b200 as dfw
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    dfw.lib()
+    dfw.check()
+
+
+def _u16(spec) -> np.ndarray:
+    return np.concatenate([workloads.as_u16_numpy(t) for t in workloads.generate_block(spec, "cpu")])
+
+
+def _scopes():
+    """Mixed scopes: Llama-3 and Llama-2 block shapes (scaled), heavy tails with
+    zeros, long codes (escapes), incompressible data, one exponent, a scope
+    that ends inside its first group."""
+    rng = np.random.default_rng(5)
+    single = ((rng.integers(0, 2, 100_003) << 15) | (121 << 7) | rng.integers(0, 128, 100_003)).astype(np.uint16)
+    return [
+        _u16(workloads.scaled(workloads.c5()[1], 1_500_000)),
+        _u16(workloads.scaled(workloads.c3(), 2_000_000)),
+        single,
+        _u16(workloads.scaled(workloads.c2(), 1000)),
+        _u16(workloads.scaled(workloads.c4("b"), 500_000)),
+        _u16(workloads.scaled(workloads.c4("c"), 300_000)),
+    ]
+
+
+def _device(u: np.ndarray) -> dfw.DeviceLanes:
+    enc = dfw.encode(u)
+    return dfw.DeviceLanes.upload(enc, dfw.plan_lanes(enc), "cuda")
+
+
+@pytest.fixture(scope="module")
+def scopes():
+    us = _scopes()
+    return us, [_device(u) for u in us]
+
+
+def _garbage(n: int) -> torch.Tensor:
+    return torch.full((n,), 0x5A5A, dtype=torch.int16, device="cuda").view(torch.bfloat16)
+
+
+def test_seq_matches_calls_in_order(oracle, scopes):
+    us, devs = scopes
+    nmax = max(u.size for u in us)
+    for rot in range(len(us)):  # every scope comes last once
+        order = list(range(rot + 1, len(us))) + list(range(rot + 1))
+        got, want = _garbage(nmax), _garbage(nmax)
+        dfw.decode_lanes_seq([devs[i] for i in order], got)
+        for i in order:
+            dfw.decode_lanes(devs[i], want)
+        dfw.check()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"order {order}"
+        last = us[order[-1]]
+        expect = oracle.decode(oracle.encode(last))
+        assert np.array_equal(workloads.as_u16_numpy(got)[: last.size], expect), f"last scope {order[-1]}"
+
+
+def test_seq_repeated_over_garbage(scopes):
+    us, devs = scopes
+    nmax = max(u.size for u in us)
+    want = _garbage(nmax)
+    for d in devs:
+        dfw.decode_lanes(d, want)
+    dfw.check()
+    for _ in range(6):
+        got = _garbage(nmax)
+        dfw.decode_lanes_seq(devs, got)
+        dfw.check()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+def test_seq_full_size_llama3_blocks():
+    """Three consecutive transformer blocks of the 8B-shaped model at full size,
+    one buffer: the buffer ends as the last block's input, bit for bit."""
+    blocks = workloads.c5()[1:4]
+    devs, last = [], None
+    for b in blocks:
+        ts = workloads.generate_block(b, "cuda")
+        enc = dfw.encode_multi([t.cpu() for t in ts], 32)
+        devs.append(dfw.DeviceLanes.upload(enc, dfw.plan_lanes(enc), "cuda"))
+        last = torch.cat([t.reshape(-1) for t in ts])
+    out = _garbage(max(d.n for d in devs))
+    for _ in range(2):
+        dfw.decode_lanes_seq(devs, out)
+        dfw.check()
+        assert torch.equal(out.view(torch.int16)[: last.numel()], last.view(torch.int16))
+
+
+def test_seq_rejects_bad_arguments_before_launch(scopes):
+    us, devs = scopes
+    lib = dfw.lib()
+    out = _garbage(max(u.size for u in us) + 8)
+    before = out.clone()
+    # k = 0 does nothing
+    assert lib.dfw_decode_lanes_seq(0, None, out.data_ptr(), None) == dfw.OK
+    # misaligned output
+    d = devs[0]
+    arr = (dfw.LanesScope * 1)()
+    arr[0] = dfw.LanesScope(d.stream.data_ptr(), d.mant.data_ptr(), d.lut.data_ptr(), d.chunk_bits.data_ptr(),
+                            d.group_start.data_ptr(), ctypes.pointer(d.table), ctypes.pointer(d.info))
+    assert lib.dfw_decode_lanes_seq(1, arr, out.data_ptr() + 2, None) == dfw.EALIGN
+    # one bad scope among good ones: nothing runs
+    bad_info = dfw.LanesInfo.from_buffer_copy(bytes(devs[1].info))
+    bad_info.n_chunks += 1
+    arr3 = (dfw.LanesScope * 3)()
+    for i, (dd, info) in enumerate([(devs[0], devs[0].info), (devs[1], bad_info), (devs[2], devs[2].info)]):
+        arr3[i] = dfw.LanesScope(dd.stream.data_ptr(), dd.mant.data_ptr(), dd.lut.data_ptr(),
+                                 dd.chunk_bits.data_ptr(), dd.group_start.data_ptr(), ctypes.pointer(dd.table),
+                                 ctypes.pointer(info))
+    assert lib.dfw_decode_lanes_seq(3, arr3, out.data_ptr(), None) == dfw.EINVAL
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), before.view(torch.int16))
+    dfw.check()
