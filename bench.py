@@ -612,6 +612,47 @@ def run_rans_mode(args, rank, world, blocks, wdesc, device):
     return 0 if ok else 1
 
 
+# ------------------------------------------------------------------ launch-cost mode
+
+def run_launch_cost_mode(args, rank, world, device):
+    """Decode time against size: one N(0, 0.02) tensor of 1, 2, ..., 32
+    groups (2048 weights) per resident warp, each size timed with CUDA events
+    around single launches; a least-squares line gives the per-launch fixed
+    cost (intercept) and the per-group cost (slope)."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
+    warps = sms * 32
+    rows = []
+    for k in (1, 2, 4, 8, 16, 32):
+        n = warps * 2048 * k
+        spec = workloads.BlockSpec("launch_cost", [workloads.TensorSpec("w", n, "normal", 77, 0.02)])
+        ref = workloads.generate_block(spec, device)[0]
+        enc = dfw.encode_multi([ref.cpu()], 32)
+        dl = dfw.DeviceLanes.upload(enc, dfw.plan_lanes(enc), device)
+        out = torch.empty(n, dtype=torch.bfloat16, device=device)
+        for _ in range(args.warmup):
+            dfw.decode_lanes(dl, out)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            a.record()
+            dfw.decode_lanes(dl, out)
+            b.record()
+        torch.cuda.synchronize()
+        ms = sorted(a.elapsed_time(b) for a, b in ev)
+        exact = bool(torch.equal(out.view(torch.int16), ref.view(torch.int16)))
+        rows.append({"groups_per_warp": k, "weights": n, "median_ms": ms[len(ms) // 2], "bit_exact": exact})
+        del dl, out, ref
+    ks = np.array([r["groups_per_warp"] for r in rows], float)
+    ts = np.array([r["median_ms"] for r in rows])
+    slope, icpt = np.linalg.lstsq(np.vstack([ks, np.ones_like(ks)]).T, ts, rcond=None)[0]
+    if rank == 0:
+        print(json.dumps({"mode": "launch-cost", "resident_warps": warps, "sizes": rows,
+                          "fixed_ms_per_launch": float(icpt), "ms_per_group_per_warp": float(slope),
+                          "verified_bit_exact": all(r["bit_exact"] for r in rows)}), flush=True)
+    return 0 if all(r["bit_exact"] for r in rows) else 1
+
+
 # ------------------------------------------------------------------ main
 
 def main(argv=None):
@@ -630,9 +671,10 @@ def main(argv=None):
     ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv", "rans"],
+    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv", "rans", "launch-cost"],
                     help="decode: the decode path (default); encode: the GPU encoder; "
-                         "gemv: decode fused with y = W x; rans: the rANS variant beside Huffman")
+                         "gemv: decode fused with y = W x; rans: the rANS variant beside Huffman; "
+                         "launch-cost: decode time against size (fixed cost per launch)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -656,6 +698,8 @@ def main(argv=None):
     import lossless_entropy_coded_canonical_b200 as dfw
     dfw.lib()
     dfw.check()
+    if args.mode == "launch-cost":
+        return run_launch_cost_mode(args, rank, world, device)
     if args.mode in ("encode", "gemv", "rans"):
         run = {"encode": run_encode_mode, "gemv": run_gemv_mode, "rans": run_rans_mode}[args.mode]
         rc = run(args, rank, world, blocks, wdesc, device)
