@@ -438,9 +438,7 @@ def run_encode_mode(args, rank, world, blocks, wdesc, device):
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
         "config": {"workload": wdesc, "weights": n_total, "code_tables": len(scopes), "mode": "encode",
                    "l2": "inputs larger than L2 (every step reads every scope's bf16)",
-                   "parallelism": f"replica{world}" if world > 1 else "single GPU",
-                   "launch": ("one dfw_decode_lanes_seq per step: one launch per scope, each a programmatic "
-                              "dependent of the previous" if lanes else "one dfw_decode_block per scope")},
+                   "parallelism": f"replica{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": None, "peak_source": peak_kind, "kernel": "encoder (4 passes + 2 host syncs)",
                      "algorithmic_bytes_per_step": alg, "mean_scope_ms": float(per_scope.mean())},
@@ -766,7 +764,9 @@ def main(argv=None):
                    "tile_windows": args.tile if args.variant == "window" else None,
                    "l2": "inputs larger than L2 (each step reads every block's compressed form and writes "
                          "every block's bf16; no reuse between steps)",
-                   "parallelism": f"replica{world}" if world > 1 else "single GPU"},
+                   "parallelism": f"replica{world}" if world > 1 else "single GPU",
+                   "launch": ("one dfw_decode_lanes_seq per step: one launch per scope, each a programmatic "
+                              "dependent of the previous" if lanes else "one dfw_decode_block per scope")},
         "effective_gbs": eff_gbs, "hbm_frac": eff_gbs / peak,
         "compression_ratio": 2 * n_total / comp, "compression_ratio_no_aux": 2 * n_total / comp_noaux,
         "bits_per_weight": 8 * comp / n_total,
