@@ -219,6 +219,31 @@ dfw_status dfw_decode_block(const uint8_t *d_stream, const uint8_t *d_mant, cons
  */
 dfw_status dfw_check(void *cuda_stream);
 
+/* Bits of the device status word (what a kernel saw; sticky until read). */
+#define DFW_ST_COUNT 1u   /* codewords ended elsewhere than the plan says */
+#define DFW_ST_LUT 2u     /* a table entry or pointer is invalid */
+#define DFW_ST_RANGE 4u   /* plan offsets out of order or out of range */
+#define DFW_ST_TIMEOUT 8u /* a wait for a bulk copy gave up; the kernel returned early */
+
+/*
+ * dfw_status_bits -- dfw_check, and the status bits it read and cleared in
+ * *bits (0 when it returns DFW_OK; bits may be NULL).  Tells a timeout
+ * (DFW_ST_TIMEOUT) from corrupt input.
+ */
+dfw_status dfw_status_bits(void *cuda_stream, uint32_t *bits);
+
+/*
+ * dfw_selftest_wait_timeout -- failure-path check with no fault: one warp
+ * waits, with the bounded wait that every bulk-copy wait here uses, on an
+ * mbarrier whose transaction no copy will complete.  The wait gives up at
+ * its limit (2 s or 2^24 tries, whichever comes first) and the kernel sets
+ * DFW_ST_TIMEOUT and returns, as a decode whose copy never landed would; the
+ * context stays usable.  Asynchronous on cuda_stream (up to about 2 s of GPU
+ * time); read the result with dfw_status_bits.  The pages describe no failure detection; this is the
+ * library's own.  Errors: DFW_ECUDA if the launch fails.
+ */
+dfw_status dfw_selftest_wait_timeout(void *cuda_stream);
+
 /*
  * KNOWN-START CHUNKS (a second decode plan over the same stream; the
  * "interleaved lanes" design of the LazyWeights write-up, Verified Facts

@@ -21,8 +21,8 @@ from dataclasses import dataclass
 import numpy as np
 import torch
 
-from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, DfwError, LanesInfo, LanesScope, PlanInfo,
-                   RansTable, Table, check as _check, lib)
+from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT,
+                   DfwError, LanesInfo, LanesScope, PlanInfo, RansTable, Table, check as _check, lib)
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
            "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "decode_lanes_seq", "LanesInfo",
@@ -451,3 +451,11 @@ def check(stream=None) -> None:
 
 def check_status(stream=None) -> int:
     return int(lib().dfw_check(_stream_handle(stream)))
+
+
+def status_bits(stream=None) -> tuple[int, int]:
+    """(status, bits): dfw_check's result and the device status bits it read
+    and cleared (ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT)."""
+    bits = ctypes.c_uint32(0)
+    st = int(lib().dfw_status_bits(_stream_handle(stream), ctypes.byref(bits)))
+    return st, int(bits.value)

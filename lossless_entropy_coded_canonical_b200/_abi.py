@@ -8,6 +8,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdfw.so")
 
 OK, EINVAL, ECAP, ENOMEM, ECORRUPT, EALIGN, ECUDA = range(7)
+ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT = 1, 2, 4, 8  # device status bits (include/dfw.h DFW_ST_*)
 FORMAT_VERSION = 1
 MAX_CAP = 32
 
@@ -72,6 +73,8 @@ SIGNATURES = {
     "dfw_plan_lanes": (_i, [_vp, _TP, _vp, _vp, _vp, _LP]),
     "dfw_decode_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _vp, _vp]),
     "dfw_decode_lanes_seq": (_i, [_i, _vp, _vp, _vp]),
+    "dfw_status_bits": (_i, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "dfw_selftest_wait_timeout": (_i, [_vp]),
     "dfw_decode_gemv_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _i, _vp, _vp, _vp, _vp, _vp, _u64, _vp]),
     "dfw_encode_device_scratch_bytes": (_u64, [_u64]),
     "dfw_encode_device": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _vp, _u64, _TP, _LP, _vp]),

@@ -526,10 +526,42 @@ extern "C" dfw_status dfw_rans_decode(const uint8_t *d_stream, const uint8_t *d_
                               sms);
 }
 
-extern "C" dfw_status dfw_check(void *cuda_stream) {
+extern "C" dfw_status dfw_status_bits(void *cuda_stream, uint32_t *bits) {
+    if (bits) *bits = 0u;
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return DFW_ECUDA;
     unsigned int v = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return DFW_ECUDA;
     if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return DFW_ECUDA;
+    if (bits) *bits = v;
     return v ? DFW_ECORRUPT : DFW_OK;
+}
+
+extern "C" dfw_status dfw_check(void *cuda_stream) { return dfw_status_bits(cuda_stream, nullptr); }
+
+namespace dfw {
+namespace {
+
+// One warp waits, with the bounded wait of the decode kernels, on an
+// mbarrier whose transaction no copy will ever complete (16 bytes expected,
+// none issued): the wait gives up at its time limit and the kernel reports
+// ST_TIMEOUT, as a decode whose bulk copy never landed does.
+__global__ void selftest_wait_timeout() {
+    __shared__ __align__(8) unsigned long long bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_mbar_init();
+        mbar_expect_tx(b, 16u);
+    }
+    __syncwarp();
+    const bool ok = mbar_wait(b, 0u);
+    if (!__all_sync(0xFFFFFFFFu, ok) && threadIdx.x == 0) atomicOr(&g_status, ST_TIMEOUT);
+}
+
+}  // namespace
+}  // namespace dfw
+
+extern "C" dfw_status dfw_selftest_wait_timeout(void *cuda_stream) {
+    dfw::selftest_wait_timeout<<<1, 32, 0, static_cast<cudaStream_t>(cuda_stream)>>>();
+    return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
 }
