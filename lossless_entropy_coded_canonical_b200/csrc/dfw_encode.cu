@@ -22,10 +22,12 @@
 //                          exclusive prefix sums in place (group_start[]);
 //                          the last range writes the total bit count; all
 //                          record the largest group span
-//   4  pack                one warp per group: each lane packs its 8
-//                          codewords at their bit offset (warp prefix sum)
-//                          into the warp's shared word buffer (shared atomic
-//                          OR: neighbours share a word); the warp then writes
+//   4  pack                one warp per group: each lane joins its 8
+//                          codewords into one 64-bit value (almost always
+//                          enough; longer runs take a general path) and ORs
+//                          it at its bit offset (warp prefix sum) into the
+//                          warp's shared word buffer (neighbours share a
+//                          word, so the ORs are atomic); the warp then writes
 //                          the group's words, big-endian, with plain stores
 //                          inside and atomic ORs on the two words it may
 //                          share with the neighbouring groups (the stream is
@@ -93,8 +95,8 @@ __global__ void __launch_bounds__(SPLIT_NT) enc_split_hist(const uint16_t *__res
     uint32_t *hw = h[warp] + (lane & (HIST_COPIES - 1));
     const uint64_t n8 = n >> 3;
     const uint64_t stride = (uint64_t)gridDim.x * SPLIT_NT;
-    for (uint64_t i = (uint64_t)blockIdx.x * SPLIT_NT + tid; i < n8; i += stride) {
-        const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(in) + i);
+    // one 16-byte item: raw bytes out, exponents into the histogram
+    auto item = [&](uint64_t i, const uint4 v) {
         uint32_t m0, e0, m1, e1;
         split4(v.x, v.y, m0, e0);
         split4(v.z, v.w, m1, e1);
@@ -104,7 +106,18 @@ __global__ void __launch_bounds__(SPLIT_NT) enc_split_hist(const uint16_t *__res
             atomicAdd(hw + HIST_COPIES * ((e0 >> (8 * k)) & 0xFFu), 1u);
             atomicAdd(hw + HIST_COPIES * ((e1 >> (8 * k)) & 0xFFu), 1u);
         }
+    };
+    uint64_t i = (uint64_t)blockIdx.x * SPLIT_NT + tid;
+    // four loads in flight per thread before any is used (the pass is bound
+    // by memory latency, not by its arithmetic)
+    for (; i + 3 * stride < n8; i += 4 * stride) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) v[u] = __ldcs(reinterpret_cast<const uint4 *>(in) + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) item(i + u * stride, v[u]);
     }
+    for (; i < n8; i += stride) item(i, __ldcs(reinterpret_cast<const uint4 *>(in) + i));
     if (blockIdx.x == 0) {  // the < 8 trailing weights and the zero padding of the raw bytes
         for (uint64_t j = (n8 << 3) + tid; j < mant_bytes; j += SPLIT_NT) {
             uint8_t m = 0;
@@ -175,12 +188,19 @@ __global__ void __launch_bounds__(GROUP_NT) enc_chunk_bits(const uint16_t *__res
         uint32_t mine = 0;
 #pragma unroll
         for (uint32_t j = 0; j < 8; ++j) {
-            uint32_t x0, x1, cnt = 8u;
-            if (whole) exps8(raw[j], x0, x1);
-            else cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
             uint32_t b = 0;
-            for (uint32_t k = 0; k < 4; ++k) b += k < cnt ? s_len[(x0 >> (8 * k)) & 0xFFu] : 0u;
-            for (uint32_t k = 4; k < 8; ++k) b += k < cnt ? s_len[(x1 >> (8 * (k - 4))) & 0xFFu] : 0u;
+            if (whole) {  // every group but the tensor's last: eight exponents, no checks
+                uint32_t x0, x1;
+                exps8(raw[j], x0, x1);
+#pragma unroll
+                for (uint32_t k = 0; k < 4; ++k)
+                    b += s_len[__byte_perm(x0, 0u, 0x4440u + k)] + s_len[__byte_perm(x1, 0u, 0x4440u + k)];
+            } else {
+                uint32_t x0, x1;
+                const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+                for (uint32_t k = 0; k < 4; ++k) b += k < cnt ? s_len[(x0 >> (8 * k)) & 0xFFu] : 0u;
+                for (uint32_t k = 4; k < 8; ++k) b += k < cnt ? s_len[(x1 >> (8 * (k - 4))) & 0xFFu] : 0u;
+            }
             // lanes 8q .. 8q + 7 hold chunk 4 j + q: sum them
             b += __shfl_xor_sync(FULL, b, 1);
             b += __shfl_xor_sync(FULL, b, 2);
@@ -274,14 +294,6 @@ __global__ void __launch_bounds__(SCAN_NT) enc_range_scan(uint64_t *__restrict__
 
 // ------------------------------------------------------------ pass 4
 
-// x << s with PTX semantics: shifts of 32 or more give 0 (a 32-bit codeword
-// shifts an empty accumulator by 32).
-__device__ __forceinline__ uint32_t shl_clamp(uint32_t x, uint32_t s) {
-    uint32_t r;
-    asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(s));
-    return r;
-}
-
 __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict__ in, uint64_t n, const CodeTable ct,
                                                       const uint64_t *__restrict__ group_start, uint32_t n_groups,
                                                       uint32_t *__restrict__ stream_words, uint32_t buf_words) {
@@ -299,16 +311,26 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
         const uint64_t base = (uint64_t)g * GROUP_W;
         const uint32_t sh0 = (uint32_t)(gs0 & 31u);
         uint32_t carry = sh0;
+        const bool whole = base + GROUP_W <= n;
         for (uint32_t j = 0; j < 8; ++j) {
             uint32_t x0, x1;
-            const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
             unsigned long long lc[8];
             uint32_t b = 0;
+            if (whole) {  // every group but the tensor's last: eight weights, no checks
+                exps8(__ldcs(reinterpret_cast<const uint4 *>(in + base + 8u * (32u * j + lane))), x0, x1);
 #pragma unroll
-            for (uint32_t k = 0; k < 8; ++k) {
-                const uint32_t e = ((k < 4 ? x0 : x1) >> (8 * (k & 3))) & 0xFFu;
-                lc[k] = k < cnt ? s_lc[e] : 0ull;
-                b += (uint32_t)(lc[k] >> 32);
+                for (uint32_t k = 0; k < 8; ++k) {
+                    lc[k] = s_lc[__byte_perm(k < 4 ? x0 : x1, 0u, 0x4440u + (k & 3u))];
+                    b += (uint32_t)(lc[k] >> 32);
+                }
+            } else {
+                const uint32_t cnt = load8(in, n, base + 8u * (32u * j + lane), x0, x1);
+#pragma unroll
+                for (uint32_t k = 0; k < 8; ++k) {
+                    const uint32_t e = ((k < 4 ? x0 : x1) >> (8 * (k & 3))) & 0xFFu;
+                    lc[k] = k < cnt ? s_lc[e] : 0ull;
+                    b += (uint32_t)(lc[k] >> 32);
+                }
             }
             uint32_t incl = b;
 #pragma unroll
@@ -318,14 +340,18 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
             }
             const uint32_t off = carry + incl - b;  // bit offset in the warp's buffer
             carry += __shfl_sync(FULL, incl, 31);
-            if (b && b <= 32u) {  // the common case: the 8 codewords fit one word, placed with <= 2 ORs
-                uint32_t v = 0;
+            if (b && b <= 64u) {
+                // almost every step: the 8 codewords fit 64 bits and are
+                // placed with at most 3 ORs (one long codeword among short
+                // ones no longer sends the lane down the general path)
+                unsigned long long v = 0;
 #pragma unroll
-                for (uint32_t k = 0; k < 8; ++k) v = shl_clamp(v, (uint32_t)(lc[k] >> 32)) | (uint32_t)lc[k];
+                for (uint32_t k = 0; k < 8; ++k) v = (v << (uint32_t)(lc[k] >> 32)) | (uint32_t)lc[k];
                 const uint32_t sh = off & 31u, wi = off >> 5;
-                const unsigned long long placed = (unsigned long long)v << (64u - sh - b);
-                atomicOr(buf + wi, (uint32_t)(placed >> 32));
-                if (sh + b > 32u) atomicOr(buf + wi + 1, (uint32_t)placed);
+                const unsigned long long a = v << (64u - b);  // first bit at bit 63
+                atomicOr(buf + wi, (uint32_t)(a >> (32u + sh)));
+                if (sh + b > 32u) atomicOr(buf + wi + 1, (uint32_t)(a >> sh));
+                if (sh + b > 64u) atomicOr(buf + wi + 2, (uint32_t)(a << (32u - sh)));
             } else if (b) {
                 unsigned long long acc = 0;
                 uint32_t nacc = off & 31u, wi = off >> 5;
