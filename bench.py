@@ -39,10 +39,13 @@ import workloads  # noqa: E402
 
 METRIC = "decoded bf16 weights/sec & effective GB/s as % of HBM roofline; compression ratio"
 FALLBACK_HBM_GBS = 6650.0
-KERNEL_SOURCES = ["lossless_entropy_coded_canonical_b200/csrc/dfw_decode.cu",
-                  "lossless_entropy_coded_canonical_b200/csrc/dfw_lanes.cuh",
-                  "lossless_entropy_coded_canonical_b200/csrc/dfw_device.cuh",
-                  "lossless_entropy_coded_canonical_b200/csrc/dfw_internal.h"]
+# the sources that define each decode kernel (a change to any of them makes a
+# committed traffic figure stale)
+_CSRC = "lossless_entropy_coded_canonical_b200/csrc/"
+KERNEL_SOURCES = {
+    "decode_lanes": [_CSRC + "dfw_lanes.cuh", _CSRC + "dfw_device.cuh", _CSRC + "dfw_internal.h"],
+    "decode_tiles": [_CSRC + "dfw_decode.cu", _CSRC + "dfw_device.cuh", _CSRC + "dfw_internal.h"],
+}
 
 
 # ------------------------------------------------------------------ helpers
@@ -55,9 +58,9 @@ def workload_blocks(name: str):
     return [table[name]], f"{name} ({table[name].numel} weights)"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str = "decode_lanes") -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -84,7 +87,7 @@ def committed_traffic(kernel: str):
         if ":" in line and not line.startswith("#"):
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
-    if kv.get("kernel_source_sha256_16") != kernel_source_hash():
+    if kv.get("kernel_source_sha256_16") != kernel_source_hash(kernel):
         return None
     try:
         return float(kv["dram_bytes_per_weight"])
