@@ -297,6 +297,59 @@ dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, cons
                             void *cuda_stream);
 
 /*
+ * CONTAINER -- the encoded artefact (a tensor, or a block of tensors with
+ * one table) as one byte buffer, to store it and decode it later.  The
+ * pages ship entropy-coded models (DFloat11 abstract) but give no file
+ * format; this one is the library's own.  All integers little-endian; every
+ * section starts on a 16-byte boundary (zero padding between sections):
+ *   0    8   magic "DFWBF16\0"
+ *   8    4   DFW_FORMAT_VERSION
+ *   12   4   flags: bit 0 = the known-start plan is present
+ *   16   4   cap          20  4  n_symbols     24  4  single_symbol
+ *   28   4   k (tensors, >= 1)
+ *   32   8   n            40  8  total_bits    48  8  stream_bytes
+ *   56   256 code lengths (dfw_table.len)
+ *   then     (k + 1) u64 tensor offsets (first 0, last n)
+ *   then     the stream (stream_bytes), then the raw bytes (dfw_mant_bytes(n))
+ *   then     [plan] 32 * n_groups u16 chunk_bits, n_groups + 1 u64 group_start
+ *   last 8   FNV-1a 64-bit hash of every byte before it
+ * The LUT is not stored: dfw_lanes_lut rebuilds it from the lengths.
+ */
+
+/* Bytes of the container for this table and k tensors, with or without the
+ * known-start plan; 0 for a bad argument. */
+uint64_t dfw_container_bytes(const dfw_table *table, int k, int with_plan);
+
+/*
+ * dfw_container_write -- host: serialises an encoded tensor or block into
+ * out (out_bytes >= dfw_container_bytes(...)).  tensor_offsets: k + 1
+ * entries (NULL for k = 1); stream and mant as dfw_encode wrote them;
+ * chunk_bits and group_start both NULL (no plan) or both as dfw_plan_lanes
+ * wrote them.  Errors: DFW_EINVAL (bad table or arguments), DFW_ENOMEM (out
+ * too small).
+ */
+dfw_status dfw_container_write(const dfw_table *table, int k, const uint64_t *tensor_offsets,
+                               const uint8_t *stream, const uint8_t *mant, const uint16_t *chunk_bits,
+                               const uint64_t *group_start, uint8_t *out, uint64_t out_bytes);
+
+/* Where dfw_container_read found the sections: byte offsets into the buffer
+ * (chunk_bits_at and group_start_at are 0 without a plan). */
+typedef struct dfw_container_view {
+    int32_t k;
+    int32_t has_plan;
+    uint64_t offsets_at, stream_at, mant_at, chunk_bits_at, group_start_at;
+} dfw_container_view;
+
+/*
+ * dfw_container_read -- host: checks a container (magic, version, size,
+ * hash, table, tensor offsets, and that the plan's chunk bits add up to its
+ * group starts) and fills *table and *view; the data stay in buf.  Errors:
+ * DFW_EINVAL (NULL arguments or another format version), DFW_ECORRUPT (any
+ * check fails).
+ */
+dfw_status dfw_container_read(const uint8_t *buf, uint64_t bytes, dfw_table *table, dfw_container_view *view);
+
+/*
  * dfw_lanes_scope -- one code-table scope of a sequence: the arguments of a
  * dfw_decode_lanes call other than the output and the stream (device
  * buffers as there; table and info in host memory).

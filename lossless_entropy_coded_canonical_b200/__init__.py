@@ -22,12 +22,12 @@ import numpy as np
 import torch
 
 from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT,
-                   DfwError, LanesInfo, LanesScope, PlanInfo, RansTable, Table, check as _check, lib)
+                   ContainerView, DfwError, LanesInfo, LanesScope, PlanInfo, RansTable, Table, check as _check, lib)
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
            "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "decode_lanes_seq", "LanesInfo",
            "encode_device", "encode_device_scratch_bytes", "decode_gemv_lanes",
-           "rans_encode", "RansEncoded", "DeviceRans", "rans_decode", "RansTable",
+           "rans_encode", "RansEncoded", "DeviceRans", "rans_decode", "RansTable", "save", "load",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
            "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
 
@@ -459,3 +459,63 @@ def status_bits(stream=None) -> tuple[int, int]:
     bits = ctypes.c_uint32(0)
     st = int(lib().dfw_status_bits(_stream_handle(stream), ctypes.byref(bits)))
     return st, int(bits.value)
+
+
+# ------------------------------------------------------------------ container
+
+def save(path, enc: Encoded, plan: LanesPlan | None = None) -> int:
+    """Writes an encoded tensor or block (and optionally its known-start
+    plan) to ``path`` as one container (dfw_container_write); returns the
+    number of bytes written."""
+    k = 1 if enc.tensor_offsets is None else int(enc.tensor_offsets.size - 1)
+    offs = None if enc.tensor_offsets is None else np.ascontiguousarray(enc.tensor_offsets, dtype=np.uint64)
+    size = int(lib().dfw_container_bytes(ctypes.byref(enc.table), k, plan is not None))
+    if size == 0:
+        raise DfwError(EINVAL, "dfw_container_bytes")
+    out = np.empty(size, dtype=np.uint8)
+    cb = gs = None
+    if plan is not None:
+        cb, gs = _ptr(plan.chunk_bits.contiguous()), _ptr(plan.group_start.contiguous())
+    _check(lib().dfw_container_write(ctypes.byref(enc.table), k, None if offs is None else _ptr(offs),
+                                     _ptr(enc.stream.contiguous()), _ptr(enc.mant.contiguous()), cb, gs,
+                                     _ptr(out), size), "dfw_container_write")
+    with open(path, "wb") as f:
+        f.write(out.tobytes())
+    return size
+
+
+def load(path):
+    """Reads a container written by :func:`save`; returns (Encoded, LanesPlan
+    or None), host tensors viewing the file's bytes (the LUT is rebuilt from
+    the code lengths)."""
+    with open(path, "rb") as f:
+        buf = np.frombuffer(f.read(), dtype=np.uint8).copy()
+    table, view = Table(), ContainerView()
+    _check(lib().dfw_container_read(_ptr(buf), buf.size, ctypes.byref(table), ctypes.byref(view)),
+           "dfw_container_read")
+    raw = torch.from_numpy(buf)
+    n, k = int(table.n), int(view.k)
+    offs = buf[view.offsets_at: view.offsets_at + 8 * (k + 1)].view(np.uint64).copy()
+    stream = raw[view.stream_at: view.stream_at + int(table.stream_bytes)]
+    mant = raw[view.mant_at: view.mant_at + mant_bytes(n)]
+    enc = Encoded(stream, mant, table, offs if k > 1 else None)
+    if not view.has_plan:
+        return enc, None
+    info = LanesInfo()
+    _check(lib().dfw_plan_lanes_query(ctypes.byref(table), ctypes.byref(info)), "dfw_plan_lanes_query")
+    ng = int(info.n_groups)
+    cb = torch.from_numpy(buf[view.chunk_bits_at: view.chunk_bits_at + 64 * ng].view(np.int16).copy())
+    gs = torch.from_numpy(buf[view.group_start_at: view.group_start_at + 8 * (ng + 1)].view(np.int64).copy())
+    if cb.numel() == 0:
+        cb = torch.zeros(1, dtype=torch.int16)
+    # the largest group span, as dfw_plan_lanes reports it
+    g = gs.numpy().view(np.uint64)
+    if ng:
+        b0 = (g[:-1] >> np.uint64(3)) & ~np.uint64(15)
+        b1 = (((g[1:] + np.uint64(7)) >> np.uint64(3)) + np.uint64(8 + 15)) & ~np.uint64(15)
+        info.max_group_bytes = max(16, int((b1 - b0).max()))
+    else:
+        info.max_group_bytes = 16
+    lut = torch.empty(int(info.lut_words), dtype=torch.int32)
+    _check(lib().dfw_lanes_lut(ctypes.byref(table), ctypes.byref(info), _ptr(lut)), "dfw_lanes_lut")
+    return enc, LanesPlan(cb, gs, lut, info)

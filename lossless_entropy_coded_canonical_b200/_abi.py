@@ -47,6 +47,13 @@ class LanesScope(ctypes.Structure):
                 ("table", ctypes.POINTER(Table)), ("info", ctypes.POINTER(LanesInfo))]
 
 
+class ContainerView(ctypes.Structure):
+    """dfw_container_view: where dfw_container_read found each section."""
+    _fields_ = [("k", ctypes.c_int32), ("has_plan", ctypes.c_int32), ("offsets_at", ctypes.c_uint64),
+                ("stream_at", ctypes.c_uint64), ("mant_at", ctypes.c_uint64), ("chunk_bits_at", ctypes.c_uint64),
+                ("group_start_at", ctypes.c_uint64)]
+
+
 class RansTable(ctypes.Structure):
     _fields_ = [("version", ctypes.c_uint32), ("scale_bits", ctypes.c_uint32), ("lanes", ctypes.c_uint32),
                 ("block_syms", ctypes.c_uint32), ("n", ctypes.c_uint64), ("n_blocks", ctypes.c_uint64),
@@ -74,6 +81,9 @@ SIGNATURES = {
     "dfw_decode_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _vp, _vp]),
     "dfw_decode_lanes_seq": (_i, [_i, _vp, _vp, _vp]),
     "dfw_status_bits": (_i, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "dfw_container_bytes": (_u64, [_TP, _i, _i]),
+    "dfw_container_write": (_i, [_TP, _i, _vp, _vp, _vp, _vp, _vp, _vp, _u64]),
+    "dfw_container_read": (_i, [_vp, _u64, _TP, ctypes.POINTER(ContainerView)]),
     "dfw_selftest_wait_timeout": (_i, [_vp]),
     "dfw_decode_gemv_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _i, _vp, _vp, _vp, _vp, _vp, _u64, _vp]),
     "dfw_encode_device_scratch_bytes": (_u64, [_u64]),

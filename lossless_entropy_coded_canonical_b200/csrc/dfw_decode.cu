@@ -439,6 +439,7 @@ using namespace dfw;
 extern "C" dfw_status dfw_decode(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
                                  const uint8_t *d_gap, const uint64_t *d_out_start, const dfw_table *table,
                                  const dfw_plan_info *info, uint16_t *d_out, void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_decode");
     return launch_decode(d_stream, d_mant, d_lut, d_gap, d_out_start, table, info, d_out,
                          static_cast<cudaStream_t>(cuda_stream));
 }
@@ -448,6 +449,7 @@ extern "C" dfw_status dfw_decode_block(const uint8_t *d_stream, const uint8_t *d
                                        const dfw_table *table, const dfw_plan_info *info,
                                        const uint64_t *tensor_offsets, int k, uint16_t *d_scratch,
                                        uint64_t scratch_elems, void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_decode_block");
     if (!table || !tensor_offsets || k < 1) return DFW_EINVAL;
     if (tensor_offsets[0] != 0 || tensor_offsets[k] != table->n) return DFW_EINVAL;
     for (int i = 0; i < k; ++i)
@@ -461,6 +463,7 @@ extern "C" dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d
                                        const uint16_t *d_chunk_bits, const uint64_t *d_group_start,
                                        const dfw_table *table, const dfw_lanes_info *info, uint16_t *d_out,
                                        void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_decode_lanes");
     dfw_status st = validate_table(table);
     if (st != DFW_OK) return st;
     if (!info) return DFW_EINVAL;
@@ -482,6 +485,7 @@ extern "C" dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d
 }
 
 extern "C" dfw_status dfw_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_decode_lanes_seq");
     if (k < 0 || (k > 0 && (!scopes || !d_out))) return DFW_EINVAL;
     if (k == 0) return DFW_OK;
     if (reinterpret_cast<uintptr_t>(d_out) & 15u) return DFW_EALIGN;
@@ -498,6 +502,7 @@ extern "C" dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8
                                             const uint64_t *tensor_offsets, const uint32_t *cols,
                                             const uint16_t *const *d_x, float *const *d_y, float *d_partial,
                                             uint64_t partial_elems, void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_decode_gemv_lanes");
     dfw_status st = validate_table(table);
     if (st != DFW_OK) return st;
     if (!info || table->n == 0) return DFW_EINVAL;
@@ -511,6 +516,7 @@ extern "C" dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8
 
 extern "C" dfw_status dfw_rans_decode(const uint8_t *d_stream, const uint8_t *d_mant, const uint64_t *d_block_start,
                                       const dfw_rans_table *table, uint16_t *d_out, void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_rans_decode");
     if (!table || table->version != DFW_FORMAT_VERSION || table->scale_bits != DFW_RANS_SCALE_BITS ||
         table->lanes != DFW_RANS_LANES || table->block_syms != DFW_RANS_BLOCK ||
         table->n_blocks != (table->n + DFW_RANS_BLOCK - 1) / DFW_RANS_BLOCK)

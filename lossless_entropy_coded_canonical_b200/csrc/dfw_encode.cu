@@ -413,6 +413,7 @@ extern "C" dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int 
                                         uint16_t *d_chunk_bits, uint64_t *d_group_start, void *d_scratch,
                                         uint64_t scratch_bytes, dfw_table *table, dfw_lanes_info *info,
                                         void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_encode_device");
     if (!table || !info || cap < 1 || cap > DFW_MAX_CAP) return DFW_EINVAL;
     const uint32_t fb = info->fast_bits;
     std::memset(table, 0, sizeof(*table));
@@ -514,6 +515,7 @@ extern "C" dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int 
 extern "C" dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *table, const dfw_lanes_info *info,
                                       const uint64_t *d_group_start, uint8_t *d_stream, uint64_t stream_capacity,
                                       void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_pack_device");
     dfw_status st = validate_table(table);
     if (st != DFW_OK) return st;
     if (!info || !d_stream) return DFW_EINVAL;

@@ -394,6 +394,7 @@ extern "C" uint64_t dfw_mant_bytes(uint64_t n) { return (n + 15) & ~15ull; }
 extern "C" dfw_status dfw_encode(const uint16_t *bf16, uint64_t n, int cap, uint8_t *stream,
                                  uint64_t stream_capacity, uint8_t *mant, uint64_t mant_capacity,
                                  dfw_table *table, int n_threads) {
+    dfw::NvtxRange nvtx_range("dfw_encode");
     if (n && !bf16) return DFW_EINVAL;
     Segments seg{&bf16, &n, 1, {0, n}};
     return encode_segments(seg, cap, stream, stream_capacity, mant, mant_capacity, table, n_threads);
@@ -403,6 +404,7 @@ extern "C" dfw_status dfw_encode_multi(const uint16_t *const *tensors, const uin
                                        int cap, uint8_t *stream, uint64_t stream_capacity,
                                        uint8_t *mant, uint64_t mant_capacity, dfw_table *table,
                                        uint64_t *tensor_offsets, int n_threads) {
+    dfw::NvtxRange nvtx_range("dfw_encode_multi");
     if (k < 1 || !tensors || !sizes || !tensor_offsets) return DFW_EINVAL;
     Segments seg{tensors, sizes, k, std::vector<uint64_t>(k + 1, 0)};
     for (int i = 0; i < k; ++i) {
@@ -457,6 +459,7 @@ extern "C" dfw_status dfw_plan_query(const dfw_table *table, uint32_t window_byt
 
 extern "C" dfw_status dfw_plan(const uint8_t *stream, const dfw_table *table, uint8_t *gap,
                                uint64_t *out_start, uint32_t *lut, dfw_plan_info *info) {
+    dfw::NvtxRange nvtx_range("dfw_plan");
     if (!info || !out_start || !lut) return DFW_EINVAL;
     dfw_plan_info q;
     q.fast_bits = info->fast_bits;
@@ -608,6 +611,7 @@ extern "C" dfw_status dfw_plan_lanes_query(const dfw_table *table, dfw_lanes_inf
 
 extern "C" dfw_status dfw_plan_lanes(const uint8_t *stream, const dfw_table *table, uint16_t *chunk_bits,
                                      uint64_t *group_start, uint32_t *lut, dfw_lanes_info *info) {
+    dfw::NvtxRange nvtx_range("dfw_plan_lanes");
     if (!info || !group_start || !lut) return DFW_EINVAL;
     dfw_lanes_info q;
     q.fast_bits = info->fast_bits;
@@ -678,5 +682,176 @@ extern "C" dfw_status dfw_lanes_lut(const dfw_table *table, const dfw_lanes_info
     if (st != DFW_OK) return st;
     std::memcpy(lut, fast.data(), fast.size() * sizeof(uint32_t));
     std::memcpy(lut + fast.size(), img.data(), img.size() * sizeof(uint32_t));
+    return DFW_OK;
+}
+
+// ------------------------------------------------------------ container
+//
+// The encoded artefact as one byte buffer (layout in include/dfw.h): a fixed
+// header of little-endian fields, the tensor offsets, the stream, the raw
+// bytes and, optionally, the known-start plan; every section starts on a
+// 16-byte boundary; an FNV-1a 64-bit hash of all earlier bytes closes it.
+
+namespace {
+
+constexpr uint64_t CONT_HEADER = 312;  // magic .. code lengths
+constexpr char CONT_MAGIC[8] = {'D', 'F', 'W', 'B', 'F', '1', '6', '\0'};
+
+uint64_t up16(uint64_t x) { return (x + 15) & ~15ull; }
+
+struct ContLayout {
+    uint64_t offsets_at, stream_at, mant_at, chunk_bits_at, group_start_at, hash_at, total;
+};
+
+// Section offsets; false if a size overflows.
+bool cont_layout(uint64_t n, uint64_t stream_bytes, uint64_t k, bool plan, ContLayout &L) {
+    if (k == 0 || k > (1ull << 32) || n > (1ull << 56) || stream_bytes > (1ull << 56)) return false;
+    const uint64_t n_chunks = (n + LANE_SYMS - 1) / LANE_SYMS;
+    const uint64_t n_groups = (n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+    L.offsets_at = up16(CONT_HEADER);
+    L.stream_at = up16(L.offsets_at + 8 * (k + 1));
+    L.mant_at = up16(L.stream_at + stream_bytes);
+    uint64_t end = L.mant_at + ((n + 15) & ~15ull);
+    L.chunk_bits_at = L.group_start_at = 0;
+    if (plan) {
+        L.chunk_bits_at = up16(end);
+        L.group_start_at = up16(L.chunk_bits_at + 2 * (uint64_t)GROUP_CHUNKS * n_groups);
+        end = L.group_start_at + 8 * (n_groups + 1);
+    }
+    L.hash_at = up16(end);
+    L.total = L.hash_at + 8;
+    return true;
+}
+
+uint64_t fnv1a64(const uint8_t *p, uint64_t bytes) {
+    uint64_t h = 0xcbf29ce484222325ull;
+    for (uint64_t i = 0; i < bytes; ++i) {
+        h ^= p[i];
+        h *= 0x100000001b3ull;
+    }
+    return h;
+}
+
+void put32(uint8_t *p, uint32_t v) {
+    for (int i = 0; i < 4; ++i) p[i] = (uint8_t)(v >> (8 * i));
+}
+void put64(uint8_t *p, uint64_t v) {
+    for (int i = 0; i < 8; ++i) p[i] = (uint8_t)(v >> (8 * i));
+}
+uint32_t get32(const uint8_t *p) {
+    uint32_t v = 0;
+    for (int i = 0; i < 4; ++i) v |= (uint32_t)p[i] << (8 * i);
+    return v;
+}
+uint64_t get64(const uint8_t *p) {
+    uint64_t v = 0;
+    for (int i = 0; i < 8; ++i) v |= (uint64_t)p[i] << (8 * i);
+    return v;
+}
+
+}  // namespace
+
+extern "C" uint64_t dfw_container_bytes(const dfw_table *table, int k, int with_plan) {
+    if (!table || k < 1) return 0;
+    ContLayout L;
+    if (!cont_layout(table->n, table->stream_bytes, (uint64_t)k, with_plan != 0, L)) return 0;
+    return L.total;
+}
+
+extern "C" dfw_status dfw_container_write(const dfw_table *table, int k, const uint64_t *tensor_offsets,
+                                          const uint8_t *stream, const uint8_t *mant, const uint16_t *chunk_bits,
+                                          const uint64_t *group_start, uint8_t *out, uint64_t out_bytes) {
+    dfw::NvtxRange nvtx_range("dfw_container_write");
+    dfw_status st = validate_table(table);
+    if (st != DFW_OK) return st;
+    if (k < 1 || !out || (table->stream_bytes && !stream) || (table->n && !mant)) return DFW_EINVAL;
+    if ((chunk_bits == nullptr) != (group_start == nullptr)) return DFW_EINVAL;
+    const bool plan = chunk_bits != nullptr;
+    ContLayout L;
+    if (!cont_layout(table->n, table->stream_bytes, (uint64_t)k, plan, L)) return DFW_EINVAL;
+    if (out_bytes < L.total) return DFW_ENOMEM;
+    if (tensor_offsets) {
+        if (tensor_offsets[0] != 0 || tensor_offsets[k] != table->n) return DFW_EINVAL;
+        for (int i = 0; i < k; ++i)
+            if (tensor_offsets[i + 1] < tensor_offsets[i]) return DFW_EINVAL;
+    } else if (k != 1) {
+        return DFW_EINVAL;
+    }
+    std::memset(out, 0, L.total);
+    std::memcpy(out, CONT_MAGIC, 8);
+    put32(out + 8, DFW_FORMAT_VERSION);
+    put32(out + 12, plan ? 1u : 0u);
+    put32(out + 16, table->cap);
+    put32(out + 20, table->n_symbols);
+    put32(out + 24, table->single_symbol);
+    put32(out + 28, (uint32_t)k);
+    put64(out + 32, table->n);
+    put64(out + 40, table->total_bits);
+    put64(out + 48, table->stream_bytes);
+    std::memcpy(out + 56, table->len, 256);
+    for (int i = 0; i <= k; ++i)
+        put64(out + L.offsets_at + 8 * i, tensor_offsets ? tensor_offsets[i] : (i ? table->n : 0));
+    if (table->stream_bytes) std::memcpy(out + L.stream_at, stream, table->stream_bytes);
+    if (table->n) std::memcpy(out + L.mant_at, mant, (table->n + 15) & ~15ull);
+    if (plan) {
+        const uint64_t n_groups = ((table->n + LANE_SYMS - 1) / LANE_SYMS + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+        for (uint64_t i = 0; i < (uint64_t)GROUP_CHUNKS * n_groups; ++i) {
+            out[L.chunk_bits_at + 2 * i] = (uint8_t)chunk_bits[i];
+            out[L.chunk_bits_at + 2 * i + 1] = (uint8_t)(chunk_bits[i] >> 8);
+        }
+        for (uint64_t g = 0; g <= n_groups; ++g) put64(out + L.group_start_at + 8 * g, group_start[g]);
+    }
+    put64(out + L.hash_at, fnv1a64(out, L.hash_at));
+    return DFW_OK;
+}
+
+extern "C" dfw_status dfw_container_read(const uint8_t *buf, uint64_t bytes, dfw_table *table,
+                                         dfw_container_view *view) {
+    dfw::NvtxRange nvtx_range("dfw_container_read");
+    if (!buf || !table || !view) return DFW_EINVAL;
+    if (bytes < CONT_HEADER + 8 || std::memcmp(buf, CONT_MAGIC, 8) != 0) return DFW_ECORRUPT;
+    if (get32(buf + 8) != DFW_FORMAT_VERSION) return DFW_EINVAL;
+    const uint32_t flags = get32(buf + 12);
+    if (flags & ~1u) return DFW_ECORRUPT;
+    const uint64_t k = get32(buf + 28), n = get64(buf + 32), stream_bytes = get64(buf + 48);
+    ContLayout L;
+    if (!cont_layout(n, stream_bytes, k, flags & 1u, L) || L.total != bytes) return DFW_ECORRUPT;
+    if (get64(buf + L.hash_at) != fnv1a64(buf, L.hash_at)) return DFW_ECORRUPT;
+    dfw_table t;
+    std::memset(&t, 0, sizeof(t));
+    t.version = DFW_FORMAT_VERSION;
+    t.cap = get32(buf + 16);
+    t.n_symbols = get32(buf + 20);
+    t.single_symbol = get32(buf + 24);
+    t.n = n;
+    t.total_bits = get64(buf + 40);
+    t.stream_bytes = stream_bytes;
+    std::memcpy(t.len, buf + 56, 256);
+    if (validate_table(&t) != DFW_OK) return DFW_ECORRUPT;
+    if (get64(buf + L.offsets_at) != 0 || get64(buf + L.offsets_at + 8 * k) != n) return DFW_ECORRUPT;
+    for (uint64_t i = 0; i < k; ++i)
+        if (get64(buf + L.offsets_at + 8 * (i + 1)) < get64(buf + L.offsets_at + 8 * i)) return DFW_ECORRUPT;
+    if (flags & 1u) {  // the plan must agree with itself and with the table
+        const uint64_t n_groups = ((n + LANE_SYMS - 1) / LANE_SYMS + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+        if (get64(buf + L.group_start_at) != 0 || get64(buf + L.group_start_at + 8 * n_groups) != t.total_bits)
+            return DFW_ECORRUPT;
+        for (uint64_t g = 0; g < n_groups; ++g) {
+            uint64_t s = 0;
+            for (uint32_t c = 0; c < GROUP_CHUNKS; ++c) {
+                const uint64_t at = L.chunk_bits_at + 2 * ((uint64_t)GROUP_CHUNKS * g + c);
+                s += (uint64_t)buf[at] | ((uint64_t)buf[at + 1] << 8);
+            }
+            if (get64(buf + L.group_start_at + 8 * (g + 1)) - get64(buf + L.group_start_at + 8 * g) != s)
+                return DFW_ECORRUPT;
+        }
+    }
+    *table = t;
+    view->k = (int)k;
+    view->has_plan = (int)(flags & 1u);
+    view->offsets_at = L.offsets_at;
+    view->stream_at = L.stream_at;
+    view->mant_at = L.mant_at;
+    view->chunk_bits_at = L.chunk_bits_at;
+    view->group_start_at = L.group_start_at;
     return DFW_OK;
 }

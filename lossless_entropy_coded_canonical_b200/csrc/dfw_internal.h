@@ -6,6 +6,8 @@
 
 #include "../../include/dfw.h"
 
+#include <nvtx3/nvToolsExt.h>
+
 namespace dfw {
 
 // LUT entry (32 bits).  Pointer entries: LUT_PTR | child table index.  Leaf
@@ -47,6 +49,15 @@ constexpr uint32_t ST_COUNT = 1u;   // a tile decoded a different number of code
 constexpr uint32_t ST_LUT = 2u;     // a LUT pointer left the table or a code ran past four levels
 constexpr uint32_t ST_RANGE = 4u;   // out_start out of order or beyond n, or tile too large
 constexpr uint32_t ST_TIMEOUT = 8u; // a wait for a bulk copy gave up (the kernel returned early)
+
+// A named range on profiler timelines (NVTX) for the duration of a call;
+// costs a function-pointer check when no tool is attached.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 dfw_status code_lengths(const uint64_t hist[256], int cap, uint8_t len[256]);
 void canonical_codes(const uint8_t len[256], uint32_t code[256]);

@@ -89,6 +89,7 @@ extern "C" dfw_status dfw_rans_encode(const uint16_t *const *tensors, const uint
                                       uint8_t *stream, uint64_t stream_capacity, uint8_t *mant,
                                       uint64_t mant_capacity, uint64_t *block_start, dfw_rans_table *table,
                                       int n_threads) {
+    dfw::NvtxRange nvtx_range("dfw_rans_encode");
     if (!table || k < 0 || (k && (!tensors || !sizes))) return DFW_EINVAL;
     uint64_t n = 0;
     for (int t = 0; t < k; ++t) {
