@@ -25,10 +25,12 @@
 // realignment: every chunk's output is 64-weight aligned.
 //
 // Bounds: a lane makes at most 64 lookups per chunk (each yields >= 1
-// codeword); stream reads are clamped to the slot; a group whose chunk_bits
-// do not add up to its group_start span, or whose lanes do not end exactly
-// where chunk_bits says, writes nothing and sets a status bit; waits on bulk
-// copies are bounded.
+// codeword; an escape resolves one codeword of at most 32 bits), so its
+// stream reads end within 2048 bits and a few words of its start: a corrupt
+// stream can read past its slot but not past the warp's own shared-memory
+// area; a group whose chunk_bits do not add up to its group_start span, or
+// whose lanes do not end exactly where chunk_bits says, writes nothing and
+// sets a status bit; waits on bulk copies are bounded.
 #pragma once
 
 #include <cstring>
