@@ -22,6 +22,7 @@ import ctypes
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -58,11 +59,20 @@ def workload_blocks(name: str):
     return [table[name]], f"{name} ({table[name].numel} weights)"
 
 
+def _code_only(src: str) -> str:
+    """Source text without comments and with whitespace collapsed, so that
+    editing a comment does not mark a committed measurement stale (none of
+    these files has // or /* inside a string literal)."""
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_source_hash(kernel: str = "decode_lanes") -> str:
     h = hashlib.sha256()
     for p in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, p), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 
