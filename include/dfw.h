@@ -471,6 +471,49 @@ dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *table, const
 dfw_status dfw_lanes_lut(const dfw_table *table, const dfw_lanes_info *info, uint32_t *lut);
 
 /*
+ * dfw_encode_device_multi -- the first call for k scopes (the blocks of a
+ * model, each with its own code), with the host's share of each scope
+ * overlapped with the GPU's work on the next: pass 1 of scope i + 1 is
+ * queued before the host waits for scope i's histogram, builds its code and
+ * queues its counting passes.  The pages describe the encoder only as an
+ * offline step; this call only schedules that step better.
+ *   scopes         host array of k dfw_encode_scope: per scope the d_bf16, n,
+ *                  d_mant, d_chunk_bits, d_group_start of dfw_encode_device
+ *   cap            length cap, 1..32, for every scope
+ *   d_scratch      device, scratch_bytes >= k * dfw_encode_device_scratch_bytes(0);
+ *                  scope i uses the i-th such slice
+ *   h_staging      host, staging_bytes >= dfw_encode_device_multi_staging_bytes(k),
+ *                  8-byte aligned: where each scope's histogram and totals are
+ *                  read back.  Page-locked memory (cudaHostAlloc) lets the copies
+ *                  run ahead of the host; pageable memory gives the same results,
+ *                  but each copy then waits for all earlier work
+ *   tables, infos  host arrays of k: outputs (infos[i].fast_bits is read first),
+ *                  each exactly what dfw_encode_device gives for scope i alone
+ * Every scope is checked before anything is launched (an error then leaves
+ * the device outputs untouched; tables and infos are unspecified).  An error
+ * found later (DFW_ECAP: 2^cap is smaller
+ * than a scope's number of exponents; DFW_ECUDA) stops the queueing; the
+ * call still waits for the work already queued, and the outputs are then
+ * unspecified.  In all cases cuda_stream is idle when the call returns (it
+ * synchronises once per non-empty scope and once at the end).  Then
+ * dfw_pack_device per scope, as after dfw_encode_device.  Errors: DFW_EINVAL,
+ * DFW_EALIGN, DFW_ENOMEM (scratch or staging too small), DFW_ECAP, DFW_ECUDA.
+ */
+typedef struct dfw_encode_scope {
+    const uint16_t *d_bf16;
+    uint64_t n;
+    uint8_t *d_mant;
+    uint16_t *d_chunk_bits;
+    uint64_t *d_group_start;
+} dfw_encode_scope;
+
+uint64_t dfw_encode_device_multi_staging_bytes(uint32_t k);
+
+dfw_status dfw_encode_device_multi(uint32_t k, const dfw_encode_scope *scopes, int cap, void *d_scratch,
+                                   uint64_t scratch_bytes, void *h_staging, uint64_t staging_bytes,
+                                   dfw_table *tables, dfw_lanes_info *infos, void *cuda_stream);
+
+/*
  * dfw_encode_device_noalloc -- dfw_encode_device without a scratch argument,
  * for callers that cannot allocate device memory when they encode: a serving
  * runtime that reserves all of the GPU's memory at start-up and allows no

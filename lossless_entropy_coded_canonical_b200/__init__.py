@@ -22,11 +22,11 @@ import numpy as np
 import torch
 
 from ._abi import (EALIGN, ECAP, ECORRUPT, ECUDA, EINVAL, ENOMEM, OK, ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT,
-                   ContainerView, DfwError, LanesInfo, LanesScope, PlanInfo, RansTable, Table, check as _check, lib)
+                   ContainerView, DfwError, EncodeScope, LanesInfo, LanesScope, PlanInfo, RansTable, Table, check as _check, lib)
 
 __all__ = ["encode", "encode_multi", "plan", "DeviceCompressed", "decode", "decode_block", "check",
            "plan_lanes", "LanesPlan", "DeviceLanes", "decode_lanes", "decode_lanes_seq", "LanesInfo",
-           "encode_device", "encode_device_scratch_bytes", "decode_gemv_lanes",
+           "encode_device", "encode_device_multi", "encode_device_scratch_bytes", "decode_gemv_lanes",
            "rans_encode", "RansEncoded", "DeviceRans", "rans_decode", "RansTable", "save", "load",
            "Encoded", "Plan", "Table", "PlanInfo", "DfwError", "lib", "mant_bytes", "stream_bound",
            "OK", "EINVAL", "ECAP", "ENOMEM", "ECORRUPT", "EALIGN", "ECUDA"]
@@ -332,16 +332,8 @@ def encode_device(x: torch.Tensor, cap: int = 32, fast_bits: int = 0, stream=Non
     uploaded.  Returns a :class:`DeviceLanes` ready for :func:`decode_lanes`.
     ``scratch`` (uint8, at least ``encode_device_scratch_bytes()``) may be
     passed to reuse one buffer across calls."""
-    if not x.is_cuda:
-        raise ValueError("encode_device takes a CUDA tensor")
-    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
-        raise TypeError(f"expected bf16 bit patterns, got {x.dtype}")
-    x = x.contiguous().reshape(-1)
+    x, mant, chunk_bits, group_start = _device_outputs(x)
     dev, n = x.device, x.numel()
-    n_groups = -(-(-(-n // 64)) // 32)
-    mant = torch.empty(mant_bytes(n), dtype=torch.uint8, device=dev)
-    chunk_bits = torch.empty(32 * n_groups, dtype=torch.int16, device=dev)
-    group_start = torch.empty(n_groups + 1, dtype=torch.int64, device=dev)
     need = encode_device_scratch_bytes()
     if scratch is None:
         scratch = torch.empty(need, dtype=torch.uint8, device=dev)
@@ -353,12 +345,64 @@ def encode_device(x: torch.Tensor, cap: int = 32, fast_bits: int = 0, stream=Non
     _check(lib().dfw_encode_device(_ptr(x), n, cap, _ptr(mant), _ptr(chunk_bits), _ptr(group_start),
                                    _ptr(scratch), scratch.numel() * scratch.element_size(), ctypes.byref(table),
                                    ctypes.byref(info), sh), "dfw_encode_device")
-    stream_buf = torch.empty(int(table.stream_bytes), dtype=torch.uint8, device=dev)
+    return _pack_device(x, mant, chunk_bits, group_start, table, info, sh)
+
+
+def _device_outputs(x: torch.Tensor):
+    if not x.is_cuda:
+        raise ValueError("encode_device takes a CUDA tensor")
+    if x.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"expected bf16 bit patterns, got {x.dtype}")
+    x = x.contiguous().reshape(-1)
+    n = x.numel()
+    n_groups = -(-(-(-n // 64)) // 32)
+    return (x, torch.empty(mant_bytes(n), dtype=torch.uint8, device=x.device),
+            torch.empty(32 * n_groups, dtype=torch.int16, device=x.device),
+            torch.empty(n_groups + 1, dtype=torch.int64, device=x.device))
+
+
+def _pack_device(x, mant, chunk_bits, group_start, table, info, sh) -> DeviceLanes:
+    """Second call (dfw_pack_device) and the LUT image, after the first."""
+    stream_buf = torch.empty(int(table.stream_bytes), dtype=torch.uint8, device=x.device)
     _check(lib().dfw_pack_device(_ptr(x), ctypes.byref(table), ctypes.byref(info), _ptr(group_start),
                                  _ptr(stream_buf), stream_buf.numel(), sh), "dfw_pack_device")
     lut = torch.empty(int(info.lut_words), dtype=torch.int32)
     _check(lib().dfw_lanes_lut(ctypes.byref(table), ctypes.byref(info), _ptr(lut.numpy())), "dfw_lanes_lut")
-    return DeviceLanes(stream_buf, mant, lut.to(dev), chunk_bits, group_start, table, info, None)
+    return DeviceLanes(stream_buf, mant, lut.to(x.device), chunk_bits, group_start, table, info, None)
+
+
+def encode_device_multi(xs, cap: int = 32, fast_bits: int = 0, stream=None,
+                        pinned_staging: bool = True) -> list[DeviceLanes]:
+    """Encodes several bf16 tensors already on the GPU, each with its own
+    code (``dfw_encode_device_multi``, then ``dfw_pack_device`` per tensor):
+    the host builds tensor i's code while the GPU runs tensor i + 1's
+    histogram pass.  Each result equals :func:`encode_device` of that tensor
+    alone.  ``pinned_staging=False`` reads the histograms back through
+    pageable memory (same results, no overlap)."""
+    outs = [_device_outputs(x) for x in xs]
+    k = len(outs)
+    if k == 0:
+        return []
+    dev = outs[0][0].device
+    arr = (EncodeScope * k)()
+    for i, (x, mant, cb, gs) in enumerate(outs):
+        if x.device != dev:
+            raise ValueError("all tensors must be on one device")
+        arr[i] = EncodeScope(_ptr(x), x.numel(), _ptr(mant), _ptr(cb), _ptr(gs))
+    scratch = torch.empty(k * encode_device_scratch_bytes(), dtype=torch.uint8, device=dev)
+    staging = torch.empty(int(lib().dfw_encode_device_multi_staging_bytes(k)), dtype=torch.uint8,
+                          pin_memory=pinned_staging)
+    tables, infos = (Table * k)(), (LanesInfo * k)()
+    for i in range(k):
+        infos[i].fast_bits = fast_bits
+    sh = _stream_handle(stream)
+    _check(lib().dfw_encode_device_multi(k, arr, cap, _ptr(scratch), scratch.numel(), staging.data_ptr(),
+                                         staging.numel(), tables, infos, sh), "dfw_encode_device_multi")
+    res = []
+    for i, (x, mant, cb, gs) in enumerate(outs):
+        t, inf = Table.from_buffer_copy(tables[i]), LanesInfo.from_buffer_copy(infos[i])
+        res.append(_pack_device(x, mant, cb, gs, t, inf, sh))
+    return res
 
 
 def encode_device_scratch_bytes() -> int:

@@ -47,6 +47,12 @@ class LanesScope(ctypes.Structure):
                 ("table", ctypes.POINTER(Table)), ("info", ctypes.POINTER(LanesInfo))]
 
 
+class EncodeScope(ctypes.Structure):
+    """dfw_encode_scope: one scope of dfw_encode_device_multi."""
+    _fields_ = [("d_bf16", ctypes.c_void_p), ("n", ctypes.c_uint64), ("d_mant", ctypes.c_void_p),
+                ("d_chunk_bits", ctypes.c_void_p), ("d_group_start", ctypes.c_void_p)]
+
+
 class ContainerView(ctypes.Structure):
     """dfw_container_view: where dfw_container_read found each section."""
     _fields_ = [("k", ctypes.c_int32), ("has_plan", ctypes.c_int32), ("offsets_at", ctypes.c_uint64),
@@ -90,6 +96,8 @@ SIGNATURES = {
     "dfw_encode_device": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _vp, _u64, _TP, _LP, _vp]),
     "dfw_pack_device": (_i, [_vp, _TP, _LP, _vp, _vp, _u64, _vp]),
     "dfw_lanes_lut": (_i, [_TP, _LP, _vp]),
+    "dfw_encode_device_multi_staging_bytes": (_u64, [ctypes.c_uint32]),
+    "dfw_encode_device_multi": (_i, [ctypes.c_uint32, _vp, _i, _vp, _u64, _vp, _u64, _vp, _vp, _vp]),
     "dfw_encode_device_noalloc": (_i, [_vp, _u64, _i, _vp, _vp, _vp, _TP, _LP, _vp]),
     "dfw_rans_stream_bound": (_u64, [_u64]),
     "dfw_rans_encode": (_i, [_vp, _vp, _i, _vp, _u64, _vp, _u64, _vp, _RP, _i]),

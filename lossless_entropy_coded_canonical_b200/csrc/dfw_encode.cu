@@ -409,107 +409,213 @@ extern "C" uint64_t dfw_encode_device_scratch_bytes(uint64_t n) {
     return (sizeof(EncScratch) + 255) & ~(uint64_t)255;
 }
 
-extern "C" dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
-                                        uint16_t *d_chunk_bits, uint64_t *d_group_start, void *d_scratch,
-                                        uint64_t scratch_bytes, dfw_table *table, dfw_lanes_info *info,
-                                        void *cuda_stream) {
-    dfw::NvtxRange nvtx_range("dfw_encode_device");
-    if (!table || !info || cap < 1 || cap > DFW_MAX_CAP) return DFW_EINVAL;
-    const uint32_t fb = info->fast_bits;
-    std::memset(table, 0, sizeof(*table));
-    table->version = DFW_FORMAT_VERSION;
-    table->cap = (uint32_t)cap;
-    table->n = n;
-    table->stream_bytes = stream_bytes_for(0);
-    const uint64_t n_chunks = (n + LANE_SYMS - 1) / LANE_SYMS;
-    const uint64_t n_groups = (n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+namespace {
+
+// One scope of the first call, in stages: prepare (host checks, no GPU work),
+// pass 1 (histogram, read back into h_hist), code + passes 2 and 3 (totals
+// read back into h_res), finish (host checks, table and info).  Between the
+// stages the caller waits for the read-backs; dfw_encode_device_multi lets
+// the GPU run the next scope's pass 1 meanwhile.
+struct EncJob {
+    const uint16_t *d_bf16;
+    uint64_t n;
+    int cap;
+    uint8_t *d_mant;
+    uint16_t *d_chunk_bits;
+    uint64_t *d_group_start;
+    EncScratch *sc;
+    dfw_table *table;
+    dfw_lanes_info *info;
+    uint32_t fb;
+    uint64_t n_groups;
+    unsigned long long *h_hist;  // 256 counts (host)
+    unsigned long long *h_res;   // total_bits, (max_group_bits << 32) | max_span (host)
+};
+
+dfw_status enc_prepare(EncJob &j, void *d_scratch, uint64_t scratch_bytes) {
+    if (!j.table || !j.info || j.cap < 1 || j.cap > DFW_MAX_CAP) return DFW_EINVAL;
+    j.fb = j.info->fast_bits;
+    std::memset(j.table, 0, sizeof(*j.table));
+    j.table->version = DFW_FORMAT_VERSION;
+    j.table->cap = (uint32_t)j.cap;
+    j.table->n = j.n;
+    j.table->stream_bytes = stream_bytes_for(0);
+    const uint64_t n_chunks = (j.n + LANE_SYMS - 1) / LANE_SYMS;
+    j.n_groups = (n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
     if (n_chunks >= (1ull << 32)) return DFW_EINVAL;
-    if (n == 0) {
-        dfw_lanes_info q;
-        std::memset(&q, 0, sizeof(q));
-        q.fast_bits = fb;
-        const dfw_status st = dfw_plan_lanes_query(table, &q);
-        if (st != DFW_OK) return st;
-        q.max_group_bytes = 16;
-        *info = q;
-        if (d_group_start && cudaMemsetAsync(d_group_start, 0, sizeof(uint64_t), static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess)
-            return DFW_ECUDA;
-        return DFW_OK;
-    }
-    if (!d_bf16 || !d_mant || !d_chunk_bits || !d_group_start || !d_scratch) return DFW_EINVAL;
-    if (misaligned(d_bf16) || misaligned(d_mant) || misaligned(d_chunk_bits) || misaligned(d_group_start) ||
+    if (j.n == 0) return DFW_OK;
+    if (!j.d_bf16 || !j.d_mant || !j.d_chunk_bits || !j.d_group_start || !d_scratch) return DFW_EINVAL;
+    if (misaligned(j.d_bf16) || misaligned(j.d_mant) || misaligned(j.d_chunk_bits) || misaligned(j.d_group_start) ||
         misaligned(d_scratch))
         return DFW_EALIGN;
     if (scratch_bytes < sizeof(EncScratch)) return DFW_ENOMEM;
-    const int sms = device_sms();
-    if (sms <= 0) return DFW_ECUDA;
-    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-    EncScratch *sc = static_cast<EncScratch *>(d_scratch);
+    j.sc = static_cast<EncScratch *>(d_scratch);
+    return DFW_OK;
+}
 
-    // pass 1: raw bytes and the exponent histogram
-    if (cudaMemsetAsync(sc, 0, sizeof(EncScratch), s) != cudaSuccess) return DFW_ECUDA;
-    {
-        const uint64_t want = ((n >> 3) + SPLIT_NT - 1) / SPLIT_NT, cap_blocks = (uint64_t)sms * 8;
-        const unsigned blocks = (unsigned)std::max<uint64_t>(1, std::min(want, cap_blocks));
-        enc_split_hist<<<blocks, SPLIT_NT, 0, s>>>(d_bf16, n, d_mant, dfw_mant_bytes(n), sc->hist);
-        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
-    }
-    uint64_t hist[256];
-    if (cudaMemcpyAsync(hist, sc->hist, sizeof(hist), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
+// An empty tensor: its plan (no groups) and group_start[0] = 0.
+dfw_status enc_empty(EncJob &j, cudaStream_t s) {
+    dfw_lanes_info q;
+    std::memset(&q, 0, sizeof(q));
+    q.fast_bits = j.fb;
+    const dfw_status st = dfw_plan_lanes_query(j.table, &q);
+    if (st != DFW_OK) return st;
+    q.max_group_bytes = 16;
+    *j.info = q;
+    if (j.d_group_start && cudaMemsetAsync(j.d_group_start, 0, sizeof(uint64_t), s) != cudaSuccess)
         return DFW_ECUDA;
+    return DFW_OK;
+}
 
-    // the code, on the host, exactly as the host encoder builds it
-    uint64_t sum = 0;
+// pass 1: raw bytes and the exponent histogram, copied to h_hist
+dfw_status enc_pass1(EncJob &j, int sms, cudaStream_t s) {
+    if (cudaMemsetAsync(j.sc, 0, sizeof(EncScratch), s) != cudaSuccess) return DFW_ECUDA;
+    const uint64_t want = ((j.n >> 3) + SPLIT_NT - 1) / SPLIT_NT, cap_blocks = (uint64_t)sms * 8;
+    const unsigned blocks = (unsigned)std::max<uint64_t>(1, std::min(want, cap_blocks));
+    enc_split_hist<<<blocks, SPLIT_NT, 0, s>>>(j.d_bf16, j.n, j.d_mant, dfw_mant_bytes(j.n), j.sc->hist);
+    if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    if (cudaMemcpyAsync(j.h_hist, j.sc->hist, 256 * sizeof(unsigned long long), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
+        return DFW_ECUDA;
+    return DFW_OK;
+}
+
+// the code, on the host, exactly as the host encoder builds it; then passes
+// 2 and 3 (chunk bits, group totals -> group starts), totals copied to h_res
+dfw_status enc_pass23(EncJob &j, int sms, cudaStream_t s) {
+    uint64_t hist[256], sum = 0;
     int k = 0, only = 0;
     for (int b = 0; b < 256; ++b) {
+        hist[b] = j.h_hist[b];
         sum += hist[b];
         if (hist[b]) {
             ++k;
             only = b;
         }
     }
-    if (sum != n) return DFW_ECUDA;  // the histogram pass did not complete
-    table->n_symbols = (uint32_t)k;
-    table->single_symbol = k == 1 ? (uint32_t)only : 0u;
-    dfw_status st = code_lengths(hist, cap, table->len);
+    if (sum != j.n) return DFW_ECUDA;  // the histogram pass did not complete
+    j.table->n_symbols = (uint32_t)k;
+    j.table->single_symbol = k == 1 ? (uint32_t)only : 0u;
+    const dfw_status st = code_lengths(hist, j.cap, j.table->len);
     if (st != DFW_OK) return st;
-
-    // passes 2 and 3: chunk bits, group totals -> group starts
     LenTable lt;
-    std::memcpy(lt.len, table->len, 256);
-    {
-        const uint64_t want = (n_groups + GROUP_NT / 32 - 1) / (GROUP_NT / 32), cap_blocks = (uint64_t)sms * 4;
-        enc_chunk_bits<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, 0, s>>>(d_bf16, n, lt, d_chunk_bits,
-                                                                                 d_group_start, (uint32_t)n_groups);
-        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
-        // pass 3: ranges of whole tiles, at most SCAN_CTAS of them
-        uint64_t range = (n_groups + SCAN_CTAS - 1) / SCAN_CTAS;
-        range = (range + SCAN_NT - 1) / SCAN_NT * SCAN_NT;
-        const unsigned ctas = (unsigned)((n_groups + range - 1) / range);
-        enc_range_totals<<<ctas, SCAN_NT, 0, s>>>(d_group_start, (uint32_t)n_groups, (uint32_t)range, sc);
-        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
-        enc_range_scan<<<ctas, SCAN_NT, 0, s>>>(d_group_start, (uint32_t)n_groups, (uint32_t)range, sc);
-        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
-    }
-    unsigned long long res[2];  // total_bits, (max_group_bits << 32) | max_span
-    if (cudaMemcpyAsync(res, &sc->total_bits, sizeof(res), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaStreamSynchronize(s) != cudaSuccess)
+    std::memcpy(lt.len, j.table->len, 256);
+    const uint64_t want = (j.n_groups + GROUP_NT / 32 - 1) / (GROUP_NT / 32), cap_blocks = (uint64_t)sms * 4;
+    enc_chunk_bits<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, 0, s>>>(j.d_bf16, j.n, lt, j.d_chunk_bits,
+                                                                             j.d_group_start, (uint32_t)j.n_groups);
+    if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    // pass 3: ranges of whole tiles, at most SCAN_CTAS of them
+    uint64_t range = (j.n_groups + SCAN_CTAS - 1) / SCAN_CTAS;
+    range = (range + SCAN_NT - 1) / SCAN_NT * SCAN_NT;
+    const unsigned ctas = (unsigned)((j.n_groups + range - 1) / range);
+    enc_range_totals<<<ctas, SCAN_NT, 0, s>>>(j.d_group_start, (uint32_t)j.n_groups, (uint32_t)range, j.sc);
+    if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    enc_range_scan<<<ctas, SCAN_NT, 0, s>>>(j.d_group_start, (uint32_t)j.n_groups, (uint32_t)range, j.sc);
+    if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    if (cudaMemcpyAsync(j.h_res, &j.sc->total_bits, 2 * sizeof(unsigned long long), cudaMemcpyDeviceToHost, s) !=
+        cudaSuccess)
         return DFW_ECUDA;
-    uint64_t expect = 0;
-    for (int b = 0; b < 256; ++b) expect += hist[b] * table->len[b];
-    if (res[0] != expect) return DFW_ECUDA;  // the counting passes disagree with the histogram
-    table->total_bits = res[0];
-    table->stream_bytes = stream_bytes_for(res[0]);
+    return DFW_OK;
+}
 
+dfw_status enc_finish(EncJob &j) {
+    uint64_t expect = 0;
+    for (int b = 0; b < 256; ++b) expect += (uint64_t)j.h_hist[b] * j.table->len[b];
+    if (j.h_res[0] != expect) return DFW_ECUDA;  // the counting passes disagree with the histogram
+    j.table->total_bits = j.h_res[0];
+    j.table->stream_bytes = stream_bytes_for(j.h_res[0]);
     dfw_lanes_info q;
     std::memset(&q, 0, sizeof(q));
-    q.fast_bits = fb;
-    st = dfw_plan_lanes_query(table, &q);
+    q.fast_bits = j.fb;
+    const dfw_status st = dfw_plan_lanes_query(j.table, &q);
     if (st != DFW_OK) return st;
-    q.max_group_bytes = std::max<uint32_t>(16u, (uint32_t)(res[1] & 0xFFFFFFFFull));
-    *info = q;
+    q.max_group_bytes = std::max<uint32_t>(16u, (uint32_t)(j.h_res[1] & 0xFFFFFFFFull));
+    *j.info = q;
     return DFW_OK;
+}
+
+}  // namespace
+
+extern "C" dfw_status dfw_encode_device(const uint16_t *d_bf16, uint64_t n, int cap, uint8_t *d_mant,
+                                        uint16_t *d_chunk_bits, uint64_t *d_group_start, void *d_scratch,
+                                        uint64_t scratch_bytes, dfw_table *table, dfw_lanes_info *info,
+                                        void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_encode_device");
+    unsigned long long h_hist[256], h_res[2];
+    EncJob j{d_bf16, n, cap, d_mant, d_chunk_bits, d_group_start, nullptr, table, info, 0, 0, h_hist, h_res};
+    dfw_status st = enc_prepare(j, d_scratch, scratch_bytes);
+    if (st != DFW_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    if (n == 0) return enc_empty(j, s);
+    const int sms = device_sms();
+    if (sms <= 0) return DFW_ECUDA;
+    if ((st = enc_pass1(j, sms, s)) != DFW_OK) return st;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DFW_ECUDA;
+    if ((st = enc_pass23(j, sms, s)) != DFW_OK) return st;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DFW_ECUDA;
+    return enc_finish(j);
+}
+
+extern "C" uint64_t dfw_encode_device_multi_staging_bytes(uint32_t k) {
+    return (uint64_t)k * 258u * sizeof(unsigned long long);
+}
+
+extern "C" dfw_status dfw_encode_device_multi(uint32_t k, const dfw_encode_scope *scopes, int cap, void *d_scratch,
+                                              uint64_t scratch_bytes, void *h_staging, uint64_t staging_bytes,
+                                              dfw_table *tables, dfw_lanes_info *infos, void *cuda_stream) {
+    dfw::NvtxRange nvtx_range("dfw_encode_device_multi");
+    if (k == 0) return DFW_OK;
+    if (!scopes || !tables || !infos || !h_staging) return DFW_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(h_staging) & 7u) != 0) return DFW_EALIGN;
+    if (staging_bytes < dfw_encode_device_multi_staging_bytes(k)) return DFW_ENOMEM;
+    const uint64_t per = dfw_encode_device_scratch_bytes(0);
+    if (scratch_bytes / per < k) return DFW_ENOMEM;
+    // every scope checked before anything is launched
+    std::vector<EncJob> jobs(k);
+    unsigned long long *stage = static_cast<unsigned long long *>(h_staging);
+    for (uint32_t i = 0; i < k; ++i) {
+        const dfw_encode_scope &c = scopes[i];
+        jobs[i] = EncJob{c.d_bf16, c.n, cap, c.d_mant, c.d_chunk_bits, c.d_group_start, nullptr, tables + i,
+                         infos + i, 0, 0, stage + 258u * i, stage + 258u * i + 256u};
+        void *sc_i = d_scratch ? static_cast<unsigned char *>(d_scratch) + per * i : nullptr;
+        const dfw_status st = enc_prepare(jobs[i], sc_i, per);
+        if (st != DFW_OK) return st;
+    }
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    const int sms = device_sms();
+    if (sms <= 0) return DFW_ECUDA;
+    cudaEvent_t ev[2] = {nullptr, nullptr};
+    if (cudaEventCreateWithFlags(&ev[0], cudaEventDisableTiming) != cudaSuccess) return DFW_ECUDA;
+    if (cudaEventCreateWithFlags(&ev[1], cudaEventDisableTiming) != cudaSuccess) {
+        cudaEventDestroy(ev[0]);
+        return DFW_ECUDA;
+    }
+    // Stream order: pass 1 of scope i + 1 is queued before the host waits
+    // for scope i's histogram, so the GPU has it to run while the host
+    // builds scope i's code and queues its passes 2 and 3.
+    auto start = [&](uint32_t i) -> dfw_status {
+        if (jobs[i].n == 0) return enc_empty(jobs[i], s);
+        const dfw_status st = enc_pass1(jobs[i], sms, s);
+        if (st != DFW_OK) return st;
+        return cudaEventRecord(ev[i & 1u], s) == cudaSuccess ? DFW_OK : DFW_ECUDA;
+    };
+    dfw_status st = start(0);
+    for (uint32_t i = 0; i < k && st == DFW_OK; ++i) {
+        if (i + 1 < k && (st = start(i + 1)) != DFW_OK) break;
+        if (jobs[i].n == 0) continue;
+        if (cudaEventSynchronize(ev[i & 1u]) != cudaSuccess) {
+            st = DFW_ECUDA;
+            break;
+        }
+        st = enc_pass23(jobs[i], sms, s);
+    }
+    // all queued work ends before the call returns, on success or not
+    if (cudaStreamSynchronize(s) != cudaSuccess && st == DFW_OK) st = DFW_ECUDA;
+    cudaEventDestroy(ev[0]);
+    cudaEventDestroy(ev[1]);
+    for (uint32_t i = 0; i < k && st == DFW_OK; ++i)
+        if (jobs[i].n) st = enc_finish(jobs[i]);
+    return st;
 }
 
 extern "C" dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *table, const dfw_lanes_info *info,
