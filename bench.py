@@ -522,9 +522,9 @@ def run_encode_mode(args, rank, world, blocks, wdesc, device):
                    "encode_api": args.encode_api,
                    "parallelism": f"replica{world}" if world > 1 else "single GPU"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "peak_source": peak_kind, "kernel": "encoder (5 kernels per scope, host code construction)",
+                     "traffic": None, "peak_source": peak_kind, "kernel": "encoder (6 kernels per scope, host code construction)",
                      "algorithmic_bytes_per_step": alg, "mean_scope_ms": ms_step / k},
-        "clocks": clocks, "gpu_launches": args.steps * k * 5, "verified_roundtrip": bool(ok),
+        "clocks": clocks, "gpu_launches": args.steps * k * 6, "verified_roundtrip": bool(ok),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

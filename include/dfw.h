@@ -448,8 +448,10 @@ dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant,
  * n_groups = ceil(ceil(n / 64) / 32).  Errors: DFW_EINVAL, DFW_EALIGN,
  * DFW_ENOMEM (scratch too small), DFW_ECAP, DFW_ECUDA.
  *
- * dfw_pack_device -- second call: zeroes the stream and packs the codewords
- * at the positions the first call counted.  Asynchronous on cuda_stream.
+ * dfw_pack_device -- second call: packs the codewords at the positions the
+ * first call counted and writes the zero padding, so every one of the
+ * stream's table->stream_bytes bytes is written (two launches: the words
+ * neighbouring groups share are cleared first).  Asynchronous on cuda_stream.
  *   d_bf16, table, info, d_group_start   as returned by the first call
  *   d_stream   device, stream_capacity >= table->stream_bytes (output)
  * Errors: DFW_EINVAL, DFW_EALIGN, DFW_ENOMEM, DFW_ECUDA.

@@ -30,8 +30,8 @@
 //                          word, so the ORs are atomic); the warp then writes
 //                          the group's words, big-endian, with plain stores
 //                          inside and atomic ORs on the two words it may
-//                          share with the neighbouring groups (the stream is
-//                          zeroed first)
+//                          share with the neighbouring groups (a small kernel
+//                          zeroes those words and the padding first)
 // Nothing waits on another CTA; every loop is bounded by n.
 #include <cuda_runtime.h>
 
@@ -293,6 +293,24 @@ __global__ void __launch_bounds__(SCAN_NT) enc_range_scan(uint64_t *__restrict__
 }
 
 // ------------------------------------------------------------ pass 4
+
+// Before packing: zeroes the words that packing ORs into (the first and the
+// last word of every group; a neighbouring group may share them) and the
+// padding words after the last codeword.  Packing writes every other word
+// whole, so the rest of the stream needs no clearing.
+__global__ void __launch_bounds__(SCAN_NT) enc_zero_edges(const uint64_t *__restrict__ group_start, uint32_t n_groups,
+                                                          uint64_t total_bits, uint32_t *__restrict__ stream_words,
+                                                          uint64_t n_words) {
+    const uint64_t stride = (uint64_t)gridDim.x * SCAN_NT, t0 = (uint64_t)blockIdx.x * SCAN_NT + threadIdx.x;
+    for (uint64_t g = t0; g < n_groups; g += stride) {
+        const uint64_t a = group_start[g], b = group_start[g + 1];
+        if (b > a && ((b - 1) >> 5) < n_words) {
+            stream_words[a >> 5] = 0u;
+            stream_words[(b - 1) >> 5] = 0u;
+        }
+    }
+    for (uint64_t w = ((total_bits + 31) >> 5) + t0; w < n_words; w += stride) stream_words[w] = 0u;
+}
 
 __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict__ in, uint64_t n, const CodeTable ct,
                                                       const uint64_t *__restrict__ group_start, uint32_t n_groups,
@@ -633,11 +651,18 @@ extern "C" dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *t
         return DFW_EINVAL;
     if (misaligned(d_stream) || (n && (misaligned(d_bf16) || misaligned(d_group_start)))) return DFW_EALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-    if (cudaMemsetAsync(d_stream, 0, table->stream_bytes, s) != cudaSuccess) return DFW_ECUDA;
-    if (table->total_bits == 0) return DFW_OK;  // zero or one distinct exponent: no bits
+    if (table->total_bits == 0)  // zero or one distinct exponent: no bits, the stream is its padding
+        return cudaMemsetAsync(d_stream, 0, table->stream_bytes, s) == cudaSuccess ? DFW_OK : DFW_ECUDA;
     if (!d_bf16 || !d_group_start) return DFW_EINVAL;
     const int sms = device_sms();
     if (sms <= 0) return DFW_ECUDA;
+    {
+        const uint64_t want = (n_groups + SCAN_NT - 1) / SCAN_NT, cap_blocks = (uint64_t)sms * 8;
+        enc_zero_edges<<<(unsigned)std::max<uint64_t>(1, std::min(want, cap_blocks)), SCAN_NT, 0, s>>>(
+            d_group_start, (uint32_t)n_groups, table->total_bits, reinterpret_cast<uint32_t *>(d_stream),
+            table->stream_bytes / 4);
+        if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+    }
     uint32_t code[256];
     canonical_codes(table->len, code);
     CodeTable ct;

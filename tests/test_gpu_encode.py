@@ -123,3 +123,26 @@ def test_device_encode_full_size_block_c3():
     out = dfw.decode_lanes(dl)
     dfw.check()
     assert torch.equal(out.view(torch.int16), x.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["c1", "c4b", "random2049", "single", "c4bp"])
+def test_pack_writes_every_stream_byte(oracle, name):
+    """dfw_pack_device into a buffer full of garbage: its first stream_bytes
+    bytes become the oracle's stream (codewords and zero padding), and the
+    bytes past them stay as they were."""
+    import ctypes
+    rng = np.random.default_rng(31)
+    u = {"random2049": lambda: rng.integers(0, 65536, size=2049, dtype=np.uint64).astype(np.uint16),
+         "single": lambda: ((rng.integers(0, 2, 5000) << 15) | (120 << 7)).astype(np.uint16)}.get(
+        name, lambda: CASES[name]())()
+    x = torch.from_numpy(np.ascontiguousarray(u).view(np.int16)).cuda()
+    dl = dfw.encode_device(x)
+    sb = int(dl.table.stream_bytes)
+    buf = torch.full((sb + 64,), 0xA5, dtype=torch.uint8, device="cuda")
+    st = dfw.lib().dfw_pack_device(x.data_ptr(), ctypes.byref(dl.table), ctypes.byref(dl.info),
+                                   dl.group_start.data_ptr(), buf.data_ptr(), buf.numel(), None)
+    assert st == dfw.OK
+    dfw.check()
+    got = buf.cpu().numpy()
+    assert np.array_equal(got[:sb], oracle.encode(u).stream)
+    assert (got[sb:] == 0xA5).all()
