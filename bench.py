@@ -282,24 +282,37 @@ def run_device(devs, scratch, steps, warmup, stream):
     return total_ms, per_launch, status
 
 
-def run_device_seq(devs, scratch, steps, warmup, stream):
+def run_device_seq(devs, scratch, steps, warmup, stream, graph=False):
     """The step as one dfw_decode_lanes_seq call over every scope: the same
     launches in the same order into the same scratch buffer, each one a
     programmatic dependent of the one before (it may start while the previous
-    drains and stores only after it completes)."""
+    drains and stores only after it completes).  With ``graph`` the call is
+    captured once into a CUDA graph and each step replays it."""
     import lossless_entropy_coded_canonical_b200 as dfw
     for _ in range(warmup):
         dfw.decode_lanes_seq(devs, scratch, stream=stream)
     dfw.check(stream)
+    g = None
+    if graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            dfw.decode_lanes_seq(devs, scratch)
+        for _ in range(warmup):
+            g.replay()
+        torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     t0.record(stream)
     for _ in range(steps):
-        dfw.decode_lanes_seq(devs, scratch, stream=stream)
+        if g is not None:
+            g.replay()
+        else:
+            dfw.decode_lanes_seq(devs, scratch, stream=stream)
     t1.record(stream)
     torch.cuda.synchronize()
     barrier()
+    del g
     return t0.elapsed_time(t1), dfw.check_status(stream)
 
 
@@ -751,6 +764,8 @@ def main(argv=None):
     ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="decode step: capture the sequence once in a CUDA graph and replay it each step")
     ap.add_argument("--encode-api", default="multi", choices=["multi", "single"],
                     help="encode mode: one dfw_encode_device_multi call for all scopes, or dfw_encode_device each")
     ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv", "rans", "launch-cost"],
@@ -801,7 +816,7 @@ def main(argv=None):
     sampler = ClockSampler(local)
     sampler.start()
     if lanes:  # the step: one sequence of launches over every scope
-        total_ms, status = run_device_seq(devs, scratch, args.steps, args.warmup, stream)
+        total_ms, status = run_device_seq(devs, scratch, args.steps, args.warmup, stream, args.graph)
     else:
         total_ms, per_launch, status = run_device(devs, scratch, args.steps, args.warmup, stream)
     clocks = sampler.stop()
@@ -854,7 +869,9 @@ def main(argv=None):
                          "every block's bf16; no reuse between steps)",
                    "parallelism": f"replica{world}" if world > 1 else "single GPU",
                    "launch": ("one dfw_decode_lanes_seq per step: one launch per scope, each a programmatic "
-                              "dependent of the previous" if lanes else "one dfw_decode_block per scope")},
+                              "dependent of the previous" + (", captured once in a CUDA graph and replayed"
+                                                             if args.graph else "")
+                              if lanes else "one dfw_decode_block per scope")},
         "effective_gbs": eff_gbs, "hbm_frac": eff_gbs / peak,
         "compression_ratio": 2 * n_total / comp, "compression_ratio_no_aux": 2 * n_total / comp_noaux,
         "bits_per_weight": 8 * comp / n_total,

@@ -133,3 +133,26 @@ def test_seq_rejects_bad_arguments_before_launch(scopes):
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), before.view(torch.int16))
     dfw.check()
+
+
+def test_seq_replays_from_a_cuda_graph(scopes):
+    """The sequence captured once into a CUDA graph (its programmatic
+    dependencies become graph edges) and replayed over garbage gives the
+    eager result every time: the call makes no host synchronisation and no
+    allocation, so a serving loop can capture it."""
+    us, devs = scopes
+    nmax = max(u.size for u in us)
+    want = _garbage(nmax)
+    dfw.decode_lanes_seq(devs, want)
+    dfw.check()
+    out = _garbage(nmax)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dfw.decode_lanes_seq(devs, out)
+    for _ in range(4):
+        out.view(torch.int16).fill_(0x5A5A)
+        g.replay()
+        torch.cuda.synchronize()
+        dfw.check()
+        assert torch.equal(out.view(torch.int16), want.view(torch.int16))
+    del g
