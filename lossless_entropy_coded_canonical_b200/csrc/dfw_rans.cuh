@@ -13,7 +13,16 @@
 // coalesced 128-byte rows, three rows (12 steps) ahead of use, and reach
 // the lane that needs them by shuffle.  A block must end with every state at
 // 2^16 and every word used; otherwise the status word records it.
+//
+// Slots per warp (nslot): two let the next block's copy run during this
+// block's decode; one halves the shared memory per warp, so twice as many
+// warps fit on an SM, and the copy of the next block is then issued after
+// this block's last read and waited for at the top of the next one.  The
+// launcher takes whichever keeps more warps resident (the decode is bound by
+// the latency of each state's chain of dependent steps, so more warps win).
 #pragma once
+
+#include <type_traits>
 
 #include "dfw_device.cuh"
 
@@ -30,7 +39,7 @@ struct RansParams {
     const uint64_t *block_start;
     uint16_t *out;
     uint64_t n, stream_bytes, mant_bytes;
-    uint32_t n_blocks, slot_bytes;
+    uint32_t n_blocks, slot_bytes, nslot;
     uint16_t freq[256];
 };
 
@@ -62,7 +71,7 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
         return;
     }
 
-    uint8_t *wbase = smem + RANS_TABLE_BYTES + warp * (16u + 2u * prm.slot_bytes);
+    uint8_t *wbase = smem + RANS_TABLE_BYTES + warp * (16u + prm.nslot * prm.slot_bytes);
     const uint32_t bar0 = smem_u32(wbase);
     uint8_t *slots = wbase + 16;
     const uint32_t gstride = gridDim.x * NWARP;
@@ -88,16 +97,17 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
     if (lane == 0) issue(b, 0);
 
     const uint32_t lt_mask = (1u << lane) - 1u;
+    const bool two = prm.nslot == 2u;
     for (uint32_t it = 0;; ++it) {
-        const uint32_t s = it & 1u;
+        const uint32_t s = two ? (it & 1u) : 0u;
         const uint32_t bn = b + gstride;
         __syncwarp();  // every lane is done with the other slot
-        if (bn < prm.n_blocks && lane == 0) issue(bn, s ^ 1u);
-        bool ok = mbar_wait(bar0 + 8u * s, (it >> 1) & 1u);
+        if (two && bn < prm.n_blocks && lane == 0) issue(bn, s ^ 1u);
+        bool ok = mbar_wait(bar0 + 8u * s, two ? (it >> 1) & 1u : it & 1u);
         if (!__all_sync(0xFFFFFFFFu, ok)) {
             if (lane == 0) {
                 atomicOr(&g_status, ST_TIMEOUT);
-                if (bn < prm.n_blocks) mbar_wait_bounded(bar0 + 8u * (s ^ 1u), ((it + 1) >> 1) & 1u);
+                if (two && bn < prm.n_blocks) mbar_wait_bounded(bar0 + 8u * (s ^ 1u), ((it + 1) >> 1) & 1u);
             }
             return;
         }
@@ -113,7 +123,6 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
             const uint32_t words = (uint32_t)(b1 - b0 - RANS_HEAD) / 2u;  // includes the zero padding
             uint32_t x = lds32(sl + 4u * lane);
             uint32_t ptr = 0;
-            bool err = false;
             // raw bytes: lane l loads the 4 bytes at 128 q + 4 l of the block
             // (coalesced), three quads ahead; step 4 q + t takes its byte from
             // lane 8 t + l / 4 by shuffle
@@ -127,43 +136,53 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
             uint16_t *op = prm.out + i0 + lane;
             const uint32_t quads = (cnt + 127u) / 128u;
             const uint32_t tab = smem_u32(s_tab), wbase = sl + RANS_HEAD;
-            const bool whole = cnt == DFW_RANS_BLOCK;  // every block but possibly the scope's last
-            for (uint32_t q = 0; q < quads; ++q) {
-                const uint32_t mc = m1;
-                m1 = m2;
-                m2 = m3;
-                m3 = mload(q + 3u);
+            // the quads of the block; WHOLE (every block but possibly the
+            // scope's last) drops the per-step checks against cnt
+            auto quads_of = [&](auto whole_c) {
+                constexpr bool WHOLE = decltype(whole_c)::value;
+                for (uint32_t q = 0; q < quads; ++q) {
+                    const uint32_t mc = m1;
+                    m1 = m2;
+                    m2 = m3;
+                    m3 = mload(q + 3u);
 #pragma unroll
-                for (uint32_t t = 0; t < 4; ++t) {
-                    const uint32_t i = 128u * q + 32u * t + lane;
-                    const bool live = whole || i < cnt;
-                    const uint32_t e = lds32(tab + 4u * (x & (RANS_SLOTS - 1u)));
-                    const uint32_t xd = (((e >> 8) & 0xFFFu) + 1u) * (x >> DFW_RANS_SCALE_BITS) + (e >> 20);
-                    x = live ? xd : x;
-                    const bool need = live && x < 65536u;
-                    const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
-                    const uint32_t w = ptr + __popc(mask & lt_mask);
-                    const bool rd = need && w < words;
-                    err |= need && !rd;
-                    const uint32_t v = lds16_if(rd, wbase + 2u * w);  // branch-free reload
-                    x = need ? (x << 16) | v : x;
-                    ptr += __popc(mask);
-                    const uint32_t mb = __byte_perm(__shfl_sync(0xFFFFFFFFu, mc, 8u * t + (lane >> 2)), 0u,
-                                                    0x4440u | (lane & 3u));
-                    // bf16 = sign << 15 | exponent << 7 | mantissa: the raw
-                    // byte doubled into both halves keeps its sign at bit 15
-                    // and its mantissa at bits 6..0; the table entry's low
-                    // byte is the exponent
-                    if (live) op[32u * t] = (uint16_t)(((mb * 0x101u) & 0x807Fu) | ((e << 7) & 0x7F80u));
+                    for (uint32_t t = 0; t < 4; ++t) {
+                        const bool live = WHOLE || 128u * q + 32u * t + lane < cnt;
+                        const uint32_t e = lds32(tab + 4u * (x & (RANS_SLOTS - 1u)));
+                        const uint32_t xd = (((e >> 8) & 0xFFFu) + 1u) * (x >> DFW_RANS_SCALE_BITS) + (e >> 20);
+                        x = live ? xd : x;
+                        const bool need = live && x < 65536u;
+                        const uint32_t mask = __ballot_sync(0xFFFFFFFFu, need);
+                        const uint32_t w = ptr + __popc(mask & lt_mask);
+                        // a reload past the block's words is skipped (a corrupt
+                        // block; the checks after the block then fail)
+                        const uint32_t v = lds16_if(need && w < words, wbase + 2u * w);
+                        x = need ? (x << 16) | v : x;
+                        ptr += __popc(mask);
+                        const uint32_t mb = __byte_perm(__shfl_sync(0xFFFFFFFFu, mc, 8u * t + (lane >> 2)), 0u,
+                                                        0x4440u | (lane & 3u));
+                        // bf16 = sign << 15 | exponent << 7 | mantissa: the
+                        // raw byte doubled into both halves keeps its sign at
+                        // bit 15 and its mantissa at bits 6..0; the table
+                        // entry's low byte is the exponent
+                        if (live) op[32u * t] = (uint16_t)(((mb * 0x101u) & 0x807Fu) | ((e << 7) & 0x7F80u));
+                    }
+                    op += 128;
                 }
-                op += 128;
-            }
-            // integrity: every state back at 2^16, every word used
-            const bool good = __all_sync(0xFFFFFFFFu, !err && x == 65536u) &&
+            };
+            if (cnt == DFW_RANS_BLOCK) quads_of(std::integral_constant<bool, true>{});
+            else quads_of(std::integral_constant<bool, false>{});
+            // integrity: every state back at 2^16, every word used and none
+            // past the block's end (a skipped reload leaves ptr beyond it)
+            const bool good = __all_sync(0xFFFFFFFFu, x == 65536u) &&
                               ((RANS_HEAD + 2ull * ptr + 15ull) & ~15ull) == b1 - b0;
             if (!good && lane == 0) atomicOr(&g_status, ST_COUNT);
         }
         if (bn >= prm.n_blocks) break;
+        if (!two) {
+            __syncwarp();  // every lane is done with the slot
+            if (lane == 0) issue(bn, 0u);
+        }
         b = bn;
     }
 }
@@ -200,26 +219,40 @@ dfw_status launch_rans_decode(const uint8_t *d_stream, const uint8_t *d_mant, co
     std::memcpy(prm.freq, t->freq, sizeof(prm.freq));
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return DFW_ECUDA;
-    // the largest CTA whose warps' double-buffered block slots fit (blocks of
-    // incompressible data need 16.5 KB slots)
-    for (RansVariant &v : g_rans) {
-        const uint32_t smem = RANS_TABLE_BYTES + (uint32_t)(v.nt / 32) * (16u + 2u * prm.slot_bytes);
-        if (smem > 227u * 1024u) continue;
-        if (!v.smem_set[dev]) {
-            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+    // the CTA size and slots per warp that keep the most warps resident per
+    // SM (blocks of incompressible data need 16.5 KB slots); on a tie, two
+    // slots (the next block's copy overlaps this block's decode)
+    RansVariant *best = nullptr;
+    uint32_t best_smem = 0, best_nslot = 0;
+    int best_warps = 0, best_per_sm = 0;
+    for (uint32_t nslot = 2; nslot >= 1; --nslot) {
+        for (RansVariant &v : g_rans) {
+            const uint32_t smem = RANS_TABLE_BYTES + (uint32_t)(v.nt / 32) * (16u + nslot * prm.slot_bytes);
+            if (smem > 227u * 1024u) continue;
+            if (!v.smem_set[dev]) {
+                if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+                    return DFW_ECUDA;
+                v.smem_set[dev] = 1;
+            }
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess)
                 return DFW_ECUDA;
-            v.smem_set[dev] = 1;
+            if (per_sm * (v.nt / 32) > best_warps) {
+                best = &v;
+                best_smem = smem;
+                best_nslot = nslot;
+                best_warps = per_sm * (v.nt / 32);
+                best_per_sm = per_sm;
+            }
         }
-        int per_sm = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess) return DFW_ECUDA;
-        if (per_sm < 1) continue;
-        const uint64_t wpc = (uint64_t)v.nt / 32;
-        const uint64_t warps = (uint64_t)per_sm * sms * wpc;
-        const uint64_t want = t->n_blocks < warps ? t->n_blocks : warps;
-        v.fn<<<(unsigned)((want + wpc - 1) / wpc), v.nt, smem, s>>>(prm);
-        return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
     }
-    return DFW_EINVAL;
+    if (!best) return DFW_EINVAL;
+    prm.nslot = best_nslot;
+    const uint64_t wpc = (uint64_t)best->nt / 32;
+    const uint64_t warps = (uint64_t)best_per_sm * sms * wpc;
+    const uint64_t want = t->n_blocks < warps ? t->n_blocks : warps;
+    best->fn<<<(unsigned)((want + wpc - 1) / wpc), best->nt, best_smem, s>>>(prm);
+    return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
 }
 
 

@@ -102,6 +102,22 @@ def test_rans_gpu_corrupt_block_detected(oracle):
     dfw.check()  # cleared
 
 
+def test_rans_gpu_short_block_detected(oracle):
+    """Block 3's extent cut by 16 bytes (its last 8 words belong to block 4 as
+    far as the decoder can tell): the states of block 3 ask for words past its
+    end, those reloads are skipped, and the checks after the block report it;
+    block 4, now read from 16 bytes early, fails its own checks."""
+    u = CASES["c1"]()
+    oenc = oracle.rans_encode(u, 12, 32, 16384)
+    dr = _device_from_oracle(oenc)
+    dr.block_start[4] -= 16
+    out = dfw.rans_decode(dr)
+    assert dfw.check_status() == dfw.ECORRUPT
+    dfw.check()  # cleared
+    got = workloads.as_u16_numpy(out)
+    assert np.array_equal(got[: 3 * 16384], u[: 3 * 16384])  # blocks before it are untouched by the damage
+
+
 def test_rans_gpu_full_size_block_c3():
     ts = [t.cpu() for t in workloads.generate_block(workloads.c3(), "cuda")]
     enc = dfw.rans_encode(ts)
