@@ -530,8 +530,10 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         }
         ok = mbar_wait(bar_m, k & 1u) && ok;
         if (!__all_sync(0xFFFFFFFFu, ok)) {  // a bulk copy never completed: give up
-            if (lane == 0) {
+            if (lane == 0) {  // report, then give each copy in flight one more bounded wait
                 atomicOr(&g_status, ST_TIMEOUT);
+                mbar_wait_bounded(bar_s0 + 8u * s, (k >> 1) & 1u);
+                mbar_wait_bounded(bar_m, k & 1u);
                 if (has_next) mbar_wait_bounded(bar_s0 + 8u * (s ^ 1u), ((k + 1) >> 1) & 1u);
             }
             return;

@@ -103,10 +103,12 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
         const uint32_t bn = b + gstride;
         __syncwarp();  // every lane is done with the other slot
         if (two && bn < prm.n_blocks && lane == 0) issue(bn, s ^ 1u);
-        bool ok = mbar_wait(bar0 + 8u * s, two ? (it >> 1) & 1u : it & 1u);
+        const uint32_t parity = two ? (it >> 1) & 1u : it & 1u;
+        bool ok = mbar_wait(bar0 + 8u * s, parity);
         if (!__all_sync(0xFFFFFFFFu, ok)) {
-            if (lane == 0) {
+            if (lane == 0) {  // report, then give the copies in flight one more bounded wait each
                 atomicOr(&g_status, ST_TIMEOUT);
+                mbar_wait_bounded(bar0 + 8u * s, parity);
                 if (two && bn < prm.n_blocks) mbar_wait_bounded(bar0 + 8u * (s ^ 1u), ((it + 1) >> 1) & 1u);
             }
             return;
