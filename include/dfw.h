@@ -524,10 +524,17 @@ dfw_status dfw_encode_device_multi(uint32_t k, const dfw_encode_scope *scopes, i
  * The pages describe no such call; it exists for those callers only.
  *
  * The scratch is an array of DFW_NOALLOC_SCRATCH_BYTES compiled into the
- * library: every GPU that loads the library holds one until the process
- * exits.  The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture begins.  All calls share the array and clear it before use,
+ * library: every GPU that uses the library holds one until the process
+ * exits.  With lazy module loading (the CUDA runtime's default) the array
+ * and the encoder's kernels are placed on a device when the library first
+ * uses that device, not when the library is loaded, so a runtime that
+ * reserves the GPU's memory up front should make one call (a warm-up) on
+ * each device before it reserves.  The first call on a device also looks
+ * up the array's device address (cudaGetSymbolAddress) and caches it; make
+ * that first call before any stream capture begins.  The cached address
+ * belongs to the device's context at that time: after cudaDeviceReset (or
+ * anything else that destroys and re-creates the context) in the same
+ * process the call is not supported.  All calls share the array and clear it before use,
  * so calls whose GPU work overlaps (two streams, two host threads) race on it:
  * the caller must not overlap them.  Arguments, outputs, synchronisation and
  * errors as dfw_encode_device; DFW_ENOMEM if the scratch that n needs

@@ -698,7 +698,9 @@ void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {nullptr};
 std::mutex g_noalloc_mu;
 
 // The array's device address on the current device; looked up (and cached)
-// on the first call there.
+// on the first call there.  The cache is never invalidated: a context
+// destroyed and re-created in the same process (cudaDeviceReset) would leave
+// a stale address, which is why such a reset is documented as unsupported.
 dfw_status noalloc_scratch(void **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return DFW_ECUDA;

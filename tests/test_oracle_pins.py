@@ -559,6 +559,8 @@ def test_gemv_hand_worked(oracle):
     w[1, 1::2] = 0xBE80
     x = np.array([_bf16_of(j + 1) for j in range(cols)], np.uint16)
     assert oracle.gemv(w.reshape(-1), rows, cols, x).tolist() == want
+    want_abs = [float(v) for v in kv["y_abs"].split()]
+    assert oracle.gemv_abs(w.reshape(-1), rows, cols, x).tolist() == want_abs
 
 
 def test_gemv_basis_vectors_pick_columns(oracle):
@@ -570,6 +572,33 @@ def test_gemv_basis_vectors_pick_columns(oracle):
         x[j] = 0x3F80  # 1.0
         y = oracle.gemv(w, rows, cols, x)
         assert np.array_equal(y, oracle.bf16_values(w).reshape(rows, cols)[:, j])
+
+
+def test_gemv_abs_against_exact_rationals(oracle):
+    """gemv_abs is the exact sum of |w x| (up to float64 rounding), with
+    negative weights and negative inputs present: a version that dropped the
+    absolute value of either operand, took it of the sum instead of the terms,
+    or used the wrong axis would miss these by far more than the rounding."""
+    from fractions import Fraction
+    rng = np.random.default_rng(8)
+    rows, cols = 4, 128
+    w, x = _u16_normal(rng, rows * cols), _u16_normal(rng, cols)
+    wv = oracle.bf16_values(w).reshape(rows, cols)
+    xv = oracle.bf16_values(x)
+    assert (wv < 0).any() and (wv > 0).any() and (xv < 0).any() and (xv > 0).any()
+    got = oracle.gemv_abs(w, rows, cols, x)
+    assert got.shape == (rows,)
+    for i in range(rows):
+        exact = sum(abs(Fraction(float(wv[i, j])) * Fraction(float(xv[j]))) for j in range(cols))
+        assert abs(Fraction(float(got[i])) - exact) <= Fraction(cols * 2.0 ** -53) * exact
+        signed = abs(sum(Fraction(float(wv[i, j])) * Fraction(float(xv[j])) for j in range(cols)))
+        assert exact > signed  # the terms have mixed signs: |sum| is strictly smaller
+    # one row of all-negative weights against all-negative inputs: every term
+    # is positive, so the signed product equals the absolute sum
+    wn = np.full(cols, 0xBF80, np.uint16)  # -1.0
+    xn = np.array([0x8000 | _bf16_of(j + 1) for j in range(cols)], np.uint16)  # -(j + 1)
+    assert oracle.gemv_abs(wn, 1, cols, xn).tolist() == [cols * (cols + 1) / 2]
+    assert oracle.gemv(wn, 1, cols, xn).tolist() == [cols * (cols + 1) / 2]
 
 
 def test_gemv_against_exact_rationals(oracle):

@@ -7,7 +7,9 @@ library rather than a caller buffer.  Two calls in a row on different inputs
 must each give exactly what dfw_encode_device gives with its own scratch
 buffer: same raw bytes, chunk bit counts, group starts, code table and plan
 info, and, after dfw_pack_device, the same stream.  The second call passing
-also shows that the shared array is cleared between calls.
+also shows that the shared array is cleared between calls.  A second test
+checks the property itself: after a warm-up call, a call leaves the device's
+free memory and torch's allocator unchanged.
 """
 from __future__ import annotations
 
@@ -83,3 +85,36 @@ def test_noalloc_matches_regular_entry_point_two_calls_in_a_row():
         out = dfw.decode_lanes(dl)
         dfw.check()
         assert np.array_equal(workloads.as_u16_numpy(out), workloads.as_u16_numpy(x))
+
+
+def test_noalloc_call_allocates_no_device_memory():
+    """What the entry point exists for: once a warm-up call has placed the
+    library's code and array on the device, a call changes neither the
+    device's free memory (cudaMemGetInfo) nor torch's allocator, and its
+    result still equals the regular entry point's.  The outputs are
+    allocated before the measurement starts."""
+    lib = dfw.lib()
+    x = torch.cat([t.reshape(-1) for t in workloads.generate_block(workloads.c1(), "cuda")])
+    n, dev = x.numel(), x.device
+    n_groups = -(-(-(-n // 64)) // 32)
+    mant = torch.empty(dfw.mant_bytes(n), dtype=torch.uint8, device=dev)
+    chunk_bits = torch.empty(32 * n_groups, dtype=torch.int16, device=dev)
+    group_start = torch.empty(n_groups + 1, dtype=torch.int64, device=dev)
+    table, info = Table(), LanesInfo()
+    sh = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+    def call():
+        st = lib.dfw_encode_device_noalloc(x.data_ptr(), n, 32, mant.data_ptr(), chunk_bits.data_ptr(),
+                                           group_start.data_ptr(), ctypes.byref(table), ctypes.byref(info), sh)
+        assert st == dfw.OK, lib.dfw_strerror(st)
+        torch.cuda.synchronize()
+
+    call()  # warm-up: module loading may place code and the array on the device here
+    free0, alloc0 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
+    call()
+    free1, alloc1 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
+    assert alloc1 == alloc0
+    assert free1 == free0
+    want = _encode_via_abi(x, noalloc=False)
+    assert torch.equal(mant.cpu(), want["mant"]) and torch.equal(group_start.cpu(), want["group_start"])
+    assert bytes(table) == want["table"] and bytes(info) == want["info"]
