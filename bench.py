@@ -45,6 +45,7 @@ FALLBACK_HBM_GBS = 6650.0
 _CSRC = "lossless_entropy_coded_canonical_b200/csrc/"
 KERNEL_SOURCES = {
     "decode_lanes": [_CSRC + "dfw_lanes.cuh", _CSRC + "dfw_device.cuh", _CSRC + "dfw_internal.h"],
+    "decode_lanes_multi": [_CSRC + "dfw_lanes.cuh", _CSRC + "dfw_device.cuh", _CSRC + "dfw_internal.h"],
     "decode_tiles": [_CSRC + "dfw_decode.cu", _CSRC + "dfw_device.cuh", _CSRC + "dfw_internal.h"],
 }
 
@@ -241,16 +242,35 @@ def decode_one(d, scratch, stream=None):
 
 
 def verify(blocks, devs, scratch, device):
-    """Decodes each block once more and compares with the regenerated input."""
+    """Decodes each block once more, with the kernel the step uses (the
+    sequence kernel for the known-start plan, one scope per call), and
+    compares with the regenerated input; for the known-start plan the whole
+    sequence is then decoded once more and the buffer must end as the last
+    scope's input."""
     import lossless_entropy_coded_canonical_b200 as dfw
-    for b, d in zip(blocks, devs):
-        decode_one(d, scratch)
-        dfw.check()
+    lanes = isinstance(devs[0], dfw.DeviceLanes)
+
+    def same(b):
         off = 0
         for t in workloads.generate_block(b, device):
             if not torch.equal(scratch[off: off + t.numel()].view(torch.int16), t.view(torch.int16)):
                 return False
             off += t.numel()
+        return True
+
+    for b, d in zip(blocks, devs):
+        if lanes:
+            dfw.decode_lanes_seq([d], scratch)
+        else:
+            decode_one(d, scratch)
+        dfw.check()
+        if not same(b):
+            return False
+    if lanes:
+        scratch.view(torch.int16).fill_(0x5A5A)
+        dfw.decode_lanes_seq(devs, scratch)
+        dfw.check()
+        return same(blocks[-1])
     return True
 
 
@@ -825,6 +845,56 @@ def run_launch_cost_mode(args, rank, world, device):
     return 0 if all(r["bit_exact"] for r in rows) else 1
 
 
+# ------------------------------------------------------------------ seq-cost mode
+
+def run_seq_cost_mode(args, rank, world, device):
+    """Cost of a scope inside a sequence: one Llama-3-8B-shaped transformer
+    block decoded k = 1, 2, 4, 8, 16 times in one dfw_decode_lanes_seq call
+    (the same resident scope repeated), CUDA events around each call; a
+    least-squares line gives the fixed cost per call (intercept) and the
+    cost per scope (slope), beside the same block decoded alone by
+    dfw_decode_lanes (CUDA events around each launch)."""
+    import lossless_entropy_coded_canonical_b200 as dfw
+    blk = workloads.c5()[1]
+    devs, _ = prepare_on_device([blk], device)
+    d = devs[0]
+    out = torch.empty(d.n, dtype=torch.bfloat16, device=device)
+    rows = []
+    for k in (1, 2, 4, 8, 16):
+        seq = [d] * k
+        for _ in range(args.warmup):
+            dfw.decode_lanes_seq(seq, out)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        torch.cuda.synchronize()
+        for a, b in ev:
+            a.record()
+            dfw.decode_lanes_seq(seq, out)
+            b.record()
+        torch.cuda.synchronize()
+        ms = sorted(a.elapsed_time(b) for a, b in ev)
+        rows.append({"scopes": k, "launches": dfw.decode_lanes_seq_launches(seq), "median_ms": ms[len(ms) // 2]})
+    for _ in range(args.warmup):
+        dfw.decode_lanes(d, out)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        a.record()
+        dfw.decode_lanes(d, out)
+        b.record()
+    torch.cuda.synchronize()
+    single = sorted(a.elapsed_time(b) for a, b in ev)[args.steps // 2]
+    ok = dfw.check_status() == dfw.OK and torch.equal(
+        out.view(torch.int16), torch.cat([t.reshape(-1) for t in workloads.generate_block(blk, device)]).view(torch.int16))
+    ks = np.array([r["scopes"] for r in rows], float)
+    ts = np.array([r["median_ms"] for r in rows])
+    slope, icpt = np.linalg.lstsq(np.vstack([ks, np.ones_like(ks)]).T, ts, rcond=None)[0]
+    if rank == 0:
+        print(json.dumps({"mode": "seq-cost", "scope": "llama3-8b-shaped transformer block (218103808 weights)",
+                          "sizes": rows, "fixed_ms_per_call": float(icpt), "ms_per_scope": float(slope),
+                          "single_launch_ms": single, "verified_bit_exact": bool(ok)}), flush=True)
+    return 0 if ok else 1
+
+
 # ------------------------------------------------------------------ main
 
 def main(argv=None):
@@ -847,10 +917,12 @@ def main(argv=None):
                     help="decode step: capture the sequence once in a CUDA graph and replay it each step")
     ap.add_argument("--encode-api", default="multi", choices=["multi", "single"],
                     help="encode mode: one dfw_encode_device_multi call for all scopes, or dfw_encode_device each")
-    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv", "rans", "launch-cost"],
+    ap.add_argument("--mode", default="decode", choices=["decode", "encode", "gemv", "rans", "launch-cost",
+                                                         "seq-cost"],
                     help="decode: the decode path (default); encode: the GPU encoder; "
                          "gemv: decode fused with y = W x; rans: the rANS variant beside Huffman; "
-                         "launch-cost: decode time against size (fixed cost per launch)")
+                         "launch-cost: decode time against size (fixed cost per launch); "
+                         "seq-cost: cost of a scope inside a sequence")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -876,6 +948,8 @@ def main(argv=None):
     dfw.check()
     if args.mode == "launch-cost":
         return run_launch_cost_mode(args, rank, world, device)
+    if args.mode == "seq-cost":
+        return run_seq_cost_mode(args, rank, world, device)
     if args.mode in ("encode", "gemv", "rans"):
         run = {"encode": run_encode_mode, "gemv": run_gemv_mode, "rans": run_rans_mode}[args.mode]
         rc = run(args, rank, world, blocks, wdesc, device)
@@ -908,14 +982,31 @@ def main(argv=None):
         status = status if status != dfw.OK else st_pl
     ok = status == dfw.OK and verify(blocks, devs, scratch, device)
 
-    # roofline of the decode kernel: algorithmic bytes / mean launch duration
+    # roofline of the step's kernel: algorithmic bytes per launch / mean
+    # launch duration.  Known-start plan: the step is dfw_decode_lanes_seq,
+    # one persistent launch per run of scopes (one for the whole 8B-shaped
+    # model), timed by the CUDA events around each step; the per-scope kernel
+    # launched one by one is reported beside it.  Windowed plan: one launch
+    # per scope, events around each.
     launch_ms = np.array(per_launch)  # [steps, blocks]
     mean_launch_ms = launch_ms.mean(axis=0)
-    achieved = alg_bytes / (mean_launch_ms.sum() * 1e-3) / 1e9
+    per_scope_achieved = alg_bytes / (mean_launch_ms.sum() * 1e-3) / 1e9
     peak, peak_kind = measured_peak_hbm()
-    kernel = "decode_lanes" if args.variant == "lanes" else "decode_tiles"
+    if lanes:
+        seq_launches = dfw.decode_lanes_seq_launches(devs)
+        kernel = "decode_lanes_multi"
+        achieved = alg_bytes / (ms_step * 1e-3) / 1e9
+        launches_per_step = seq_launches
+        mean_kernel_ms = ms_step / seq_launches
+        weights_per_launch = n_total / seq_launches
+    else:
+        kernel = "decode_tiles"
+        achieved = per_scope_achieved
+        launches_per_step = len(devs)
+        mean_kernel_ms = float(mean_launch_ms.mean())
+        weights_per_launch = n_total / len(devs)
     tpw = committed_traffic(kernel)
-    traffic = None if tpw is None else tpw * n_total / len(devs)
+    traffic = None if tpw is None else tpw * weights_per_launch
 
     e2e = None
     if not args.no_e2e:
@@ -952,9 +1043,8 @@ def main(argv=None):
                    "tile_windows": args.tile if args.variant == "window" else None,
                    "l2": guard.label("every scope's compressed form read, its bf16 written"),
                    "parallelism": f"replica{world}" if world > 1 else "single GPU",
-                   "launch": ("one dfw_decode_lanes_seq per step: one launch per scope, each a programmatic "
-                              "dependent of the previous" + (", captured once in a CUDA graph and replayed"
-                                                             if args.graph else "")
+                   "launch": ("one dfw_decode_lanes_seq per step: one persistent launch per run of up to 40 "
+                              "scopes" + (", captured once in a CUDA graph and replayed" if args.graph else "")
                               if lanes else "one dfw_decode_block per scope")},
         "effective_gbs": eff_gbs, "hbm_frac": eff_gbs / peak,
         "compression_ratio": 2 * n_total / comp, "compression_ratio_no_aux": 2 * n_total / comp_noaux,
@@ -963,10 +1053,17 @@ def main(argv=None):
                      "traffic": traffic, "peak_source": peak_kind,
                      "kernel": kernel,
                      "algorithmic_bytes_per_step": alg_bytes,
-                     "mean_launch_ms": float(mean_launch_ms.mean()),
-                     "timing": "per-launch CUDA events around each scope's launch, launched one by one",
-                     "one_by_one_ms_per_step": per_launch_step_ms},
-        "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": args.steps * len(devs),
+                     "launches_per_step": launches_per_step,
+                     "mean_launch_ms": mean_kernel_ms,
+                     "timing": ("CUDA events around each timed step (the step is the kernel's launches)" if lanes
+                                else "per-launch CUDA events around each scope's launch, launched one by one"),
+                     "per_scope_kernel": ({"kernel": "decode_lanes", "achieved": per_scope_achieved,
+                                           "frac": per_scope_achieved / peak,
+                                           "mean_launch_ms": float(mean_launch_ms.mean()),
+                                           "one_by_one_ms_per_step": per_launch_step_ms,
+                                           "timing": "CUDA events around each scope's launch, launched one by one"}
+                                          if lanes else None)},
+        "cpu_baseline": cpu, "clocks": clocks, "e2e": e2e, "gpu_launches": args.steps * launches_per_step,
         "verified_bit_exact": bool(ok),
     }
     if rank == 0:

@@ -224,6 +224,7 @@ dfw_status dfw_check(void *cuda_stream);
 #define DFW_ST_LUT 2u     /* a table entry or pointer is invalid */
 #define DFW_ST_RANGE 4u   /* plan offsets out of order or out of range */
 #define DFW_ST_TIMEOUT 8u /* a wait for a bulk copy gave up; the kernel returned early */
+#define DFW_ST_CHECK 16u  /* checks build only: an index or copy range left its buffer (the access was skipped) */
 
 /*
  * dfw_status_bits -- dfw_check, and the status bits it read and cleared in
@@ -243,6 +244,20 @@ dfw_status dfw_status_bits(void *cuda_stream, uint32_t *bits);
  * library's own.  Errors: DFW_ECUDA if the launch fails.
  */
 dfw_status dfw_selftest_wait_timeout(void *cuda_stream);
+
+/*
+ * dfw_checks_report -- the checks build (libdfw compiled with DFW_CHECKS,
+ * the library's stand-in for a memory checker): every copy range, shared-
+ * memory extent and output index the kernels compute is checked against its
+ * buffer before use; a failing access is skipped and reported through
+ * DFW_ST_CHECK and a site number (the first failing site is kept, sticky
+ * until read).  *enabled = 1 in the checks build, 0 in the ordinary one
+ * (whose kernels carry no checks); *site = the first failing site since the
+ * last call, 0 if none, then cleared.  Synchronises the device.  The pages
+ * describe no such build; it is the library's own.  Errors: DFW_EINVAL for
+ * null pointers, DFW_ECUDA if reading the device word fails.
+ */
+dfw_status dfw_checks_report(uint32_t *enabled, uint32_t *site);
 
 /*
  * KNOWN-START CHUNKS (a second decode plan over the same stream; the
@@ -369,13 +384,19 @@ typedef struct dfw_lanes_scope {
  * output buffer: transformer-block-level decompression of a model, block by
  * block, into one scratch buffer (DFloat11 abstract, point (iii)).  The
  * result is exactly that of k dfw_decode_lanes calls in order on cuda_stream:
- * scope i writes d_out[0, n_i) only after scope i - 1 has finished writing.
- * What differs is scheduling: from the second scope on, each launch is a
- * programmatic dependent of the one before, so it may start on SMs the
- * previous launch has left (loading its table, fetching and decoding its
- * first groups) and it holds its stores until that launch has completed.
- * Hence every scope's inputs must be complete when the call is made (all
- * earlier work on cuda_stream counts) and no input may overlap d_out.
+ * every byte of d_out ends as the last scope covering it wrote it.  What
+ * differs is scheduling: one persistent launch serves up to
+ * DFW_SEQ_MAX_SCOPES consecutive scopes.  Its warps keep the same 2048-weight
+ * output groups in every scope (group g of any scope is written by the same
+ * threads), so a later scope's writes follow an earlier one's in each
+ * thread's program order and no grid-wide barrier separates the scopes; each
+ * CTA switches fast tables between scopes, while its copies for the next
+ * scope's first groups are already in flight.  A new launch starts when the
+ * run limit is reached or a scope needs a smaller CTA (long codewords need
+ * bigger stream slots); it is a programmatic dependent of the previous one
+ * and holds its stores until that launch has completed.  Hence every scope's
+ * inputs must be complete when the call is made (all earlier work on
+ * cuda_stream counts) and no input may overlap d_out.
  *   scopes   host array of k scopes (k = 0 does nothing)
  *   d_out    max over scopes of n bf16, 16-byte aligned (32-byte alignment
  *            lets the kernel store whole 32-byte sectors)
@@ -383,7 +404,19 @@ typedef struct dfw_lanes_scope {
  * dfw_decode_lanes (nothing is launched on a host-side error); corrupt
  * streams or plans are flagged through dfw_check.  Asynchronous.
  */
+#define DFW_SEQ_MAX_SCOPES 40 /* scopes one launch of dfw_decode_lanes_seq serves */
+
 dfw_status dfw_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, void *cuda_stream);
+
+/*
+ * dfw_decode_lanes_seq_launches -- how many kernel launches
+ * dfw_decode_lanes_seq would make for these scopes (one per run of
+ * consecutive scopes that share a CTA shape, at most DFW_SEQ_MAX_SCOPES per
+ * run; empty scopes take none).  Host only: checks the scopes as the call
+ * would and launches nothing.  Errors as dfw_decode_lanes_seq's host-side
+ * checks; DFW_EINVAL for a null launches pointer.
+ */
+dfw_status dfw_decode_lanes_seq_launches(int k, const dfw_lanes_scope *scopes, int *launches);
 
 /*
  * dfw_decode_gemv_lanes -- decode fused with its consumer: y_i = W_i x_i for

@@ -276,22 +276,38 @@ def decode_lanes(dl: DeviceLanes, out: torch.Tensor | None = None, stream=None) 
     return out
 
 
+def _scope_array(dls):
+    arr = (LanesScope * len(dls))()
+    for i, d in enumerate(dls):
+        arr[i] = LanesScope(_ptr(d.stream), _ptr(d.mant), _ptr(d.lut), _ptr(d.chunk_bits), _ptr(d.group_start),
+                            ctypes.pointer(d.table), ctypes.pointer(d.info))
+    return arr
+
+
 def decode_lanes_seq(dls, out: torch.Tensor, stream=None) -> torch.Tensor:
     """Decodes the scopes ``dls`` one after another into ``out``
     (``dfw_decode_lanes_seq``): the same result as ``decode_lanes`` on each
-    in order, with each launch allowed to start while the previous drains.
-    ``out`` must hold the largest scope; returns it."""
+    in order, from one persistent launch per run of up to
+    ``DFW_SEQ_MAX_SCOPES`` scopes.  ``out`` must hold the largest scope;
+    returns it."""
     dls = list(dls)
     if not dls:
         return out
     if out.numel() < max(d.n for d in dls) or not out.is_contiguous():
         raise ValueError("out must be a contiguous tensor holding the largest scope")
-    arr = (LanesScope * len(dls))()
-    for i, d in enumerate(dls):
-        arr[i] = LanesScope(_ptr(d.stream), _ptr(d.mant), _ptr(d.lut), _ptr(d.chunk_bits), _ptr(d.group_start),
-                            ctypes.pointer(d.table), ctypes.pointer(d.info))
+    arr = _scope_array(dls)
     _check(lib().dfw_decode_lanes_seq(len(dls), arr, _ptr(out), _stream_handle(stream)), "dfw_decode_lanes_seq")
     return out
+
+
+def decode_lanes_seq_launches(dls) -> int:
+    """Kernel launches ``decode_lanes_seq`` makes for these scopes
+    (``dfw_decode_lanes_seq_launches``; host only)."""
+    dls = list(dls)
+    n = ctypes.c_int(0)
+    _check(lib().dfw_decode_lanes_seq_launches(len(dls), _scope_array(dls) if dls else None, ctypes.byref(n)),
+           "dfw_decode_lanes_seq_launches")
+    return int(n.value)
 
 
 def decode_gemv_lanes(dl: DeviceLanes, xs, cols, ys=None, partial: torch.Tensor | None = None,

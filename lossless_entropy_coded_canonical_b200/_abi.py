@@ -8,7 +8,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libdfw.so")
 
 OK, EINVAL, ECAP, ENOMEM, ECORRUPT, EALIGN, ECUDA = range(7)
-ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT = 1, 2, 4, 8  # device status bits (include/dfw.h DFW_ST_*)
+ST_COUNT, ST_LUT, ST_RANGE, ST_TIMEOUT, ST_CHECK = 1, 2, 4, 8, 16  # device status bits (include/dfw.h DFW_ST_*)
 FORMAT_VERSION = 1
 MAX_CAP = 32
 
@@ -86,7 +86,9 @@ SIGNATURES = {
     "dfw_plan_lanes": (_i, [_vp, _TP, _vp, _vp, _vp, _LP]),
     "dfw_decode_lanes": (_i, [_vp, _vp, _vp, _vp, _vp, _TP, _LP, _vp, _vp]),
     "dfw_decode_lanes_seq": (_i, [_i, _vp, _vp, _vp]),
+    "dfw_decode_lanes_seq_launches": (_i, [_i, _vp, _vp]),
     "dfw_status_bits": (_i, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+    "dfw_checks_report": (_i, [ctypes.POINTER(ctypes.c_uint32), ctypes.POINTER(ctypes.c_uint32)]),
     "dfw_container_bytes": (_u64, [_TP, _i, _i]),
     "dfw_container_write": (_i, [_TP, _i, _vp, _vp, _vp, _vp, _vp, _vp, _u64]),
     "dfw_container_read": (_i, [_vp, _u64, _TP, ctypes.POINTER(ContainerView)]),
@@ -107,14 +109,24 @@ SIGNATURES = {
 }
 
 
+def lib_path() -> str:
+    """The library this process uses: libdfw.so, or with DFW_LIBRARY=checks
+    in the environment the checks build libdfw_checks.so (every copy range,
+    shared-memory extent and output index checked before use)."""
+    if os.environ.get("DFW_LIBRARY", "") == "checks":
+        return os.path.join(os.path.dirname(LIB_PATH), "libdfw_checks.so")
+    return LIB_PATH
+
+
 def lib():
-    """Loads libdfw.so from the package directory; fails loudly if absent."""
+    """Loads the library from the package directory; fails loudly if absent."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libdfw.so is not built ({LIB_PATH}); run "
+        path = lib_path()
+        if not os.path.exists(path):
+            raise ImportError(f"{os.path.basename(path)} is not built ({path}); run "
                               "`python -m lossless_entropy_coded_canonical_b200.build`")
-        handle = ctypes.CDLL(LIB_PATH)
+        handle = ctypes.CDLL(path)
         for name, (res, args) in SIGNATURES.items():
             fn = getattr(handle, name)
             fn.restype = res

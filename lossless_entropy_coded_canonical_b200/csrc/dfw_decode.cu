@@ -39,7 +39,8 @@
 #include "dfw_internal.h"
 
 namespace dfw {
-__device__ unsigned int g_status;  // device status word (sticky error bits)
+__device__ unsigned int g_status;      // device status word (sticky error bits)
+__device__ unsigned int g_check_site;  // checks build: the first range check that failed (0: none)
 }
 
 #include "dfw_device.cuh"
@@ -163,11 +164,16 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
         const uint32_t sbytes = (uint32_t)min((uint64_t)L::SBUF, prm.stream_bytes - sb0);
         const bool ok = oe >= os && oe <= prm.n && oe - os + 32 <= prm.mbuf_bytes;
         const uint64_t m0 = os & ~15ull, m1 = (oe + 15) & ~15ull;
-        const uint32_t mbytes = ok ? (uint32_t)(m1 - m0) : 0u;
+        uint32_t mbytes = ok ? (uint32_t)(m1 - m0) : 0u;
+        const bool cp_ok = check(t < prm.n_tiles && sb0 < prm.stream_bytes && sbytes <= L::SBUF, CK_TILES_COPY);
+        if (!check(mbytes <= prm.mbuf_bytes && (mbytes == 0u || m1 <= ((prm.n + 15) & ~15ull)), CK_TILES_COPY))
+            mbytes = 0u;
         fence_proxy_async();
-        mbar_expect_tx(bar0 + 8 * s, sbytes + NT + mbytes);
-        bulk_load(smem_u32(slot), prm.stream + sb0, sbytes, bar0 + 8 * s);
-        bulk_load(smem_u32(slot + L::SBUF), prm.gap + t * NT, NT, bar0 + 8 * s);
+        mbar_expect_tx(bar0 + 8 * s, (cp_ok ? sbytes + NT : 0u) + mbytes);
+        if (cp_ok) {
+            bulk_load(smem_u32(slot), prm.stream + sb0, sbytes, bar0 + 8 * s);
+            bulk_load(smem_u32(slot + L::SBUF), prm.gap + t * NT, NT, bar0 + 8 * s);
+        }
         if (mbytes) bulk_load(smem_u32(slot + L::SBUF + NT), prm.mant + m0, mbytes, bar0 + 8 * s);
     };
 
@@ -239,6 +245,7 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
             const uint64_t rem = prm.total_bits - w * (8ull * W);
             const int wend = rem < 8ull * W ? (int)rem : 8 * W;
             cnt = decode_window<NSEG, NT>(wd, p, wend, s_fast, kshift, g_hier, prm.n_tables, s_priv + tid, err);
+            if (!check(cnt <= 4u * L::PRIV_WORDS, CK_TILES_WINDOW)) cnt = 0;
             if (err) atomicOr(&g_status, err);
         }
 
@@ -280,7 +287,7 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
             uint16_t *st = reinterpret_cast<uint16_t *>(ebuf);
             const uint8_t *mb = slot + L::SBUF + NT;
             const uint32_t b16 = (uint32_t)(os & 15u);
-            if (cnt) {
+            if (cnt && check(b16 + excl + cnt <= prm.ebuf_bytes && b16 + excl + cnt <= prm.mbuf_bytes, CK_TILES_WINDOW)) {
                 const uint32_t d = b16 + excl;
                 const uint32_t *src = s_priv + tid;
                 const uint32_t h = min((4u - (d & 3u)) & 3u, cnt);
@@ -310,7 +317,9 @@ __global__ void __launch_bounds__(NT) decode_tiles(const Params prm) {
 
             // store: the warp's range [lo_i, hi_i) of local indices; ot[i] is weight (os & ~15) + i
             uint16_t *ot = prm.out + (os & ~15ull);
-            const uint32_t lo_i = b16 + wbase, hi_i = lo_i + wcount;
+            const uint32_t lo_i = b16 + wbase;
+            uint32_t hi_i = lo_i + wcount;
+            if (!check((os & ~15ull) + hi_i <= prm.n, CK_TILES_STORE)) hi_i = lo_i;
             const uint32_t A = (lo_i + 7u) & ~7u, B = hi_i & ~7u;  // 16-byte aligned interior
             if (lane == 0 && B > A) bulk_store(ot + A, smem_u32(st + A), 2u * (B - A));
             if (lane < 8) {
@@ -493,7 +502,14 @@ extern "C" dfw_status dfw_decode_lanes_seq(int k, const dfw_lanes_scope *scopes,
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return DFW_ECUDA;
-    return launch_decode_lanes_seq(k, scopes, d_out, static_cast<cudaStream_t>(cuda_stream), sms);
+    return launch_decode_lanes_seq(k, scopes, d_out, static_cast<cudaStream_t>(cuda_stream), sms, nullptr, false);
+}
+
+extern "C" dfw_status dfw_decode_lanes_seq_launches(int k, const dfw_lanes_scope *scopes, int *launches) {
+    if (k < 0 || !launches || (k > 0 && !scopes)) return DFW_EINVAL;
+    *launches = 0;
+    if (k == 0) return DFW_OK;
+    return launch_decode_lanes_seq(k, scopes, nullptr, nullptr, 0, launches, true);
 }
 
 extern "C" dfw_status dfw_decode_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
@@ -543,6 +559,27 @@ extern "C" dfw_status dfw_status_bits(void *cuda_stream, uint32_t *bits) {
 }
 
 extern "C" dfw_status dfw_check(void *cuda_stream) { return dfw_status_bits(cuda_stream, nullptr); }
+
+namespace dfw {
+uint32_t take_encoder_check_site();  // dfw_encode.cu: the encoder kernels' own word (0 on failure to read)
+}
+
+extern "C" dfw_status dfw_checks_report(uint32_t *enabled, uint32_t *site) {
+    if (!enabled || !site) return DFW_EINVAL;
+#ifdef DFW_CHECKS
+    *enabled = 1u;
+#else
+    *enabled = 0u;
+#endif
+    *site = 0u;
+    if (cudaDeviceSynchronize() != cudaSuccess) return DFW_ECUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_check_site, sizeof(v)) != cudaSuccess) return DFW_ECUDA;
+    if (cudaMemcpyToSymbol(g_check_site, &zero, sizeof(zero)) != cudaSuccess) return DFW_ECUDA;
+    const uint32_t e = take_encoder_check_site();
+    *site = v ? v : e;
+    return DFW_OK;
+}
 
 namespace dfw {
 namespace {

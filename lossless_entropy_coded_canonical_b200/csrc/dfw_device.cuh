@@ -10,6 +10,22 @@ namespace dfw {
 namespace {
 
 constexpr uint32_t ESC_BAD = 0x40000000u;
+
+// The checks build (DFW_CHECKS): check(ok, site) records a failed range check
+// (status bit and the first failing site) and returns whether the access may
+// go ahead; in the ordinary build it is the constant true and costs nothing.
+#ifdef DFW_CHECKS
+__device__ __noinline__ void check_failed(uint32_t site) {
+    atomicOr(&g_status, ST_CHECK);
+    atomicCAS(&g_check_site, 0u, site);
+}
+__device__ __forceinline__ bool check(bool ok, uint32_t site) {
+    if (!ok) check_failed(site);
+    return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool check(bool, uint32_t) { return true; }
+#endif
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s, far above any copy
 
 // --------------------------------------------------------------- PTX helpers

@@ -44,6 +44,20 @@
 namespace dfw {
 namespace {
 
+// The checks build (DFW_CHECKS): the encoder kernels' own record of the first
+// range check that failed (this file's kernels have no status word); in the
+// ordinary build enc_check is the constant true.
+__device__ unsigned int g_enc_check_site;
+#ifdef DFW_CHECKS
+__device__ __noinline__ void enc_check_failed(uint32_t site) { atomicCAS(&g_enc_check_site, 0u, site); }
+__device__ __forceinline__ bool enc_check(bool ok, uint32_t site) {
+    if (!ok) enc_check_failed(site);
+    return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool enc_check(bool, uint32_t) { return true; }
+#endif
+
 constexpr int SPLIT_NT = 256;     // threads per CTA of pass 1
 constexpr int HIST_COPIES = 4;    // histogram copies per warp
 constexpr int GROUP_NT = 512;     // threads per CTA of passes 2 and 4
@@ -100,7 +114,8 @@ __global__ void __launch_bounds__(SPLIT_NT) enc_split_hist(const uint16_t *__res
         uint32_t m0, e0, m1, e1;
         split4(v.x, v.y, m0, e0);
         split4(v.z, v.w, m1, e1);
-        __stcs(reinterpret_cast<uint2 *>(mant) + i, make_uint2(m0, m1));
+        if (enc_check(8u * i + 8u <= mant_bytes, CK_ENC_SPLIT))
+            __stcs(reinterpret_cast<uint2 *>(mant) + i, make_uint2(m0, m1));
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             atomicAdd(hw + HIST_COPIES * ((e0 >> (8 * k)) & 0xFFu), 1u);
@@ -314,7 +329,8 @@ __global__ void __launch_bounds__(SCAN_NT) enc_zero_edges(const uint64_t *__rest
 
 __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict__ in, uint64_t n, const CodeTable ct,
                                                       const uint64_t *__restrict__ group_start, uint32_t n_groups,
-                                                      uint32_t *__restrict__ stream_words, uint32_t buf_words) {
+                                                      uint32_t *__restrict__ stream_words, uint64_t n_words,
+                                                      uint32_t buf_words) {
     extern __shared__ __align__(16) uint32_t s_dyn[];
     unsigned long long *s_lc = reinterpret_cast<unsigned long long *>(s_dyn);
     const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
@@ -367,6 +383,7 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
                 for (uint32_t k = 0; k < 8; ++k) v = (v << (uint32_t)(lc[k] >> 32)) | (uint32_t)lc[k];
                 const uint32_t sh = off & 31u, wi = off >> 5;
                 const unsigned long long a = v << (64u - b);  // first bit at bit 63
+                if (!enc_check(wi + ((sh + b + 31u) >> 5) <= buf_words, CK_ENC_PACK_BUF)) continue;
                 atomicOr(buf + wi, (uint32_t)(a >> (32u + sh)));
                 if (sh + b > 32u) atomicOr(buf + wi + 1, (uint32_t)(a >> sh));
                 if (sh + b > 64u) atomicOr(buf + wi + 2, (uint32_t)(a << (32u - sh)));
@@ -380,16 +397,17 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
                     acc = (acc << L) | (uint32_t)lc[k];
                     nacc += L;
                     if (nacc >= 32u) {
-                        atomicOr(buf + wi, (uint32_t)(acc >> (nacc - 32u)));
+                        if (enc_check(wi < buf_words, CK_ENC_PACK_BUF)) atomicOr(buf + wi, (uint32_t)(acc >> (nacc - 32u)));
                         ++wi;
                         nacc -= 32u;
                     }
                 }
-                if (nacc) atomicOr(buf + wi, (uint32_t)(acc << (32u - nacc)));
+                if (nacc && enc_check(wi < buf_words, CK_ENC_PACK_BUF)) atomicOr(buf + wi, (uint32_t)(acc << (32u - nacc)));
             }
         }
         __syncwarp();
-        const uint32_t nw = (uint32_t)((sh0 + (gs1 - gs0) + 31u) >> 5);
+        uint32_t nw = (uint32_t)((sh0 + (gs1 - gs0) + 31u) >> 5);
+        if (!enc_check(nw <= buf_words && (gs0 >> 5) + nw <= n_words, CK_ENC_PACK_STREAM)) nw = 0;
         uint32_t *dst = stream_words + (gs0 >> 5);
         for (uint32_t i = lane; i < nw; i += 32) {
             const uint32_t v = bswap32_dev(buf[i]);
@@ -405,6 +423,17 @@ __global__ void __launch_bounds__(GROUP_NT) enc_pack(const uint16_t *__restrict_
 }  // namespace dfw
 
 // ------------------------------------------------------------ host side
+
+namespace dfw {
+// Reads and clears the encoder kernels' check word (0 if none failed or the
+// read fails).
+uint32_t take_encoder_check_site() {
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_enc_check_site, sizeof(v)) != cudaSuccess) return 0u;
+    if (cudaMemcpyToSymbol(g_enc_check_site, &zero, sizeof(zero)) != cudaSuccess) return 0u;
+    return v;
+}
+}  // namespace dfw
 
 namespace {
 
@@ -677,7 +706,8 @@ extern "C" dfw_status dfw_pack_device(const uint16_t *d_bf16, const dfw_table *t
     const uint64_t want = (n_groups + GROUP_NT / 32 - 1) / (GROUP_NT / 32);
     const uint64_t cap_blocks = (uint64_t)sms * (uint64_t)std::max(1, per_sm);
     enc_pack<<<(unsigned)std::min(want, cap_blocks), GROUP_NT, smem, s>>>(
-        d_bf16, n, ct, d_group_start, (uint32_t)n_groups, reinterpret_cast<uint32_t *>(d_stream), buf_words);
+        d_bf16, n, ct, d_group_start, (uint32_t)n_groups, reinterpret_cast<uint32_t *>(d_stream),
+        table->stream_bytes / 4, buf_words);
     return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
 }
 

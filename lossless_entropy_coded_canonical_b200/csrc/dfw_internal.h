@@ -49,6 +49,28 @@ constexpr uint32_t ST_COUNT = 1u;   // a tile decoded a different number of code
 constexpr uint32_t ST_LUT = 2u;     // a LUT pointer left the table or a code ran past four levels
 constexpr uint32_t ST_RANGE = 4u;   // out_start out of order or beyond n, or tile too large
 constexpr uint32_t ST_TIMEOUT = 8u; // a wait for a bulk copy gave up (the kernel returned early)
+constexpr uint32_t ST_CHECK = 16u;  // checks build only: an index or range left its buffer (access skipped)
+
+// Sites of the checks build's range checks (the first failing one is kept).
+enum CheckSite : uint32_t {
+    CK_NONE = 0,
+    CK_LANES_STREAM_COPY = 1,   // a group's stream span or chunk bits beyond their buffers or slot
+    CK_LANES_MANT_COPY = 2,     // a group's raw bytes beyond their buffer
+    CK_LANES_READ_END = 3,      // a lane's stream reads ran past its warp's shared area
+    CK_LANES_SLOT_END = 4,      // a lane's exponent slots ran past their rows
+    CK_LANES_STORE = 5,         // an output store beyond n
+    CK_LANES_TABLE_COPY = 6,    // a fast table larger than its shared area
+    CK_FILL_READ = 7,           // a one-exponent fill read past the raw bytes
+    CK_TILES_COPY = 8,          // a tile's copies beyond their buffers or slots
+    CK_TILES_WINDOW = 9,        // a window's words or slots beyond their shared areas
+    CK_TILES_STORE = 10,        // a tile's output beyond n
+    CK_RANS_COPY = 11,          // a rANS block's copy beyond its buffer or slot
+    CK_RANS_READ = 12,          // a rANS reload beyond its block
+    CK_RANS_STORE = 13,         // a rANS output beyond n
+    CK_ENC_SPLIT = 14,          // encoder pass 1 beyond its buffers
+    CK_ENC_PACK_BUF = 15,       // encoder packing beyond its shared word buffer
+    CK_ENC_PACK_STREAM = 16,    // encoder packing beyond the stream
+};
 
 // A named range on profiler timelines (NVTX) for the duration of a call;
 // costs a function-pointer check when no tool is attached.

@@ -114,7 +114,8 @@ constexpr int LANES_ESC_DEC = 0x00FFFF00;
 // key) leaves it early.
 __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int left8, uint32_t fast,
                                                  uint32_t kshift, const uint32_t *__restrict__ g_hier,
-                                                 uint32_t n_tables, uint32_t ep, uint32_t &err) {
+                                                 uint32_t n_tables, uint32_t ep, uint32_t &err, uint32_t &rd_end,
+                                                 uint32_t &wr_end) {
     // p is the bit position (from sw); a and b hold the two stream words the
     // window [p, p + 32) lies in (the funnel shift takes p mod 32), c the
     // word after them (not yet byte-swapped), wa the address of the word
@@ -231,6 +232,8 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         if (left8 <= 0) break;
     }
     if (m != 1u) sts32(ep, lo);
+    rd_end = wa;  // one past the last stream word read
+    wr_end = ep;  // the last slot word written
     uint32_t end = p;
     if (left8 < 0) {
         // the last lookup (a fast entry) ran -left8 / 8 codewords past the
@@ -271,47 +274,57 @@ __device__ __forceinline__ void join16(uint32_t m_addr, uint32_t e_addr, uint4 &
 // l & 3 (16 weights) of chunk 8 j + l / 4, so each store instruction writes
 // eight whole 128-byte lines; the raw bytes it reads are one contiguous 512
 // bytes and its exponent words fall in 32 different banks.
+// Lane l writes weights 512 j + 16 l .. + 15 of group g (j = 0..3) in every
+// path below; the multi-scope kernel relies on that (a group's bytes are
+// written by the same lane whichever scope it belongs to).
+__device__ __forceinline__ void store_group(uint16_t *out, uint32_t out32, uint32_t n_chunks, uint32_t last_t,
+                                            uint32_t lane, uint32_t g, uint32_t mbuf, uint32_t exps0) {
+    const uint32_t i = lane & 3u, cl = lane >> 2;
+    const uint32_t mrow = mbuf + 16u * lane;                             // + 512 j
+    const uint32_t erow = exps0 + 4u * cl + 4u * EXP_STRIDE * i;         // + 32 j, + EXP_STRIDE per word
+    uint16_t *dst = out + (size_t)g * GROUP_SYMS + 16u * lane;         // + 512 j
+    const uint32_t c0 = g * GROUP_CHUNKS;
+    const bool whole = c0 + GROUP_CHUNKS < n_chunks || (c0 + GROUP_CHUNKS == n_chunks && last_t == LANE_SYMS);
+    if (!check(c0 < n_chunks, CK_LANES_STORE)) return;
+    if (whole && out32) {  // every group but the scope's last: no checks
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            uint4 r0, r1;
+            join16(mrow + 512u * j, erow + 32u * j, r0, r1);
+            stg256_cs(dst + 512u * j, r0, r1);  // a whole sector per lane, 1 KB per warp
+        }
+        return;
+    }
+#pragma unroll 1
+    for (int j = 0; j < 4; ++j) {
+        uint4 r0, r1;
+        join16(mrow + 512u * j, erow + 32u * j, r0, r1);
+        const uint32_t c = c0 + 8u * j + cl;
+        const uint32_t t = whole ? LANE_SYMS : (c + 1u < n_chunks ? LANE_SYMS : (c + 1u == n_chunks ? last_t : 0u));
+        if (16u * i + 16u <= t) {
+            if (out32) {
+                stg256_cs(dst + 512u * j, r0, r1);
+            } else {
+                __stcs(reinterpret_cast<uint4 *>(dst + 512u * j), r0);
+                __stcs(reinterpret_cast<uint4 *>(dst + 512u * j + 8u), r1);
+            }
+        } else {  // the last, partial chunk of the scope: one weight at a time
+            const uint32_t cw = 8u * j + cl;
+            for (uint32_t w = 16u * i; w < t; ++w) {
+                const uint32_t e = (lds32(exps0 + EXP_STRIDE * (w >> 2) + 4u * cw) >> (8u * (w & 3u))) & 0xFFu;
+                const uint32_t mb = (lds32(mbuf + 64u * cw + (w & ~3u)) >> (8u * (w & 3u))) & 0xFFu;
+                if (check(c0 + cw + 1u < n_chunks || (c0 + cw + 1u == n_chunks && w < last_t), CK_LANES_STORE))
+                    out[(size_t)(c0 + cw) * LANE_SYMS + w] = join1(e, mb);
+            }
+        }
+    }
+}
+
 struct StoreEpi {
     struct Params {};
     __device__ static __forceinline__ void apply(const LanesParams &prm, const Params &, uint32_t lane, uint32_t g,
                                                  uint32_t mbuf, uint32_t exps0) {
-        const uint32_t i = lane & 3u, cl = lane >> 2;
-        const uint32_t mrow = mbuf + 16u * lane;                             // + 512 j
-        const uint32_t erow = exps0 + 4u * cl + 4u * EXP_STRIDE * i;         // + 32 j, + EXP_STRIDE per word
-        uint16_t *dst = prm.out + (size_t)g * GROUP_SYMS + 16u * lane;     // + 512 j
-        const uint32_t c0 = g * GROUP_CHUNKS;
-        const bool whole = c0 + GROUP_CHUNKS < prm.n_chunks ||
-                           (c0 + GROUP_CHUNKS == prm.n_chunks && prm.last_t == LANE_SYMS);
-        if (whole && prm.out32) {  // every group but the scope's last: no checks
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                uint4 r0, r1;
-                join16(mrow + 512u * j, erow + 32u * j, r0, r1);
-                stg256_cs(dst + 512u * j, r0, r1);  // a whole sector per lane, 1 KB per warp
-            }
-            return;
-        }
-#pragma unroll 1
-        for (int j = 0; j < 4; ++j) {
-            uint4 r0, r1;
-            join16(mrow + 512u * j, erow + 32u * j, r0, r1);
-            const uint32_t t = whole ? LANE_SYMS : chunk_weights(prm, c0 + 8u * j + cl);
-            if (16u * i + 16u <= t) {
-                if (prm.out32) {
-                    stg256_cs(dst + 512u * j, r0, r1);
-                } else {
-                    __stcs(reinterpret_cast<uint4 *>(dst + 512u * j), r0);
-                    __stcs(reinterpret_cast<uint4 *>(dst + 512u * j + 8u), r1);
-                }
-            } else {  // the last, partial chunk of the scope: one weight at a time
-                const uint32_t cw = 8u * j + cl;
-                for (uint32_t w = 16u * i; w < t; ++w) {
-                    const uint32_t e = (lds32(exps0 + EXP_STRIDE * (w >> 2) + 4u * cw) >> (8u * (w & 3u))) & 0xFFu;
-                    const uint32_t mb = (lds32(mbuf + 64u * cw + (w & ~3u)) >> (8u * (w & 3u))) & 0xFFu;
-                    prm.out[(size_t)(c0 + cw) * LANE_SYMS + w] = join1(e, mb);
-                }
-            }
-        }
+        store_group(prm.out, prm.out32, prm.n_chunks, prm.last_t, lane, g, mbuf, exps0);
     }
 };
 
@@ -373,6 +386,28 @@ __host__ __device__ constexpr uint32_t warp_smem_bytes(uint32_t sbuf_bytes) {
     return 32u + 2u * (64u + sbuf_bytes) + GROUP_SYMS + EXP_BYTES;
 }
 static_assert(warp_smem_bytes(16u) % 16u == 0u, "per-warp shared areas must stay 16-byte aligned");
+
+// Checks this thread's share of the fast table in shared memory (every
+// entry of 2^fast_bits) and gives escapes the loop's escape word; true if an
+// entry is malformed.
+template <int NT>
+__device__ __forceinline__ bool check_fast_table(uint2 *s_fast, uint32_t n_fast, uint32_t fast_bits, int tid) {
+    bool bad = false;
+    for (uint32_t i = tid; i < n_fast; i += NT) {
+        uint2 e = s_fast[i];
+        if (e.y & FAST_ESC) {
+            bad |= e.y != FAST_ESC_WORD || e.x != 0u;
+            s_fast[i].y = LANES_ESC_WORD;
+        } else {
+            const uint32_t cb = e.y & 255u, c8 = (e.y >> FAST_C8_SHIFT) & 255u,
+                           ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
+            bad |= c8 == 0u || (c8 & 7u) || c8 > 8u * FAST_MAX_SYMS || cb == 0u || cb > fast_bits ||
+                   8u * cb < c8 || (uint32_t)__popc(ends) * 8u != c8 || (ends >> (cb - 1u)) != 1u ||
+                   (e.y & 0x70000000u) || (c8 < 32u && (e.x >> c8) != 0u);
+        }
+    }
+    return bad;
+}
 
 template <int NT, class Epi>
 __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const typename Epi::Params ep) {
@@ -436,20 +471,7 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         return;
     }
     // check every entry; escapes get the loop's escape word
-    bool bad = false;
-    for (uint32_t i = tid; i < n_fast; i += NT) {
-        uint2 e = s_fast[i];
-        if (e.y & FAST_ESC) {
-            bad |= e.y != FAST_ESC_WORD || e.x != 0u;
-            s_fast[i].y = LANES_ESC_WORD;
-        } else {
-            const uint32_t cb = e.y & 255u, c8 = (e.y >> FAST_C8_SHIFT) & 255u,
-                           ends = (e.y >> FAST_ENDS_SHIFT) & 0xFFFu;
-            bad |= c8 == 0u || (c8 & 7u) || c8 > 8u * FAST_MAX_SYMS || cb == 0u || cb > prm.fast_bits ||
-                   8u * cb < c8 || (uint32_t)__popc(ends) * 8u != c8 || (ends >> (cb - 1u)) != 1u ||
-                   (e.y & 0x70000000u) || (c8 < 32u && (e.x >> c8) != 0u);
-        }
-    }
+    const bool bad = check_fast_table<NT>(s_fast, n_fast, prm.fast_bits, tid);
     if (__syncthreads_or(bad)) {
         if (tid == 0) atomicOr(&g_status, ST_LUT);
         return;
@@ -469,18 +491,22 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
             sbytes = min(span_bytes((uint32_t)s0 & 127u, d < (1u << 17) ? (uint32_t)d : (1u << 17)), prm.sbuf_bytes);
             sbytes = (uint32_t)min((uint64_t)sbytes, prm.stream_bytes - sb0);
         }
+        const bool cb_ok = check(gg < prm.n_groups, CK_LANES_STREAM_COPY);
+        const bool st_ok = check(sbytes <= prm.sbuf_bytes && (sbytes == 0u || sb0 + sbytes <= prm.stream_bytes),
+                                 CK_LANES_STREAM_COPY);
         fence_proxy_async();
-        mbar_expect_tx(bar, 64u + sbytes);
-        bulk_load(smem_u32(slot), prm.chunk_bits + (size_t)gg * GROUP_CHUNKS, 64u, bar);
-        if (sbytes) bulk_load(smem_u32(slot + 64), prm.stream + sb0, sbytes, bar);
+        mbar_expect_tx(bar, (cb_ok ? 64u : 0u) + (st_ok ? sbytes : 0u));
+        if (cb_ok) bulk_load(smem_u32(slot), prm.chunk_bits + (size_t)gg * GROUP_CHUNKS, 64u, bar);
+        if (st_ok && sbytes) bulk_load(smem_u32(slot + 64), prm.stream + sb0, sbytes, bar);
     };
     // lane 0: the group's raw bytes into the warp buffer
     auto issue_mant = [&](uint32_t gg) {
         const uint64_t m0 = (uint64_t)gg * GROUP_SYMS;
         const uint32_t bytes = (uint32_t)min((uint64_t)GROUP_SYMS, prm.mant_bytes - m0);
+        const bool ok = check(m0 < prm.mant_bytes && m0 + bytes <= prm.mant_bytes, CK_LANES_MANT_COPY);
         fence_proxy_async();
-        mbar_expect_tx(bar_m, bytes);
-        bulk_load(smem_u32(mbuf), prm.mant + m0, bytes, bar_m);
+        mbar_expect_tx(bar_m, ok ? bytes : 0u);
+        if (ok) bulk_load(smem_u32(mbuf), prm.mant + m0, bytes, bar_m);
     };
 
     if (lane == 0) {
@@ -516,9 +542,12 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         uint32_t err = 0;
         if (ok && valid && t) {
             const uint32_t r = r0 + excl;
+            uint32_t rd_end, wr_end;
             const uint32_t end = decode_chunk(smem_u32(slot + 64), r, (int)(8u * t), smem_u32(s_fast), kshift,
-                                              g_hier, prm.n_tables, exps, err);
+                                              g_hier, prm.n_tables, exps, err, rd_end, wr_end);
             if (end != r + cbits) err |= ST_COUNT;
+            check(rd_end <= smem_u32(wbase) + wbytes, CK_LANES_READ_END);
+            check(wr_end < exps + EXP_STRIDE * EXP_WORDS, CK_LANES_SLOT_END);
         }
         // starts two groups ahead, for the copy issued next round: loaded
         // after the decode loop, so they hold no registers during it, and
@@ -560,6 +589,409 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
         ns0 = ms0;
         ns1 = ms1;
     }
+}
+
+// ------------------------------------------------------------ many scopes, one launch
+//
+// A sequence of code-table scopes (a model's blocks) decoded by one
+// persistent launch into one output buffer.  Warp slot w (numbered
+// warp-major across CTAs, as in decode_lanes) takes groups w, w + S, w + 2S,
+// ... (S = resident warps) of every scope in turn, and within a group lane l
+// always writes the same weights (store_group), so any output byte is written
+// by one thread in every scope: the scopes' writes land in order by program
+// order alone, and the buffer ends as k separate decodes in order would leave
+// it, with no barrier between scopes across the grid.  Per scope each CTA
+// loads that scope's fast table after a CTA barrier (every warp is done with
+// the previous one); a warp's copies for its next group, which may belong to
+// a later scope, are issued one group ahead as in decode_lanes, so they are
+// in flight across the table switch.  One-exponent scopes are filled from
+// their raw bytes with the same lane-to-weight layout.  Control flow over the
+// scopes is uniform across the CTA: a warp whose copy wait gave up stops
+// decoding but still takes every CTA barrier.
+
+struct SeqScope {
+    const uint8_t *stream;
+    const uint8_t *mant;
+    const uint32_t *lut;
+    const uint16_t *chunk_bits;
+    const uint64_t *group_start;
+    uint64_t stream_bytes, mant_bytes;
+    uint32_t n_chunks, n_groups;  // n_groups == 0: an empty scope
+    uint32_t last_t;              // codewords in the last chunk (1..64)
+    uint32_t fast_bits;           // 0: one distinct exponent (fill)
+    uint32_t n_tables;            // hierarchy tables, or the exponent of a one-exponent scope
+    uint32_t reserved;
+};
+
+constexpr uint32_t SEQ_MAX_SCOPES = DFW_SEQ_MAX_SCOPES;
+
+struct SeqParams {
+    uint16_t *out;
+    uint32_t k;               // scopes in this launch
+    uint32_t out32;           // out is 32-byte aligned
+    uint32_t wait_prior;      // a programmatic dependent of an earlier decode into out
+    uint32_t sbuf_bytes;      // stream slot bytes (the largest group span of the launch's scopes)
+    uint32_t fast_bytes;      // shared bytes of the fast table (the largest of the launch's scopes)
+    uint32_t reserved;
+    SeqScope sc[SEQ_MAX_SCOPES];
+};
+static_assert(sizeof(SeqParams) <= 4096, "kernel parameters stay within the classic 4 KB limit");
+
+// One-exponent scope: the warp's groups filled from their raw bytes.
+__device__ __forceinline__ void fill_groups(const SeqScope &S, uint16_t *out, uint32_t out32, uint32_t slot0,
+                                            uint32_t gstride, uint32_t lane) {
+    const uint32_t R = rot_sym(S.n_tables) * 0x01010101u;
+    const uint64_t n = (uint64_t)(S.n_chunks - 1u) * LANE_SYMS + S.last_t;
+    for (uint32_t g = slot0; g < S.n_groups; g += gstride) {
+        const uint64_t w0 = (uint64_t)g * GROUP_SYMS + 16u * lane;  // + 512 j
+        for (int j = 0; j < 4; ++j) {
+            const uint64_t w = w0 + 512u * j;
+            if (w >= n) break;
+            if (!check(w + 16u <= S.mant_bytes, CK_FILL_READ)) break;
+            const uint4 m = __ldcs(reinterpret_cast<const uint4 *>(S.mant + w));  // w + 16 <= mant_bytes
+            uint4 r0, r1;
+            join4(R, m.x, r0.x, r0.y);
+            join4(R, m.y, r0.z, r0.w);
+            join4(R, m.z, r1.x, r1.y);
+            join4(R, m.w, r1.z, r1.w);
+            if (w + 16u <= n) {
+                if (out32) {
+                    stg256_cs(out + w, r0, r1);
+                } else {
+                    __stcs(reinterpret_cast<uint4 *>(out + w), r0);
+                    __stcs(reinterpret_cast<uint4 *>(out + w + 8u), r1);
+                }
+            } else {  // the scope's last weights, one at a time
+                for (uint32_t q = 0; w + q < n; ++q) {
+                    const uint32_t mq = q < 4u ? m.x : q < 8u ? m.y : q < 12u ? m.z : m.w;
+                    out[w + q] = join1(rot_sym(S.n_tables), (mq >> (8u * (q & 3u))) & 0xFFu);
+                }
+            }
+        }
+    }
+}
+
+template <int NT>
+__global__ void __launch_bounds__(NT, 1) decode_lanes_multi(const SeqParams P) {
+    constexpr int NWARP = NT / 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    uint2 *s_fast = reinterpret_cast<uint2 *>(smem);
+    const uint32_t wbytes = warp_smem_bytes(P.sbuf_bytes);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint8_t *wbase = smem + P.fast_bytes + warp * wbytes;
+    const uint32_t bar_s0 = smem_u32(wbase), bar_m = bar_s0 + 16u;
+    uint8_t *wslots = wbase + 32;
+    const uint32_t slot_bytes = 64u + P.sbuf_bytes;
+    uint8_t *mbuf = wslots + 2u * slot_bytes;
+    const uint32_t exps0 = smem_u32(mbuf + GROUP_SYMS), exps = exps0 + 4u * lane;
+    const uint32_t bar_t = smem_u32(smem + P.fast_bytes) + 24u;  // spare word of warp 0's barriers
+    griddep_launch_dependents();
+
+    const uint32_t gstride = gridDim.x * NWARP;
+    // this warp's slot, recomputed where needed (off the per-group path)
+    auto slot_of = [&]() -> uint32_t { return (threadIdx.x >> 5) * gridDim.x + blockIdx.x; };
+    // this warp's decode work is the sequence of (scope, group) pairs with a
+    // stream: groups slot0, slot0 + gstride, ... of each such scope in turn
+    auto first_from = [&](uint32_t j) -> uint32_t {
+        const uint32_t slot0 = slot_of();
+        while (j < P.k && (P.sc[j].fast_bits == 0u || slot0 >= P.sc[j].n_groups)) ++j;
+        return j;
+    };
+    auto advance = [&](uint32_t &j, uint32_t &g) {
+        g += gstride;
+        if (g >= P.sc[j].n_groups) {
+            j = first_from(j + 1u);
+            g = slot_of();
+        }
+    };
+    uint32_t jc = first_from(0), gc = slot_of();  // the group this warp decodes next (number kc)
+    uint32_t jn = jc, gn = gc;                 // the one after it (kc + 1)
+    if (jn < P.k) advance(jn, gn);
+    // Group starts reach the lanes through shared memory: the 8 bytes at the
+    // end of each exponent-slot row (bytes 128..135 of the 136) are never used
+    // by the slots, so rows 0..3 hold the starts of group kc in pair kc & 1.
+    // Lane 0 loads group kc + 2's starts after a decode loop, keeps them in
+    // registers until the top of the next iteration (no decode loop in
+    // between), then stores them and issues that group's stream copy.
+    auto stash = [&](uint32_t pair, uint32_t which) { return exps0 + EXP_STRIDE * (2u * pair + which) + 128u; };
+    auto lds64 = [](uint32_t a) {
+        uint64_t v;
+        asm volatile("ld.shared.u64 %0, [%1];" : "=l"(v) : "r"(a) : "memory");
+        return v;
+    };
+    auto sts64 = [](uint32_t a, uint64_t v) { asm volatile("st.shared.u64 [%0], %1;" ::"r"(a), "l"(v) : "memory"); };
+
+    // The first scope with a table: its copy goes out right after the
+    // barriers are set up (every warp waits for it; each warp's first group
+    // copies follow once it is in, as in decode_lanes).
+    uint32_t j0 = 0;
+    while (j0 < P.k && (P.sc[j0].fast_bits == 0u || P.sc[j0].n_groups == 0u)) ++j0;
+    if (lane == 0) {
+        mbar_init(bar_s0, 1);
+        mbar_init(bar_s0 + 8u, 1);
+        mbar_init(bar_m, 1);
+        if (tid == 0) mbar_init(bar_t, 1);
+        fence_mbar_init();
+        if (tid == 0 && j0 < P.k) {
+            mbar_expect_tx(bar_t, 8u << P.sc[j0].fast_bits);
+            bulk_load(smem_u32(s_fast), P.sc[j0].lut, 8u << P.sc[j0].fast_bits, bar_t);
+        }
+    }
+    __syncthreads();  // the barriers are initialised
+
+    // lane 0: chunk_bits and stream span of group gg of scope jj into slot s
+    auto issue_stream = [&](uint32_t jj, uint32_t gg, uint32_t s, uint64_t s0, uint64_t s1) {
+        const SeqScope &S = P.sc[jj];
+        uint8_t *slot = wslots + s * slot_bytes;
+        const uint32_t bar = bar_s0 + 8u * s;
+        const uint64_t sb0 = (s0 >> 3) & ~15ull;
+        uint32_t sbytes = 0;
+        if (sb0 < S.stream_bytes) {
+            const uint64_t d = s1 - s0;
+            sbytes = min(span_bytes((uint32_t)s0 & 127u, d < (1u << 17) ? (uint32_t)d : (1u << 17)), P.sbuf_bytes);
+            sbytes = (uint32_t)min((uint64_t)sbytes, S.stream_bytes - sb0);
+        }
+        const bool cb_ok = check(gg < S.n_groups, CK_LANES_STREAM_COPY);
+        const bool st_ok = check(sbytes <= P.sbuf_bytes && (sbytes == 0u || sb0 + sbytes <= S.stream_bytes),
+                                 CK_LANES_STREAM_COPY);
+        fence_proxy_async();
+        mbar_expect_tx(bar, (cb_ok ? 64u : 0u) + (st_ok ? sbytes : 0u));
+        if (cb_ok) bulk_load(smem_u32(slot), S.chunk_bits + (size_t)gg * GROUP_CHUNKS, 64u, bar);
+        if (st_ok && sbytes) bulk_load(smem_u32(slot + 64), S.stream + sb0, sbytes, bar);
+    };
+    // lane 0: the raw bytes of group gg of scope jj into the warp buffer
+    auto issue_mant = [&](uint32_t jj, uint32_t gg) {
+        const SeqScope &S = P.sc[jj];
+        const uint64_t m0 = (uint64_t)gg * GROUP_SYMS;
+        const uint32_t bytes = (uint32_t)min((uint64_t)GROUP_SYMS, S.mant_bytes - m0);
+        const bool ok = check(m0 < S.mant_bytes && m0 + bytes <= S.mant_bytes, CK_LANES_MANT_COPY);
+        fence_proxy_async();
+        mbar_expect_tx(bar_m, ok ? bytes : 0u);
+        if (ok) bulk_load(smem_u32(mbuf), S.mant + m0, bytes, bar_m);
+    };
+    uint64_t ms0 = 0, ms1 = 0;  // lane 0: the starts of group kc + 1, waiting to be stored and issued
+    uint64_t a0 = 0, a1 = 0;    // lane 0: the first group's starts (its copies go out after the first table)
+    if (lane == 0 && jc < P.k) {
+        a0 = __ldg(P.sc[jc].group_start + gc);
+        a1 = __ldg(P.sc[jc].group_start + gc + 1);
+        if (jn < P.k) {
+            ms0 = __ldg(P.sc[jn].group_start + gn);
+            ms1 = __ldg(P.sc[jn].group_start + gn + 1);
+        }
+    }
+
+    uint32_t kc = 0;        // groups this warp has taken (slot, phase and stash bookkeeping)
+    uint32_t tphase = 0;    // phase of the table barrier
+    // a launch chained after another decode into out holds its first store
+    // (and everything after it) until that launch has completed
+    if (P.wait_prior) griddep_wait();
+    for (uint32_t j = 0; j < P.k; ++j) {  // uniform across the CTA
+        const uint32_t fb = P.sc[j].fast_bits;
+        if (P.sc[j].n_groups == 0u) continue;
+        if (fb == 0u) {  // one distinct exponent: no table, no stream
+            const uint32_t slot0 = slot_of();
+            if (slot0 < P.sc[j].n_groups && jc <= P.k) fill_groups(P.sc[j], P.out, P.out32, slot0, gstride, lane);
+            continue;
+        }
+        // scope j's fast table replaces the previous one once every warp is
+        // done with it (the first one is already on its way)
+        if (j != j0) {
+            __syncthreads();
+            if (tid == 0) {
+                const bool ok = check((8u << fb) <= P.fast_bytes, CK_LANES_TABLE_COPY);
+                fence_proxy_async();
+                mbar_expect_tx(bar_t, ok ? 8u << fb : 0u);
+                if (ok) bulk_load(smem_u32(s_fast), P.sc[j].lut, 8u << fb, bar_t);
+            }
+        }
+        if (tid == 0) {
+            for (uint32_t jj = j + 1u; jj < P.k; ++jj)  // the next table, into L2 meanwhile
+                if (P.sc[jj].fast_bits && P.sc[jj].n_groups) {
+                    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(P.sc[jj].lut),
+                                 "r"(8u << P.sc[jj].fast_bits)
+                                 : "memory");
+                    break;
+                }
+        }
+        const bool tok = mbar_wait(bar_t, tphase);
+        tphase ^= 1u;
+        if (!__syncthreads_and(tok)) {  // the table copy never completed: give up, after the copies in flight
+            if (tid == 0) {
+                atomicOr(&g_status, ST_TIMEOUT);
+                mbar_wait_bounded(bar_t, tphase ^ 1u);
+            }
+            if (lane == 0 && jc < P.k && kc > 0u) {  // (a warp's first copies go out after the first table)
+                mbar_wait_bounded(bar_s0 + 8u * (kc & 1u), (kc >> 1) & 1u);
+                mbar_wait_bounded(bar_m, kc & 1u);
+            }
+            return;
+        }
+        const bool table_ok = !__syncthreads_or(check_fast_table<NT>(s_fast, 1u << fb, fb, tid));
+        if (!table_ok && tid == 0) atomicOr(&g_status, ST_LUT);
+        // Scope j's fields, read once here: j is the same across the CTA, so
+        // these stay uniform values for the group loop below instead of
+        // indexed parameter loads on every group.  The next group is in
+        // scope j too except at a warp's last group of the scope.
+        const uint8_t *const j_stream = P.sc[j].stream;
+        const uint8_t *const j_mant = P.sc[j].mant;
+        const uint32_t *const j_lut = P.sc[j].lut;
+        const uint16_t *const j_chunk_bits = P.sc[j].chunk_bits;
+        const uint64_t *const j_group_start = P.sc[j].group_start;
+        const uint64_t j_stream_bytes = P.sc[j].stream_bytes, j_mant_bytes = P.sc[j].mant_bytes;
+        const uint32_t j_n_chunks = P.sc[j].n_chunks, j_n_groups = P.sc[j].n_groups, j_last_t = P.sc[j].last_t;
+        const uint32_t j_n_tables = P.sc[j].n_tables;
+        // lane 0: copies of group gg (scope jj) into slot s; starts s0, s1
+        auto issue_next_stream = [&](uint32_t jj, uint32_t gg, uint32_t s, uint64_t s0, uint64_t s1) {
+            if (jj != j) {
+                issue_stream(jj, gg, s, s0, s1);
+                return;
+            }
+            uint8_t *slot = wslots + s * slot_bytes;
+            const uint32_t bar = bar_s0 + 8u * s;
+            const uint64_t sb0 = (s0 >> 3) & ~15ull;
+            uint32_t sbytes = 0;
+            if (sb0 < j_stream_bytes) {
+                const uint64_t d = s1 - s0;
+                sbytes = min(span_bytes((uint32_t)s0 & 127u, d < (1u << 17) ? (uint32_t)d : (1u << 17)),
+                             P.sbuf_bytes);
+                sbytes = (uint32_t)min((uint64_t)sbytes, j_stream_bytes - sb0);
+            }
+            const bool cb_ok = check(gg < j_n_groups, CK_LANES_STREAM_COPY);
+            const bool st_ok = check(sbytes <= P.sbuf_bytes && (sbytes == 0u || sb0 + sbytes <= j_stream_bytes),
+                                     CK_LANES_STREAM_COPY);
+            fence_proxy_async();
+            mbar_expect_tx(bar, (cb_ok ? 64u : 0u) + (st_ok ? sbytes : 0u));
+            if (cb_ok) bulk_load(smem_u32(slot), j_chunk_bits + (size_t)gg * GROUP_CHUNKS, 64u, bar);
+            if (st_ok && sbytes) bulk_load(smem_u32(slot + 64), j_stream + sb0, sbytes, bar);
+        };
+        auto issue_next_mant = [&](uint32_t jj, uint32_t gg) {
+            if (jj != j) {
+                issue_mant(jj, gg);
+                return;
+            }
+            const uint64_t m0 = (uint64_t)gg * GROUP_SYMS;
+            const uint32_t bytes = (uint32_t)min((uint64_t)GROUP_SYMS, j_mant_bytes - m0);
+            const bool ok = check(m0 < j_mant_bytes && m0 + bytes <= j_mant_bytes, CK_LANES_MANT_COPY);
+            fence_proxy_async();
+            mbar_expect_tx(bar_m, ok ? bytes : 0u);
+            if (ok) bulk_load(smem_u32(mbuf), j_mant + m0, bytes, bar_m);
+        };
+
+        while (jc == j) {  // this warp's groups of scope j
+            const uint32_t s = kc & 1u;
+            const uint8_t *slot = wslots + s * slot_bytes;
+            const bool has_next = jn < P.k;
+            __syncwarp();  // every lane is done with the other slot and with stash pair s ^ 1
+            if (kc == 0u && lane == 0) {  // the warp's first group: its starts and copies
+                sts64(stash(0, 0), a0);
+                sts64(stash(0, 1), a1);
+                issue_next_stream(jc, gc, 0, a0, a1);
+                issue_next_mant(jc, gc);
+            }
+            if (has_next && lane == 0) {
+                sts64(stash(s ^ 1u, 0), ms0);
+                sts64(stash(s ^ 1u, 1), ms1);
+                issue_next_stream(jn, gn, s ^ 1u, ms0, ms1);
+            }
+
+            bool ok = mbar_wait(bar_s0 + 8u * s, (kc >> 1) & 1u);
+            const uint64_t gs0 = lds64(stash(s, 0)), gs1 = lds64(stash(s, 1));
+            const uint32_t cbits = reinterpret_cast<const uint16_t *>(slot)[lane];
+            uint32_t incl = cbits;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+                if (lane >= d) incl += y;
+            }
+            const uint32_t excl = incl - cbits, gbits = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            const uint32_t c = gc * GROUP_CHUNKS + lane;
+            const uint32_t t = c + 1u < j_n_chunks ? LANE_SYMS : (c + 1u == j_n_chunks ? j_last_t : 0u);
+            const uint32_t r0 = (uint32_t)gs0 & 127u;
+            const uint32_t span = span_bytes(r0, gbits);
+            const bool valid = __all_sync(0xFFFFFFFFu, gs1 - gs0 == gbits && cbits <= 32u * LANE_SYMS &&
+                                                           span <= P.sbuf_bytes &&
+                                                           ((gs0 >> 3) & ~15ull) + span <= j_stream_bytes &&
+                                                           (t != 0u || cbits == 0u));
+            uint32_t err = 0;
+            if (ok && valid && table_ok && t) {
+                const uint32_t r = r0 + excl;
+                uint32_t rd_end, wr_end;
+                const uint32_t end = decode_chunk(smem_u32(slot + 64), r, (int)(8u * t), smem_u32(s_fast), 32u - fb,
+                                                  j_lut + (2u << fb), j_n_tables, exps, err, rd_end, wr_end);
+                if (end != r + cbits) err |= ST_COUNT;
+                check(rd_end <= smem_u32(wbase) + wbytes, CK_LANES_READ_END);
+                check(wr_end < exps + EXP_STRIDE * EXP_WORDS, CK_LANES_SLOT_END);
+            }
+            // move on: the current group is kept only as gcur (for the store);
+            // (jc, gc) becomes the next group, (jn, gn) the one after it, whose
+            // starts lane 0 loads now
+            const uint32_t gcur = gc;
+            jc = jn;
+            gc = gn;
+            if (has_next) {
+                gn += gstride;
+                if (gn >= (jn == j ? j_n_groups : P.sc[jn].n_groups)) {
+                    jn = first_from(jn + 1u);
+                    gn = slot_of();
+                }
+                if (jn < P.k && lane == 0) {
+                    const uint64_t *gsp = (jn == j ? j_group_start : P.sc[jn].group_start) + gn;
+                    ms0 = __ldg(gsp);
+                    ms1 = __ldg(gsp + 1);
+                }
+            }
+            ok = mbar_wait(bar_m, kc & 1u) && ok;
+            if (!__all_sync(0xFFFFFFFFu, ok)) {  // a copy never completed: this warp stops decoding
+                if (lane == 0) {
+                    atomicOr(&g_status, ST_TIMEOUT);
+                    mbar_wait_bounded(bar_s0 + 8u * s, (kc >> 1) & 1u);
+                    mbar_wait_bounded(bar_m, kc & 1u);
+                    if (has_next) mbar_wait_bounded(bar_s0 + 8u * (s ^ 1u), ((kc + 1) >> 1) & 1u);
+                }
+                jc = P.k + 1u;  // past every scope: no more groups, no fills; the CTA barriers still come
+                break;
+            }
+            const bool good = valid && table_ok && !__any_sync(0xFFFFFFFFu, err != 0u);
+            if (!valid) {
+                if (lane == 0) atomicOr(&g_status, ST_RANGE);
+            } else if (good) {
+                __syncwarp();  // the join reads other lanes' exponent slots
+                store_group(P.out, P.out32, j_n_chunks, j_last_t, lane, gcur, smem_u32(mbuf), exps0);
+            } else if (err) {
+                atomicOr(&g_status, err);
+            }
+            __syncwarp();  // all lanes have read the raw bytes
+            if (has_next && lane == 0) issue_next_mant(jc, gc);
+            ++kc;
+        }
+    }
+}
+
+template <int NT>
+uint32_t lanes_multi_smem(uint32_t fast_bytes, uint32_t sbuf_bytes) {
+    return fast_bytes + (NT / 32) * warp_smem_bytes(sbuf_bytes);
+}
+
+struct MultiVariant {
+    int nt;
+    void (*fn)(const SeqParams);
+    uint32_t (*smem)(uint32_t, uint32_t);
+    int smem_set[16];
+};
+static MultiVariant g_multi[5] = {
+    {1024, decode_lanes_multi<1024>, lanes_multi_smem<1024>, {0}},
+    {768, decode_lanes_multi<768>, lanes_multi_smem<768>, {0}},
+    {512, decode_lanes_multi<512>, lanes_multi_smem<512>, {0}},
+    {256, decode_lanes_multi<256>, lanes_multi_smem<256>, {0}},
+    {128, decode_lanes_multi<128>, lanes_multi_smem<128>, {0}},
+};
+
+// The largest CTA whose shared memory fits (fast table + per-warp areas);
+// -1 if none does.
+int multi_variant(uint32_t fast_bytes, uint32_t sbuf_bytes) {
+    for (int i = 0; i < 5; ++i)
+        if (g_multi[i].smem(fast_bytes, sbuf_bytes) <= 227u * 1024u) return i;
+    return -1;
 }
 
 template <int NT>
@@ -751,7 +1183,10 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     return launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, info->n_groups, s, sms);
 }
 
-dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, cudaStream_t s, int sms) {
+// launches: if not null, receives the number of launches; dry: count them,
+// launch nothing (no GPU call is made).
+dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_t *d_out, cudaStream_t s, int sms,
+                                   int *launches, bool dry) {
     // every scope is checked before the first launch
     for (int i = 0; i < k; ++i) {
         const dfw_lanes_scope &sc = scopes[i];
@@ -764,27 +1199,116 @@ dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_
         st = lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);
         if (st != DFW_OK) return st;
     }
-    bool prior = false;  // a decode into d_out is already on the stream from this call
+    int dev = 0;
+    if (!dry && (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16)) return DFW_ECUDA;
+    if (launches) *launches = 0;
+    // One launch per run of consecutive scopes (at most SEQ_MAX_SCOPES) that
+    // the same CTA shape serves: a scope whose table or group spans would
+    // need a smaller CTA than the run so far starts a new run.
+    SeqParams P;
+    std::memset(&P, 0, sizeof(P));
+    uint32_t groups_max = 0, fast_bytes = 0, sbuf = 16;
+    int run_var = -1;
+    bool prior = false;  // a launch into d_out is already on the stream from this call
+    auto flush = [&]() -> dfw_status {
+        if (P.k == 0) return DFW_OK;
+        if (launches) ++*launches;
+        if (dry) {
+            std::memset(&P, 0, sizeof(P));
+            groups_max = 0;
+            fast_bytes = 0;
+            sbuf = 16;
+            run_var = -1;
+            return DFW_OK;
+        }
+        const int vi = run_var < 0 ? 0 : run_var;
+        MultiVariant &v = g_multi[vi];
+        const uint32_t smem = v.smem(fast_bytes, sbuf);
+        if (!v.smem_set[dev]) {
+            if (cudaFuncSetAttribute(v.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+                return DFW_ECUDA;
+            v.smem_set[dev] = 1;
+        }
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, v.fn, v.nt, smem) != cudaSuccess) return DFW_ECUDA;
+        if (per_sm < 1) return DFW_EINVAL;
+        const uint64_t wpc = (uint64_t)v.nt / 32, warps = (uint64_t)per_sm * sms * wpc;
+        const uint64_t want = groups_max < warps ? groups_max : warps;
+        P.out = d_out;
+        P.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
+        P.wait_prior = prior ? 1u : 0u;
+        P.sbuf_bytes = sbuf;
+        P.fast_bytes = fast_bytes;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((want + wpc - 1) / wpc));
+        cfg.blockDim = dim3((unsigned)v.nt);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = prior ? 1 : 0;
+        if (cudaLaunchKernelEx(&cfg, v.fn, P) != cudaSuccess) return DFW_ECUDA;
+        prior = true;
+        std::memset(&P, 0, sizeof(P));
+        groups_max = 0;
+        fast_bytes = 0;
+        sbuf = 16;
+        run_var = -1;
+        return DFW_OK;
+    };
     for (int i = 0; i < k; ++i) {
         const dfw_lanes_scope &sc = scopes[i];
         const uint64_t n = sc.table->n;
         if (n == 0) continue;
-        if (sc.table->total_bits == 0) {  // one exponent: an ordinary launch, after the previous one
-            const uint64_t want = ((n >> 3) + 256) / 256, cap = (uint64_t)sms * 8;
-            fill_single<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(sc.d_mant, sc.table->single_symbol, n, d_out);
-            if (cudaGetLastError() != cudaSuccess) return DFW_ECUDA;
+        SeqScope q;
+        std::memset(&q, 0, sizeof(q));
+        const uint64_t n_chunks = (n + LANE_SYMS - 1) / LANE_SYMS;
+        const uint64_t n_groups = (n_chunks + GROUP_CHUNKS - 1) / GROUP_CHUNKS;
+        if (n_chunks >= (1ull << 32)) return DFW_EINVAL;
+        q.mant = sc.d_mant;
+        q.mant_bytes = (n + 15) & ~15ull;
+        q.n_chunks = (uint32_t)n_chunks;
+        q.n_groups = (uint32_t)n_groups;
+        q.last_t = (uint32_t)(n - LANE_SYMS * (n_chunks - 1));
+        uint32_t fb_bytes = 0, sb = 16;
+        if (sc.table->total_bits == 0) {  // one distinct exponent: a fill
+            q.fast_bits = 0;
+            q.n_tables = sc.table->single_symbol;
         } else {
             LanesParams prm;
             lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);
-            prm.out = d_out;
-            prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
-            prm.wait_prior = prior ? 1u : 0u;
-            const dfw_status st = launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, sc.info->n_groups, s, sms, prior);
+            q.stream = prm.stream;
+            q.lut = prm.lut;
+            q.chunk_bits = prm.chunk_bits;
+            q.group_start = prm.group_start;
+            q.stream_bytes = prm.stream_bytes;
+            q.fast_bits = prm.fast_bits;
+            q.n_tables = prm.n_tables;
+            fb_bytes = 8u << prm.fast_bits;
+            sb = prm.sbuf_bytes;
+        }
+        const uint32_t nf = fast_bytes > fb_bytes ? fast_bytes : fb_bytes, ns = sbuf > sb ? sbuf : sb;
+        const bool fill = q.fast_bits == 0u;  // needs no table or slot: joins any run
+        const int alone = fill && P.k > 0 ? run_var : multi_variant(fb_bytes, sb), joined = multi_variant(nf, ns);
+        if (alone < 0) return DFW_EINVAL;  // even the smallest CTA does not fit
+        if (P.k > 0 && (P.k == SEQ_MAX_SCOPES || joined != run_var || alone != run_var)) {
+            const dfw_status st = flush();
             if (st != DFW_OK) return st;
         }
-        prior = true;
+        if (P.k == 0) {
+            run_var = alone;
+            fast_bytes = fb_bytes;
+            sbuf = sb;
+        } else {
+            fast_bytes = nf;
+            sbuf = ns;
+        }
+        P.sc[P.k++] = q;
+        if (q.n_groups > groups_max) groups_max = q.n_groups;
     }
-    return DFW_OK;
+    return flush();
 }
 
 dfw_status launch_gemv_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,

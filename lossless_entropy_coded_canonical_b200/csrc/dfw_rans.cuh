@@ -90,6 +90,9 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
         uint32_t bytes = 0;
         if (b1 > b0 && b1 <= prm.stream_bytes && !(b0 & 15u)) bytes = (uint32_t)min(b1 - b0, (uint64_t)prm.slot_bytes);
         bytes &= ~15u;
+        if (!check(bb < prm.n_blocks && bytes <= prm.slot_bytes && (bytes == 0u || b0 + bytes <= prm.stream_bytes),
+                   CK_RANS_COPY))
+            bytes = 0u;
         fence_proxy_async();
         mbar_expect_tx(bar0 + 8u * s, bytes);
         if (bytes) bulk_load(smem_u32(slots + s * prm.slot_bytes), prm.stream + b0, bytes, bar0 + 8u * s);
@@ -167,7 +170,8 @@ __global__ void __launch_bounds__(NT) rans_decode_kernel(const RansParams prm) {
                         // raw byte doubled into both halves keeps its sign at
                         // bit 15 and its mantissa at bits 6..0; the table
                         // entry's low byte is the exponent
-                        if (live) op[32u * t] = (uint16_t)(((mb * 0x101u) & 0x807Fu) | ((e << 7) & 0x7F80u));
+                        if (live && check(i0 + 128u * q + 32u * t + lane < prm.n, CK_RANS_STORE))
+                            op[32u * t] = (uint16_t)(((mb * 0x101u) & 0x807Fu) | ((e << 7) & 0x7F80u));
                     }
                     op += 128;
                 }

@@ -1,5 +1,6 @@
 """dfw_decode_lanes_seq: several scopes decoded one after another into one
-output buffer, each launch a programmatic dependent of the previous one.
+output buffer by one persistent launch per run of scopes (runs chained as
+programmatic dependents).
 
 The result must be exactly that of dfw_decode_lanes called on each scope in
 order (same bytes everywhere in the buffer, including what earlier, larger
@@ -156,3 +157,76 @@ def test_seq_replays_from_a_cuda_graph(scopes):
         dfw.check()
         assert torch.equal(out.view(torch.int16), want.view(torch.int16))
     del g
+
+
+def test_seq_longer_than_one_launch(oracle, scopes):
+    """More scopes than one persistent launch serves (40): the call chains
+    launches, each holding its stores until the previous has completed; the
+    buffer must still end as the calls in order leave it."""
+    us, devs = scopes
+    order = [i % len(devs) for i in range(2 * 40 + 3)]
+    seq = [devs[i] for i in order]
+    assert dfw.decode_lanes_seq_launches(seq) >= 3
+    nmax = max(u.size for u in us)
+    got, want = _garbage(nmax), _garbage(nmax)
+    dfw.decode_lanes_seq(seq, got)
+    for d in seq:
+        dfw.decode_lanes(d, want)
+    dfw.check()
+    assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+def test_seq_corrupt_scope_in_the_middle(scopes):
+    """A scope whose plan or fast table is corrupt writes nothing and is
+    reported; the scopes around it decode as the calls in order would."""
+    us, devs = scopes
+    nmax = max(u.size for u in us)
+    big, small = devs[1], devs[0]  # the corrupt one is the largest, so its region is visible at the end
+    for what in ("chunk_bits", "lut"):
+        bad = dfw.DeviceLanes(big.stream, big.mant, big.lut.clone(), big.chunk_bits.clone(), big.group_start,
+                              big.table, big.info)
+        if what == "chunk_bits":
+            bad.chunk_bits[40] += 3
+        else:
+            bad.lut[9] = 0
+        seq = [small, bad, small]
+        got, want = _garbage(nmax), _garbage(nmax)
+        dfw.decode_lanes_seq(seq, got)
+        assert dfw.check_status() == dfw.ECORRUPT, what
+        for d in seq:
+            dfw.decode_lanes(d, want)
+        assert dfw.check_status() == dfw.ECORRUPT, what
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), what
+    # the context decodes correctly afterwards
+    out = _garbage(nmax)
+    dfw.decode_lanes_seq(devs, out)
+    dfw.check()
+
+
+@pytest.mark.parametrize("offset", [8, 16])
+def test_seq_output_alignment(scopes, offset):
+    """A 16-byte (not 32-byte) aligned output takes two 128-bit stores per 16
+    weights; the bytes around the output stay untouched."""
+    us, devs = scopes
+    nmax = max(u.size for u in us)
+    want = _garbage(nmax)
+    for d in devs:
+        dfw.decode_lanes(d, want)
+    dfw.check()
+    buf = torch.zeros(nmax + 64, dtype=torch.int16, device="cuda")
+    out = buf[offset: offset + nmax].view(torch.bfloat16)
+    out.view(torch.int16).fill_(0x5A5A)
+    dfw.decode_lanes_seq(devs, out)
+    dfw.check()
+    assert torch.equal(out.view(torch.int16), want.view(torch.int16))
+    assert not buf[:offset].any() and not buf[offset + nmax:].any()
+
+
+def test_seq_one_scope_equals_single_decode(oracle, scopes):
+    """Each scope alone through the sequence kernel equals the oracle's decode."""
+    us, devs = scopes
+    for u, d in zip(us, devs):
+        out = _garbage(u.size)
+        dfw.decode_lanes_seq([d], out)
+        dfw.check()
+        assert np.array_equal(workloads.as_u16_numpy(out), oracle.decode(oracle.encode(u)))
