@@ -1,0 +1,87 @@
+"""The benchmark's measurement policy, on the CPU: when L2 is flushed between
+timed steps and what the line says about it, the host record beside the
+oracle baseline, the oracle's samples, and the reference arm's step count."""
+import json
+import os
+import subprocess
+import sys
+
+import numpy as np
+import torch
+
+import bench
+import workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_l2_guard_flushes_only_below_eight_times_l2():
+    l2 = 126 << 20
+    small = bench.L2Guard("cpu", 683_000_000)  # a Llama-2 block's step: 5.4x the L2
+    big = bench.L2Guard("cpu", 26_974_239_280)  # the 8B-shaped model's step
+    assert small.l2 == l2 and big.l2 == l2  # no CUDA device here: the B200's L2 size
+    assert small.flushing and small.buf.numel() == 4 * l2
+    assert not big.flushing and big.buf is None
+    assert "flushed" in small.label("x") and "683 MB" in small.label("x")
+    assert "larger than L2" in big.label("x") and "26974 MB" in big.label("x")
+    assert bench.L2Guard("cpu", 8 * l2).flushing is False
+    assert bench.L2Guard("cpu", 8 * l2 - 1).flushing is True
+
+
+def test_timed_steps_calls_the_step_exactly_k_times():
+    calls = []
+
+    class _Ev:
+        def __init__(self, **_):
+            pass
+
+        def record(self, *_):
+            pass
+
+        def elapsed_time(self, other):
+            return 1.0
+
+    real = torch.cuda.Event, torch.cuda.synchronize
+    torch.cuda.Event, torch.cuda.synchronize = _Ev, (lambda *a: None)
+    try:
+        guard = bench.L2Guard("cpu", 1000)
+        flushes = []
+        guard.flush = lambda stream=None: flushes.append(1)
+        assert bench.timed_steps(lambda: calls.append(1), 7, None, guard) == 7.0  # one pair of events per step
+        assert len(calls) == 7 and len(flushes) == 7
+        calls.clear()
+        assert bench.timed_steps(lambda: calls.append(1), 5, None, None) == 1.0  # one pair around all steps
+        assert len(calls) == 5
+    finally:
+        torch.cuda.Event, torch.cuda.synchronize = real
+
+
+def test_host_cpu_record():
+    h = bench.host_cpu()
+    assert h["nproc"] >= 1 and h["logical_cpus"] >= h["nproc"] and isinstance(h["model"], str)
+
+
+def test_cpu_sample_follows_the_recipe():
+    # a Llama-3 block: the first 5 M weights are all of q (4096 x 4096 = 16.8 M)
+    blk = workloads.c5()[1]
+    u = bench.cpu_sample(blk, 5_000_000)
+    assert u.dtype == np.uint16 and u.size == 5_000_000
+    # the sampled scope of the 34-scope model is its first transformer block
+    assert bench._sample_scope(workloads.c5()).name == "layer0"
+    assert bench._sample_scope([workloads.c1()]).name == "c1"
+    # size-dependent bit-pattern tensors (their exponent counts depend on n) are
+    # drawn whole with the recipe's size, then cut: the sample is a prefix of that draw
+    blk4 = workloads.c4("b", 1 << 20)
+    v = bench.cpu_sample(blk4, 1 << 19)
+    whole = workloads.as_u16_numpy(workloads.generate(blk4.tensors[0], "cpu"))
+    assert v.size == 1 << 19 and np.array_equal(v, whole[: 1 << 19])
+
+
+def test_reference_arm_runs_exactly_the_steps_asked():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "c1",
+                          "--steps", "4", "--warmup", "3"], capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads(out.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["steps"] == 4 and line["warmup"] == 3
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] == line["e2e"]["value"]
