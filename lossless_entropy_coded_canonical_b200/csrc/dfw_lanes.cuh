@@ -241,7 +241,9 @@ __device__ __forceinline__ uint32_t decode_chunk(uint32_t sw, uint32_t r, int le
         uint32_t ends = (ey >> FAST_ENDS_SHIFT) & 0xFFFu;
         const uint32_t c8 = (ey >> FAST_C8_SHIFT) & 255u;
         const uint32_t keep = (c8 - (uint32_t)(-left8)) >> 3;  // >= 1
-        for (uint32_t i = 1; i < keep; ++i) ends &= ends - 1u;
+#pragma unroll
+        for (uint32_t i = 1; i < FAST_MAX_SYMS; ++i)  // keep <= FAST_MAX_SYMS: predicated, no branch
+            if (i < keep) ends &= ends - 1u;
         end = end - (ey & 255u) + (uint32_t)__ffs(ends);
     }
     return end;
@@ -877,17 +879,17 @@ __global__ void __launch_bounds__(NT, 1) decode_lanes_multi(const SeqParams P) {
             if (ok) bulk_load(smem_u32(mbuf), j_mant + m0, bytes, bar_m);
         };
 
+        if (kc == 0u && jc == j && lane == 0) {  // the warp's first group: its starts and copies
+            sts64(stash(0, 0), a0);
+            sts64(stash(0, 1), a1);
+            issue_next_stream(jc, gc, 0, a0, a1);
+            issue_next_mant(jc, gc);
+        }
         while (jc == j) {  // this warp's groups of scope j
             const uint32_t s = kc & 1u;
             const uint8_t *slot = wslots + s * slot_bytes;
             const bool has_next = jn < P.k;
             __syncwarp();  // every lane is done with the other slot and with stash pair s ^ 1
-            if (kc == 0u && lane == 0) {  // the warp's first group: its starts and copies
-                sts64(stash(0, 0), a0);
-                sts64(stash(0, 1), a1);
-                issue_next_stream(jc, gc, 0, a0, a1);
-                issue_next_mant(jc, gc);
-            }
             if (has_next && lane == 0) {
                 sts64(stash(s ^ 1u, 0), ms0);
                 sts64(stash(s ^ 1u, 1), ms1);
