@@ -994,7 +994,8 @@ def main(argv=None):
     peak, peak_kind = measured_peak_hbm()
     if lanes:
         seq_launches = dfw.decode_lanes_seq_launches(devs)
-        kernel = "decode_lanes_multi"
+        # a sequence of one scope runs the one-scope kernel
+        kernel = "decode_lanes_multi" if len(devs) > 1 else "decode_lanes"
         achieved = alg_bytes / (ms_step * 1e-3) / 1e9
         launches_per_step = seq_launches
         mean_kernel_ms = ms_step / seq_launches

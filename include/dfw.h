@@ -386,10 +386,12 @@ typedef struct dfw_lanes_scope {
  * result is exactly that of k dfw_decode_lanes calls in order on cuda_stream:
  * every byte of d_out ends as the last scope covering it wrote it.  What
  * differs is scheduling: one persistent launch serves up to
- * DFW_SEQ_MAX_SCOPES consecutive scopes.  Its warps keep the same 2048-weight
- * output groups in every scope (group g of any scope is written by the same
- * threads), so a later scope's writes follow an earlier one's in each
- * thread's program order and no grid-wide barrier separates the scopes; each
+ * DFW_SEQ_MAX_SCOPES consecutive scopes (a run of a single scope uses
+ * dfw_decode_lanes' kernel, which has no scope bookkeeping).  Its warps keep
+ * the same 2048-weight output groups in every scope (group g of any scope is
+ * written by the same threads), so a later scope's writes follow an earlier
+ * one's in each thread's program order and no grid-wide barrier separates the
+ * scopes; each
  * CTA switches fast tables between scopes, while its copies for the next
  * scope's first groups are already in flight.  A new launch starts when the
  * run limit is reached or a scope needs a smaller CTA (long codewords need

@@ -1212,10 +1212,30 @@ dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_
     uint32_t groups_max = 0, fast_bytes = 0, sbuf = 16;
     int run_var = -1;
     bool prior = false;  // a launch into d_out is already on the stream from this call
+    int solo = -1;  // the scope index of a run's only scope
     auto flush = [&]() -> dfw_status {
         if (P.k == 0) return DFW_OK;
         if (launches) ++*launches;
         if (dry) {
+            std::memset(&P, 0, sizeof(P));
+            groups_max = 0;
+            fast_bytes = 0;
+            sbuf = 16;
+            run_var = -1;
+            return DFW_OK;
+        }
+        if (P.k == 1 && P.sc[0].fast_bits != 0u) {
+            // a run of one scope with a table: the one-scope kernel, which has
+            // no scope bookkeeping (same output, same ordering after a prior launch)
+            const dfw_lanes_scope &sc = scopes[solo];
+            LanesParams prm;
+            lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);
+            prm.out = d_out;
+            prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
+            prm.wait_prior = prior ? 1u : 0u;
+            const dfw_status st = launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, sc.info->n_groups, s, sms, prior);
+            if (st != DFW_OK) return st;
+            prior = true;
             std::memset(&P, 0, sizeof(P));
             groups_max = 0;
             fast_bytes = 0;
@@ -1307,6 +1327,7 @@ dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_
             fast_bytes = nf;
             sbuf = ns;
         }
+        if (P.k == 0) solo = i;
         P.sc[P.k++] = q;
         if (q.n_groups > groups_max) groups_max = q.n_groups;
     }

@@ -230,3 +230,29 @@ def test_seq_one_scope_equals_single_decode(oracle, scopes):
         dfw.decode_lanes_seq([d], out)
         dfw.check()
         assert np.array_equal(workloads.as_u16_numpy(out), oracle.decode(oracle.encode(u)))
+
+
+def test_seq_tiny_and_ragged_scopes(oracle):
+    """Scopes smaller than one group (most warps own no group in them), sizes
+    around the chunk and group edges, and a one-exponent scope among them: the
+    buffer ends as the calls in order leave it, and every scope alone through
+    the sequence kernel equals the oracle's decode."""
+    rng = np.random.default_rng(11)
+    sizes = [1, 63, 64, 65, 2047, 2048, 2049, 70_001]
+    us = [_u16(workloads.BlockSpec("t", [workloads.TensorSpec("w", n, "normal", 500 + n, 0.02)])) for n in sizes]
+    assert [u.size for u in us] == sizes
+    us.insert(4, ((rng.integers(0, 2, 3000) << 15) | (118 << 7) | rng.integers(0, 128, 3000)).astype(np.uint16))
+    devs = [_device(u) for u in us]
+    nmax = max(u.size for u in us)
+    for order in (list(range(len(us))), list(range(len(us)))[::-1]):
+        got, want = _garbage(nmax), _garbage(nmax)
+        dfw.decode_lanes_seq([devs[i] for i in order], got)
+        for i in order:
+            dfw.decode_lanes(devs[i], want)
+        dfw.check()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), order
+    for u, d in zip(us, devs):
+        out = _garbage(u.size)
+        dfw.decode_lanes_seq([d], out)
+        dfw.check()
+        assert np.array_equal(workloads.as_u16_numpy(out), oracle.decode(oracle.encode(u)))
