@@ -52,6 +52,18 @@ KERNEL_SOURCES = {
 
 # ------------------------------------------------------------------ helpers
 
+CAP = 32  # code length cap of every encoding this run makes (--cap)
+
+
+def reseed(blocks, offset: int):
+    """The same workload with every tensor's recipe seed moved by offset
+    (offset 0 leaves the workload's own seeds)."""
+    if not offset:
+        return blocks
+    return [workloads.BlockSpec(b.name, [workloads.TensorSpec(t.name, t.numel, t.kind, t.seed + offset, t.std,
+                                                              t.zero_frac) for t in b.tensors]) for b in blocks]
+
+
 def workload_blocks(name: str):
     if name == "c5":
         return workloads.c5(), "llama3-8b-shaped model: embed + 32 blocks + lm_head, 34 code tables, N(0,0.02)"
@@ -187,7 +199,7 @@ def prepare(blocks, device, window, tile, threads, variant="window"):
     pool = cf.ThreadPoolExecutor(max_workers=min(8, host_threads))
 
     def host_side(i, tensors):
-        enc = dfw.encode_multi(tensors, 32, n_threads=enc_threads, pin=True)
+        enc = dfw.encode_multi(tensors, CAP, n_threads=enc_threads, pin=True)
         pl = dfw.plan_lanes(enc, pin=True) if variant == "lanes" else dfw.plan(enc, window, tile, pin=True)
         return i, enc, pl
 
@@ -218,7 +230,7 @@ def prepare_on_device(blocks, device):
         sizes = [t.numel() for t in ts]
         x = torch.cat([t.reshape(-1) for t in ts]) if len(ts) > 1 else ts[0].reshape(-1)
         del ts
-        dl = dfw.encode_device(x, 32, scratch=scratch)
+        dl = dfw.encode_device(x, CAP, scratch=scratch)
         del x
         offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.uint64)
         dl.tensor_offsets = offs
@@ -577,7 +589,7 @@ def run_encode_mode(args, rank, world, blocks, wdesc, device):
     torch.cuda.empty_cache()
 
     def encode_scope(sc):
-        dfw._check(lib.dfw_encode_device(sc["x"].data_ptr(), sc["n"], 32, sc["mant"].data_ptr(), sc["cb"].data_ptr(),
+        dfw._check(lib.dfw_encode_device(sc["x"].data_ptr(), sc["n"], CAP, sc["mant"].data_ptr(), sc["cb"].data_ptr(),
                                          sc["gs"].data_ptr(), scratch.data_ptr(), scratch.numel(),
                                          ctypes.byref(sc["table"]), ctypes.byref(sc["info"]), sh), "dfw_encode_device")
         if sc["stream"] is None:  # sized by the first (warm-up) encode; the data do not change
@@ -600,7 +612,7 @@ def run_encode_mode(args, rank, world, blocks, wdesc, device):
             for sc in scopes:
                 encode_scope(sc)
             return
-        dfw._check(lib.dfw_encode_device_multi(k, arr, 32, mscratch.data_ptr(), mscratch.numel(), staging.data_ptr(),
+        dfw._check(lib.dfw_encode_device_multi(k, arr, CAP, mscratch.data_ptr(), mscratch.numel(), staging.data_ptr(),
                                                staging.numel(), tables, infos, sh), "dfw_encode_device_multi")
         for i, sc in enumerate(scopes):
             sc["table"], sc["info"] = tables[i], infos[i]
@@ -909,6 +921,9 @@ def main(argv=None):
     ap.add_argument("--variant", default="lanes", choices=["window", "lanes"],
                     help="window: gap/out_start plan (count phase + scan); lanes: known-start chunks")
     ap.add_argument("--threads", type=int, default=0)
+    ap.add_argument("--cap", type=int, default=32, help="code length cap of the encoding, 1..32")
+    ap.add_argument("--seed", type=int, default=0,
+                    help="offset added to every tensor's recipe seed (0: the workload's own seeds)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--cpu-sample", type=int, default=32 * 1024 * 1024)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -930,7 +945,14 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not 1 <= args.cap <= 32:
+        ap.error("--cap must be in 1..32")
+    global CAP
+    CAP = args.cap
     blocks, wdesc = workload_blocks(args.workload)
+    blocks = reseed(blocks, args.seed)
+    if args.cap != 32 or args.seed:
+        wdesc += f", cap {args.cap}, seed offset {args.seed}"
     n_total = sum(b.numel for b in blocks)
 
     if args.impl == "reference":
@@ -1040,6 +1062,7 @@ def main(argv=None):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8", "data": "synthetic",
         "config": {"workload": wdesc, "weights": n_total, "code_tables": len(devs), "plan": args.variant,
+                   "cap": CAP, "seed_offset": args.seed,
                    "window_bytes": args.window if args.variant == "window" else None,
                    "tile_windows": args.tile if args.variant == "window" else None,
                    "l2": guard.label("every scope's compressed form read, its bf16 written"),

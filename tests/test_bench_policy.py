@@ -85,3 +85,14 @@ def test_reference_arm_runs_exactly_the_steps_asked():
     assert line["impl"] == "reference" and line["steps"] == 4 and line["warmup"] == 3
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] == line["e2e"]["value"]
+
+
+def test_seed_offset_and_cap_flags():
+    blocks = workloads.c5()[:2]
+    moved = bench.reseed(blocks, 7)
+    assert [t.seed for b in moved for t in b.tensors] == [t.seed + 7 for b in blocks for t in b.tensors]
+    assert [t.numel for b in moved for t in b.tensors] == [t.numel for b in blocks for t in b.tensors]
+    assert bench.reseed(blocks, 0) is blocks
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--cap", "0"], capture_output=True,
+                         text=True, timeout=300, cwd=ROOT)
+    assert out.returncode == 2 and "--cap" in out.stderr
