@@ -256,3 +256,25 @@ def test_seq_tiny_and_ragged_scopes(oracle):
         dfw.decode_lanes_seq([d], out)
         dfw.check()
         assert np.array_equal(workloads.as_u16_numpy(out), oracle.decode(oracle.encode(u)))
+
+
+def test_seq_alternating_scopes_end_with_the_last(scopes):
+    """Forty scopes in one launch, two contents of nearly the same size taking
+    turns over the same bytes: a store of any scope that landed after the
+    next scope's store of the same group would leave the wrong content."""
+    us, devs = scopes
+    a, b = devs[0], devs[1]  # 1.5 M and 2.0 M weights: ragged per-CTA group counts
+    want_a, want_b = _garbage(max(a.n, b.n)), _garbage(max(a.n, b.n))
+    for d in (b, a):
+        dfw.decode_lanes(d, want_a)
+    for d in (a, b):
+        dfw.decode_lanes(d, want_b)
+    dfw.check()
+    for last, want in ((b, want_b), (a, want_a)):
+        order = [a, b] * 20 if last is b else [b, a] * 20
+        assert dfw.decode_lanes_seq_launches(order) == 1
+        for _ in range(3):
+            got = _garbage(max(a.n, b.n))
+            dfw.decode_lanes_seq(order, got)
+            dfw.check()
+            assert torch.equal(got.view(torch.int16), want.view(torch.int16))
