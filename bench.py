@@ -324,21 +324,24 @@ class L2Guard:
                 f"CUDA events): a step moves only {mb:.0f} MB ({what}) against the {self.l2 >> 20} MB L2")
 
 
-def timed_steps(fn, steps: int, stream, guard: L2Guard | None = None) -> float:
-    """Device time of ``steps`` calls of fn on ``stream`` (ms, total): one
-    pair of CUDA events around all of them, or, when the guard flushes L2,
-    a pair around each call with the flush in between."""
+def timed_steps(fn, steps: int, stream, guard: L2Guard | None = None, per_step: list | None = None) -> float:
+    """Device time of ``steps`` calls of fn on ``stream`` (ms, total): CUDA
+    events between consecutive calls (the total spans all of them), or, when
+    the guard flushes L2, a pair around each call with the flush in between.
+    ``per_step``, if a list, receives each call's own time (ms)."""
     barrier()
     torch.cuda.synchronize()
     if guard is None or not guard.flushing:
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(steps):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        ev[0].record(stream)
+        for i in range(steps):
             fn()
-        t1.record(stream)
+            ev[i + 1].record(stream)
         torch.cuda.synchronize()
         barrier()
-        return t0.elapsed_time(t1)
+        if per_step is not None:
+            per_step.extend(ev[i].elapsed_time(ev[i + 1]) for i in range(steps))
+        return ev[0].elapsed_time(ev[-1])
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in ev:
         guard.flush(stream)
@@ -347,7 +350,17 @@ def timed_steps(fn, steps: int, stream, guard: L2Guard | None = None) -> float:
         b.record(stream)
     torch.cuda.synchronize()
     barrier()
+    if per_step is not None:
+        per_step.extend(a.elapsed_time(b) for a, b in ev)
     return sum(a.elapsed_time(b) for a, b in ev)
+
+
+def step_stats(per_step: list) -> dict | None:
+    """Median, best and worst of the timed steps (ms, this rank's own)."""
+    if not per_step:
+        return None
+    a = np.array(per_step, dtype=np.float64)
+    return {"median": float(np.median(a)), "best": float(a.min()), "worst": float(a.max()), "steps": int(a.size)}
 
 
 # ------------------------------------------------------------------ timed arms
@@ -380,7 +393,8 @@ def run_device(devs, scratch, steps, warmup, stream, guard: L2Guard | None = Non
     return total_ms, per_launch, status
 
 
-def run_device_seq(devs, scratch, steps, warmup, stream, graph=False, guard: L2Guard | None = None):
+def run_device_seq(devs, scratch, steps, warmup, stream, graph=False, guard: L2Guard | None = None,
+                   per_step: list | None = None):
     """The step as one dfw_decode_lanes_seq call over every scope: the same
     launches in the same order into the same scratch buffer, each one a
     programmatic dependent of the one before (it may start while the previous
@@ -405,7 +419,7 @@ def run_device_seq(devs, scratch, steps, warmup, stream, graph=False, guard: L2G
         else:
             dfw.decode_lanes_seq(devs, scratch, stream=stream)
 
-    total = timed_steps(step, steps, stream, guard)
+    total = timed_steps(step, steps, stream, guard, per_step)
     del g
     return total, dfw.check_status(stream)
 
@@ -990,9 +1004,11 @@ def main(argv=None):
     lanes = args.variant == "lanes"
     guard = L2Guard(device, alg_bytes)
     sampler = ClockSampler(local)
+    per_step = []
     sampler.start()
     if lanes:  # the step: one sequence of launches over every scope
-        total_ms, status = run_device_seq(devs, scratch, args.steps, args.warmup, stream, args.graph, guard)
+        total_ms, status = run_device_seq(devs, scratch, args.steps, args.warmup, stream, args.graph, guard,
+                                          per_step)
     else:
         total_ms, per_launch, status = run_device(devs, scratch, args.steps, args.warmup, stream, guard)
     clocks = sampler.stop()
@@ -1070,6 +1086,7 @@ def main(argv=None):
                    "launch": ("one dfw_decode_lanes_seq per step: one persistent launch per run of up to 40 "
                               "scopes" + (", captured once in a CUDA graph and replayed" if args.graph else "")
                               if lanes else "one dfw_decode_block per scope")},
+        "step_ms": step_stats(per_step),
         "effective_gbs": eff_gbs, "hbm_frac": eff_gbs / peak,
         "compression_ratio": 2 * n_total / comp, "compression_ratio_no_aux": 2 * n_total / comp_noaux,
         "bits_per_weight": 8 * comp / n_total,

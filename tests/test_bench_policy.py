@@ -50,10 +50,20 @@ def test_timed_steps_calls_the_step_exactly_k_times():
         assert bench.timed_steps(lambda: calls.append(1), 7, None, guard) == 7.0  # one pair of events per step
         assert len(calls) == 7 and len(flushes) == 7
         calls.clear()
-        assert bench.timed_steps(lambda: calls.append(1), 5, None, None) == 1.0  # one pair around all steps
-        assert len(calls) == 5
+        per = []
+        assert bench.timed_steps(lambda: calls.append(1), 5, None, None, per) == 1.0  # first to last event
+        assert len(calls) == 5 and per == [1.0] * 5  # an event between consecutive steps
+        per.clear()
+        calls.clear()
+        assert bench.timed_steps(lambda: calls.append(1), 3, None, guard, per) == 3.0 and per == [1.0] * 3
     finally:
         torch.cuda.Event, torch.cuda.synchronize = real
+
+
+def test_step_stats():
+    s = bench.step_stats([3.0, 1.0, 2.0, 5.0])
+    assert s == {"median": 2.5, "best": 1.0, "worst": 5.0, "steps": 4}
+    assert bench.step_stats([]) is None
 
 
 def test_host_cpu_record():
