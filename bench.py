@@ -67,6 +67,9 @@ def reseed(blocks, offset: int):
 def workload_blocks(name: str):
     if name == "c5":
         return workloads.c5(), "llama3-8b-shaped model: embed + 32 blocks + lm_head, 34 code tables, N(0,0.02)"
+    if name == "c4":  # the three edge-case tensors as one sequence (their own table each)
+        return ([workloads.c4("a"), workloads.c4("b"), workloads.c4("c")],
+                "c4: tensors 4a, 4b, 4c (3 x 67108864 weights), one code table each")
     table = {"c1": workloads.c1(), "c2": workloads.c2(), "c3": workloads.c3(), "c4a": workloads.c4("a"),
              "c4b": workloads.c4("b"), "c4bp": workloads.c4("bp"), "c4c": workloads.c4("c")}
     return [table[name]], f"{name} ({table[name].numel} weights)"
