@@ -304,7 +304,11 @@ dfw_status dfw_plan_lanes(const uint8_t *stream, const dfw_table *table, uint16_
  * n must be below 2^38 (chunk indices are 32-bit; DFW_EINVAL otherwise).
  * Errors as dfw_decode; a group whose chunk bits disagree with
  * group_start, or whose codewords do not end where chunk_bits says, writes
- * nothing / is flagged through dfw_check.
+ * nothing / is flagged through dfw_check.  Two closed forms of the code are
+ * read in place instead (the plan and LUT are still checked on the host,
+ * but not read on the device): two exponents with 1-bit codes (the stream
+ * is a bitmap) and all 256 exponents with 8-bit codes (stream byte i is
+ * exponent i); every stream is a valid code then, so nothing is flagged.
  */
 dfw_status dfw_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
                             const uint16_t *d_chunk_bits, const uint64_t *d_group_start,

@@ -593,6 +593,97 @@ __global__ void __launch_bounds__(NT) decode_lanes(const LanesParams prm, const 
     }
 }
 
+// ------------------------------------------------------------ closed forms
+//
+// Two shapes of the canonical code decode without a table walk: two symbols
+// with 1-bit codes (the stream is a bitmap, code 0 being the smaller symbol)
+// and all 256 symbols with 8-bit codes (ordered by symbol, code s is symbol
+// s: stream byte i is exponent i).  With every codeword L bits long, weight
+// w's code starts at bit L w, so the 16 weights from a multiple of 16 have
+// their codes in 2 L whole bytes; no plan is needed to find them.
+constexpr uint32_t CLOSED_NONE = 0, CLOSED_BITMAP = 1, CLOSED_IDENTITY = 8;
+
+// Which closed form a (validated) table has; for a bitmap, syms gets the
+// symbols of codes 0 (bits 0..7) and 1 (bits 8..15).
+inline uint32_t closed_form(const dfw_table *t, uint32_t &syms) {
+    syms = 0;
+    if (t->total_bits == 0 || (t->n_symbols != 2u && t->n_symbols != 256u)) return CLOSED_NONE;
+    uint32_t k = 0, len = 0, s[2] = {0, 0};
+    for (uint32_t e = 0; e < 256u; ++e) {
+        if (!t->len[e]) continue;
+        if (len && t->len[e] != len) return CLOSED_NONE;
+        len = t->len[e];
+        if (k < 2u) s[k] = e;
+        ++k;
+    }
+    if (k == 2u && len == 1u) {
+        syms = s[0] | (s[1] << 8);
+        return CLOSED_BITMAP;
+    }
+    return k == 256u && len == 8u ? CLOSED_IDENTITY : CLOSED_NONE;
+}
+
+// Exponent bytes of four weights, each rotated as the joins take them.
+__device__ __forceinline__ uint32_t rot4(uint32_t x) { return ((x >> 1) & 0x7F7F7F7Fu) | ((x << 7) & 0x80808080u); }
+
+// The rotated exponents of the 16 weights from w (a multiple of 16 below the
+// scope's n), four to a word: R[q] holds weights w + 4 q .. w + 4 q + 3.
+// The stream holds at least ceil(L n / 8) + 16 bytes, so both reads stay in it.
+__device__ __forceinline__ void closed_exps(uint32_t mode, const uint8_t *stream, uint32_t syms, uint64_t w,
+                                            uint32_t (&R)[4]) {
+    if (mode == CLOSED_IDENTITY) {
+        const uint4 x = __ldcs(reinterpret_cast<const uint4 *>(stream + w));
+        R[0] = rot4(x.x);
+        R[1] = rot4(x.y);
+        R[2] = rot4(x.z);
+        R[3] = rot4(x.w);
+        return;
+    }
+    // bitmap: bytes w / 8 and w / 8 + 1, weight w + j at bit 7 - j of the
+    // first (MSB first); reversed, weight w + j is bit 24 + j, w + 8 + j bit 16 + j
+    const uint32_t v = __brev((uint32_t)__ldcs(reinterpret_cast<const unsigned short *>(stream + (w >> 3))));
+    const uint32_t e0 = rot_sym(syms & 0xFFu) * 0x01010101u, d = (rot_sym(syms >> 8) * 0x01010101u) ^ e0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t nib = (v >> (q < 2 ? 24 + 4 * q : 8 + 4 * q)) & 0xFu;  // weights w + 4 q .. + 3, bit j = w + 4 q + j
+        const uint32_t mask = ((nib * 0x00204081u) & 0x01010101u) * 0xFFu;  // bit j -> byte j all ones
+        R[q] = e0 ^ (d & mask);
+    }
+}
+
+// A scope in a closed form, one thread per 16 weights (raw bytes, codes and
+// output all whole 16- or 32-byte pieces).
+__global__ void __launch_bounds__(256) decode_closed(const uint8_t *__restrict__ stream,
+                                                     const uint8_t *__restrict__ mant, uint32_t mode, uint32_t syms,
+                                                     uint64_t n, uint16_t *__restrict__ out, uint32_t out32) {
+    const uint64_t pieces = (n + 15u) >> 4;
+    for (uint64_t p = (uint64_t)blockIdx.x * 256u + threadIdx.x; p < pieces; p += (uint64_t)gridDim.x * 256u) {
+        const uint64_t w = p << 4;
+        uint32_t R[4];
+        closed_exps(mode, stream, syms, w, R);
+        const uint4 m = __ldcs(reinterpret_cast<const uint4 *>(mant + w));  // raw bytes: a multiple of 16
+        uint4 r0, r1;
+        join4(R[0], m.x, r0.x, r0.y);
+        join4(R[1], m.y, r0.z, r0.w);
+        join4(R[2], m.z, r1.x, r1.y);
+        join4(R[3], m.w, r1.z, r1.w);
+        if (w + 16u <= n) {
+            if (out32) {
+                stg256_cs(out + w, r0, r1);
+            } else {
+                __stcs(reinterpret_cast<uint4 *>(out + w), r0);
+                __stcs(reinterpret_cast<uint4 *>(out + w + 8u), r1);
+            }
+        } else {  // the scope's last weights, one at a time
+            for (uint32_t q = 0; w + q < n; ++q) {
+                const uint32_t mq = q < 4u ? m.x : q < 8u ? m.y : q < 12u ? m.z : m.w;
+                const uint32_t rq = q < 4u ? R[0] : q < 8u ? R[1] : q < 12u ? R[2] : R[3];
+                out[w + q] = join1(rq >> (8u * (q & 3u)), (mq >> (8u * (q & 3u))) & 0xFFu);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------ many scopes, one launch
 //
 // A sequence of code-table scopes (a model's blocks) decoded by one
@@ -620,9 +711,9 @@ struct SeqScope {
     uint64_t stream_bytes, mant_bytes;
     uint32_t n_chunks, n_groups;  // n_groups == 0: an empty scope
     uint32_t last_t;              // codewords in the last chunk (1..64)
-    uint32_t fast_bits;           // 0: one distinct exponent (fill)
-    uint32_t n_tables;            // hierarchy tables, or the exponent of a one-exponent scope
-    uint32_t reserved;
+    uint32_t fast_bits;           // 0: no table (one distinct exponent, or a closed form)
+    uint32_t n_tables;            // hierarchy tables; the exponent of a one-exponent scope; a bitmap's symbols
+    uint32_t closed;              // with fast_bits 0: CLOSED_BITMAP or CLOSED_IDENTITY (the stream is read)
 };
 
 constexpr uint32_t SEQ_MAX_SCOPES = DFW_SEQ_MAX_SCOPES;
@@ -639,10 +730,11 @@ struct SeqParams {
 };
 static_assert(sizeof(SeqParams) <= 4096, "kernel parameters stay within the classic 4 KB limit");
 
-// One-exponent scope: the warp's groups filled from their raw bytes.
+// A scope without a table (one exponent, or a closed form): the warp's
+// groups built from their raw bytes and, for a closed form, their codes.
 __device__ __forceinline__ void fill_groups(const SeqScope &S, uint16_t *out, uint32_t out32, uint32_t slot0,
                                             uint32_t gstride, uint32_t lane) {
-    const uint32_t R = rot_sym(S.n_tables) * 0x01010101u;
+    const uint32_t C = rot_sym(S.n_tables) * 0x01010101u;
     const uint64_t n = (uint64_t)(S.n_chunks - 1u) * LANE_SYMS + S.last_t;
     for (uint32_t g = slot0; g < S.n_groups; g += gstride) {
         const uint64_t w0 = (uint64_t)g * GROUP_SYMS + 16u * lane;  // + 512 j
@@ -651,11 +743,17 @@ __device__ __forceinline__ void fill_groups(const SeqScope &S, uint16_t *out, ui
             if (w >= n) break;
             if (!check(w + 16u <= S.mant_bytes, CK_FILL_READ)) break;
             const uint4 m = __ldcs(reinterpret_cast<const uint4 *>(S.mant + w));  // w + 16 <= mant_bytes
+            uint32_t R[4] = {C, C, C, C};
+            if (S.closed) {
+                if (!check((S.closed == CLOSED_IDENTITY ? w + 16u : (w >> 3) + 2u) <= S.stream_bytes, CK_FILL_READ))
+                    break;
+                closed_exps(S.closed, S.stream, S.n_tables, w, R);
+            }
             uint4 r0, r1;
-            join4(R, m.x, r0.x, r0.y);
-            join4(R, m.y, r0.z, r0.w);
-            join4(R, m.z, r1.x, r1.y);
-            join4(R, m.w, r1.z, r1.w);
+            join4(R[0], m.x, r0.x, r0.y);
+            join4(R[1], m.y, r0.z, r0.w);
+            join4(R[2], m.z, r1.x, r1.y);
+            join4(R[3], m.w, r1.z, r1.w);
             if (w + 16u <= n) {
                 if (out32) {
                     stg256_cs(out + w, r0, r1);
@@ -666,7 +764,8 @@ __device__ __forceinline__ void fill_groups(const SeqScope &S, uint16_t *out, ui
             } else {  // the scope's last weights, one at a time
                 for (uint32_t q = 0; w + q < n; ++q) {
                     const uint32_t mq = q < 4u ? m.x : q < 8u ? m.y : q < 12u ? m.z : m.w;
-                    out[w + q] = join1(rot_sym(S.n_tables), (mq >> (8u * (q & 3u))) & 0xFFu);
+                    const uint32_t rq = q < 4u ? R[0] : q < 8u ? R[1] : q < 12u ? R[2] : R[3];
+                    out[w + q] = join1(rq >> (8u * (q & 3u)), (mq >> (8u * (q & 3u))) & 0xFFu);
                 }
             }
         }
@@ -1065,6 +1164,14 @@ dfw_status launch_lanes(const LanesParams &prm, const typename Epi::Params &ep, 
     return DFW_EINVAL;  // even the smallest CTA does not fit
 }
 
+// A scope in a closed form: decode_closed over its 16-weight pieces.
+dfw_status launch_closed(const LanesParams &prm, uint32_t mode, uint32_t syms, uint64_t n, cudaStream_t s, int sms) {
+    const uint64_t want = (((n + 15u) >> 4) + 255u) / 256u, cap = (uint64_t)sms * 8u;
+    decode_closed<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(prm.stream, prm.mant, mode, syms, n, prm.out,
+                                                                        prm.out32);
+    return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
+}
+
 // Checks a known-start plan against its table and fills the kernel
 // parameters (out left null).
 dfw_status lanes_params(const uint8_t *d_stream, const uint8_t *d_mant, const uint32_t *d_lut,
@@ -1182,6 +1289,8 @@ dfw_status launch_decode_lanes(const uint8_t *d_stream, const uint8_t *d_mant, c
     if (st != DFW_OK) return st;
     prm.out = d_out;
     prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
+    uint32_t syms = 0;
+    if (const uint32_t mode = closed_form(table, syms)) return launch_closed(prm, mode, syms, table->n, s, sms);
     return launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, info->n_groups, s, sms);
 }
 
@@ -1224,16 +1333,21 @@ dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_
             run_var = -1;
             return DFW_OK;
         }
-        if (P.k == 1 && P.sc[0].fast_bits != 0u) {
-            // a run of one scope with a table: the one-scope kernel, which has
-            // no scope bookkeeping (same output, same ordering after a prior launch)
+        if (P.k == 1 && (P.sc[0].fast_bits != 0u || P.sc[0].closed)) {
+            // a run of one scope with a table or in a closed form: the
+            // one-scope kernels, which have no scope bookkeeping (same output;
+            // after a prior launch the table kernel is its programmatic
+            // dependent and holds its stores, the closed-form kernel simply
+            // follows it on the stream)
             const dfw_lanes_scope &sc = scopes[solo];
             LanesParams prm;
             lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);
             prm.out = d_out;
             prm.out32 = (reinterpret_cast<uintptr_t>(d_out) & 31u) == 0u;
             prm.wait_prior = prior ? 1u : 0u;
-            const dfw_status st = launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, sc.info->n_groups, s, sms, prior);
+            const dfw_status st = P.sc[0].closed
+                                      ? launch_closed(prm, P.sc[0].closed, P.sc[0].n_tables, sc.table->n, s, sms)
+                                      : launch_lanes<StoreEpi>(prm, StoreEpi::Params{}, sc.info->n_groups, s, sms, prior);
             if (st != DFW_OK) return st;
             prior = true;
             std::memset(&P, 0, sizeof(P));
@@ -1294,10 +1408,16 @@ dfw_status launch_decode_lanes_seq(int k, const dfw_lanes_scope *scopes, uint16_
         q.n_chunks = (uint32_t)n_chunks;
         q.n_groups = (uint32_t)n_groups;
         q.last_t = (uint32_t)(n - LANE_SYMS * (n_chunks - 1));
-        uint32_t fb_bytes = 0, sb = 16;
+        uint32_t fb_bytes = 0, sb = 16, syms = 0;
         if (sc.table->total_bits == 0) {  // one distinct exponent: a fill
             q.fast_bits = 0;
             q.n_tables = sc.table->single_symbol;
+        } else if (const uint32_t mode = closed_form(sc.table, syms)) {  // codes read in place: no table
+            q.stream = sc.d_stream;
+            q.stream_bytes = sc.table->stream_bytes;
+            q.fast_bits = 0;
+            q.n_tables = syms;
+            q.closed = mode;
         } else {
             LanesParams prm;
             lanes_params(sc.d_stream, sc.d_mant, sc.d_lut, sc.d_chunk_bits, sc.d_group_start, sc.table, sc.info, prm);

@@ -66,6 +66,23 @@ def test_step_stats():
     assert bench.step_stats([]) is None
 
 
+def test_closed_form_labels():
+    import lossless_entropy_coded_canonical_b200 as dfw
+
+    class _D:
+        def __init__(self, lens, total_bits=1):
+            self.table = dfw.Table()
+            for s, v in lens.items():
+                self.table.len[s] = v
+            self.table.total_bits = total_bits
+
+    assert bench.scope_kernel(_D({126: 1, 127: 1})) == "decode_closed"
+    assert bench.scope_kernel(_D({s: 8 for s in range(256)})) == "decode_closed"
+    assert bench.scope_kernel(_D({s: 8 for s in range(254)} | {254: 9, 255: 9})) == "decode_lanes"
+    assert bench.scope_kernel(_D({1: 1, 2: 2, 3: 2})) == "decode_lanes"
+    assert bench.scope_kernel(_D({}, total_bits=0)) == "fill_single"
+
+
 def test_host_cpu_record():
     h = bench.host_cpu()
     assert h["nproc"] >= 1 and h["logical_cpus"] >= h["nproc"] and isinstance(h["model"], str)

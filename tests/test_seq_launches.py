@@ -25,11 +25,18 @@ def kinds():
                             workloads.generate_block(workloads.scaled(workloads.c5()[1], 70_000))])
     rng = np.random.default_rng(3)
     single = ((rng.integers(0, 2, 5000) << 15) | (119 << 7) | rng.integers(0, 128, 5000)).astype(np.uint16)
-    # incompressible bits: 8-bit codewords, 2 KB group spans, too big for the 1024-thread CTA
-    wide = workloads.as_u16_numpy(workloads.generate_block(workloads.c4("c", 70_000))[0])
+    # uniform 16-bit patterns: all 256 exponents with 8-bit codes, a closed
+    # form (codes read in place, no table); with exponent 0 folded into 1,
+    # 255 exponents and codes of 7 and 8 bits: 2 KB group spans, too big for
+    # the 1024-thread CTA
+    closed = workloads.as_u16_numpy(workloads.generate_block(workloads.c4("c", 70_000))[0])
+    wide = closed.copy()
+    e = (wide >> 7) & 0xFF
+    wide[e == 0] |= np.uint16(1 << 7)
     empty = _host_scope(np.zeros(0, np.uint16))
     empty.mant = torch.zeros(16, dtype=torch.uint8)  # a scope's raw-byte pointer may not be null, even when empty
-    return {"gauss": _host_scope(gauss), "single": _host_scope(single), "wide": _host_scope(wide), "empty": empty}
+    return {"gauss": _host_scope(gauss), "single": _host_scope(single), "wide": _host_scope(wide),
+            "closed": _host_scope(closed), "empty": empty}
 
 
 def test_model_sized_sequence_is_one_launch(kinds):
@@ -49,11 +56,17 @@ def test_runs_break_where_the_cta_shape_changes(kinds):
 
 
 def test_fills_and_empty_scopes_take_no_launch_of_their_own(kinds):
-    g, s, e, w = kinds["gauss"], kinds["single"], kinds["empty"], kinds["wide"]
+    g, s, e, w, c = kinds["gauss"], kinds["single"], kinds["empty"], kinds["wide"], kinds["closed"]
     assert dfw.decode_lanes_seq_launches([g, s, g, e, g]) == 1
     assert dfw.decode_lanes_seq_launches([w, s, w]) == 1
     assert dfw.decode_lanes_seq_launches([s]) == 1
     assert dfw.decode_lanes_seq_launches([e, e]) == 0
+    # a closed form needs no table or stream slot either
+    assert c.table.n_symbols == 256 and all(c.table.len[x] == 8 for x in range(256))
+    assert w.table.n_symbols == 255
+    assert dfw.decode_lanes_seq_launches([g, c, g, c, g]) == 1
+    assert dfw.decode_lanes_seq_launches([w, c, w]) == 1
+    assert dfw.decode_lanes_seq_launches([c]) == 1
 
 
 def test_bad_scope_is_refused(kinds):
