@@ -70,6 +70,7 @@ enum CheckSite : uint32_t {
     CK_ENC_SPLIT = 14,          // encoder pass 1 beyond its buffers
     CK_ENC_PACK_BUF = 15,       // encoder packing beyond its shared word buffer
     CK_ENC_PACK_STREAM = 16,    // encoder packing beyond the stream
+    CK_CLOSED_READ = 17,        // a closed-form decode read past the stream
 };
 
 // A named range on profiler timelines (NVTX) for the duration of a call;

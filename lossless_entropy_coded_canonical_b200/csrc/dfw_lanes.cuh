@@ -655,10 +655,12 @@ __device__ __forceinline__ void closed_exps(uint32_t mode, const uint8_t *stream
 // output all whole 16- or 32-byte pieces).
 __global__ void __launch_bounds__(256) decode_closed(const uint8_t *__restrict__ stream,
                                                      const uint8_t *__restrict__ mant, uint32_t mode, uint32_t syms,
-                                                     uint64_t n, uint16_t *__restrict__ out, uint32_t out32) {
+                                                     uint64_t n, uint64_t stream_bytes, uint16_t *__restrict__ out,
+                                                     uint32_t out32) {
     const uint64_t pieces = (n + 15u) >> 4;
     for (uint64_t p = (uint64_t)blockIdx.x * 256u + threadIdx.x; p < pieces; p += (uint64_t)gridDim.x * 256u) {
         const uint64_t w = p << 4;
+        if (!check((mode == CLOSED_IDENTITY ? w + 16u : (w >> 3) + 2u) <= stream_bytes, CK_CLOSED_READ)) break;
         uint32_t R[4];
         closed_exps(mode, stream, syms, w, R);
         const uint4 m = __ldcs(reinterpret_cast<const uint4 *>(mant + w));  // raw bytes: a multiple of 16
@@ -745,7 +747,7 @@ __device__ __forceinline__ void fill_groups(const SeqScope &S, uint16_t *out, ui
             const uint4 m = __ldcs(reinterpret_cast<const uint4 *>(S.mant + w));  // w + 16 <= mant_bytes
             uint32_t R[4] = {C, C, C, C};
             if (S.closed) {
-                if (!check((S.closed == CLOSED_IDENTITY ? w + 16u : (w >> 3) + 2u) <= S.stream_bytes, CK_FILL_READ))
+                if (!check((S.closed == CLOSED_IDENTITY ? w + 16u : (w >> 3) + 2u) <= S.stream_bytes, CK_CLOSED_READ))
                     break;
                 closed_exps(S.closed, S.stream, S.n_tables, w, R);
             }
@@ -1167,8 +1169,8 @@ dfw_status launch_lanes(const LanesParams &prm, const typename Epi::Params &ep, 
 // A scope in a closed form: decode_closed over its 16-weight pieces.
 dfw_status launch_closed(const LanesParams &prm, uint32_t mode, uint32_t syms, uint64_t n, cudaStream_t s, int sms) {
     const uint64_t want = (((n + 15u) >> 4) + 255u) / 256u, cap = (uint64_t)sms * 8u;
-    decode_closed<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(prm.stream, prm.mant, mode, syms, n, prm.out,
-                                                                        prm.out32);
+    decode_closed<<<(unsigned)(want < cap ? want : cap), 256, 0, s>>>(prm.stream, prm.mant, mode, syms, n,
+                                                                        prm.stream_bytes, prm.out, prm.out32);
     return cudaGetLastError() == cudaSuccess ? DFW_OK : DFW_ECUDA;
 }
 

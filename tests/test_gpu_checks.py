@@ -20,7 +20,7 @@ import torch
 pytestmark = pytest.mark.gpu
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SUITES = ["tests/test_gpu_decode.py", "tests/test_gpu_seq.py", "tests/test_gpu_rans.py",
+SUITES = ["tests/test_gpu_decode.py", "tests/test_gpu_closed.py", "tests/test_gpu_seq.py", "tests/test_gpu_rans.py",
           "tests/test_gpu_encode.py", "tests/test_gpu_encode_multi.py", "tests/test_gpu_gemv.py",
           "tests/test_gpu_failure.py"]
 
