@@ -278,3 +278,50 @@ def test_seq_alternating_scopes_end_with_the_last(scopes):
             dfw.decode_lanes_seq(order, got)
             dfw.check()
             assert torch.equal(got.view(torch.int16), want.view(torch.int16))
+
+
+def test_seq_random_mixes(oracle):
+    """Seeded random sequences of up to 45 scopes (so some take two launches):
+    Gaussian blocks, long-code and incompressible tensors, closed forms, one
+    exponent and empty scopes at random sizes, in random order with repeats.
+    Each must leave the buffer exactly as separate decodes in order do."""
+    rng = np.random.default_rng(2024)
+
+    def make(kind: str, n: int) -> np.ndarray:
+        r = np.random.default_rng(int(rng.integers(1 << 31)))
+        if kind == "gauss":
+            return np.concatenate([workloads.as_u16_numpy(t) for t in workloads.generate_block(
+                workloads.scaled(workloads.c5()[1], max(n, 7 * 64)), "cpu")])
+        if kind == "geometric":
+            return workloads.as_u16_numpy(workloads.generate_block(workloads.c4("b", max(n, 4096)))[0])
+        if kind == "uniform":
+            return r.integers(0, 65536, n, dtype=np.uint64).astype(np.uint16)
+        if kind == "bitmap":
+            e = np.where(r.integers(0, 2, n) == 1, 140, 139).astype(np.uint64)
+            return ((e << 7) | r.integers(0, 128, n).astype(np.uint64)).astype(np.uint16)
+        if kind == "single":
+            return ((r.integers(0, 2, n) << 15) | (118 << 7) | r.integers(0, 128, n)).astype(np.uint16)
+        return np.zeros(0, np.uint16)
+
+    kinds = ["gauss", "gauss", "geometric", "uniform", "bitmap", "single", "empty"]
+    pool = []
+    for i in range(12):
+        kind = kinds[i % len(kinds)]
+        u = make(kind, int(rng.integers(1, 300_000)))
+        enc = dfw.encode(u)
+        d = dfw.DeviceLanes.upload(enc, dfw.plan_lanes(enc), "cuda")
+        if kind == "empty":
+            d.mant = torch.zeros(16, dtype=torch.uint8, device="cuda")
+        pool.append((u, d))
+    nmax = max(u.size for u, _ in pool)
+    for trial in range(6):
+        k = int(rng.integers(2, 46))
+        order = [int(i) for i in rng.integers(0, len(pool), k)]
+        devs = [pool[i][1] for i in order]
+        got, want = _garbage(nmax), _garbage(nmax)
+        dfw.decode_lanes_seq(devs, got)
+        for d in devs:
+            if d.n:
+                dfw.decode_lanes(d, want)
+        dfw.check()
+        assert torch.equal(got.view(torch.int16), want.view(torch.int16)), f"trial {trial}: {order}"
